@@ -1,0 +1,186 @@
+/*
+ * bi.h -- C ABI of libbi.so: batch-invariant reduction kernels for NVIDIA B200 (sm_100a).
+ *
+ * A kernel is batch-invariant when the bits it returns for one row of its input
+ * do not depend on how many other rows share the call or where the row sits in
+ * the batch.  The source pages state the property and its cause: inference
+ * kernels such as matmul and RMSNorm reduce in an order shaped by the total
+ * batch size, so a row's last bits change with the batch (readhandoff.com,
+ * agent-run-reproducibility-pinning, "What does temperature zero actually
+ * guarantee?"); the remedy is that the same input always takes the same
+ * accumulation order (wiki.aimuse.me "Thinking Machines", batch-invariant
+ * kernel section; glasp.co "How to achieve deterministic LLMs with batch
+ * invariant inference", Key Insights), which rules out split-K and
+ * shape-aware tiling (wiki.aimuse.me "Thinking Machines", section on the loss
+ * of dynamic-batching optimisations).  The operations are those the public
+ * library replaces -- mm, addmm, log_softmax, mean (ross.abutalabs.com
+ * "thinking-machines-lab/batch_invariant_ops", "When to avoid") -- plus RMSNorm
+ * and the SiLU-times-up glue of a gated MLP.
+ *
+ * How each entry point fixes its order (the same for every M):
+ *   - bi_matmul / bi_addmm: one tcgen05/TMEM tile configuration fed by TMA for
+ *     every shape; every output element accumulates its K products in fp32,
+ *     16 at a time, in ascending K; no split-K, no stream-K, no tile switch.
+ *   - bi_rmsnorm / bi_mean / bi_log_softmax: one thread block per row; the
+ *     block size and each thread's element set depend only on the row length;
+ *     partial results merge through a fixed warp-shuffle tree and a fixed
+ *     cross-warp tree.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are row-major.  Pointers marked "device" point to global memory
+ *     of the current CUDA device; the caller allocates, owns and frees every
+ *     buffer.  The library allocates no device memory in any call.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous on that stream.  Argument errors are returned before anything
+ *     is launched; a launch failure returns BI_ERR_CUDA.
+ *   - M = 0 (no rows) is a no-op that returns BI_OK.
+ *   - Outputs must not overlap inputs.
+ *   - bf16 is IEEE-style bfloat16 (1-8-7); every bf16 output is rounded once,
+ *     to nearest-even, from an fp32 value.
+ *   - Every device-side wait is bounded; a wait that runs out records
+ *     BI_ERR_TIMEOUT in a per-device status word, the kernel releases what it
+ *     holds and returns.  Read it with bi_get_device_status.
+ */
+#ifndef BI_H
+#define BI_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BI_OK = 0,
+    BI_ERR_INVALID_ARG = 1,  /* null pointer, negative size, leading dim too small, bad enum */
+    BI_ERR_UNSUPPORTED = 2,  /* a size the kernels do not handle (e.g. > 2^31-1 rows)        */
+    BI_ERR_ALIGNMENT = 3,    /* base pointer or leading dimension breaks the 16-byte rule   */
+    BI_ERR_CUDA = 4,         /* a CUDA runtime/driver call or a launch failed                */
+    BI_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out (reported via the status) */
+} bi_status;
+
+typedef enum { BI_BF16 = 0, BI_F32 = 1 } bi_dtype;
+
+typedef enum {
+    BI_B_KN = 0, /* B stored [K, N] row-major: the right operand of torch.mm           */
+    BI_B_NK = 1  /* B stored [N, K] row-major: an nn.Linear weight (C = A . B^T)       */
+} bi_b_layout;
+
+/*
+ * bi_matmul -- C = A . B  (torch.mm; for BI_B_NK, torch.nn.functional.linear without bias).
+ * Passage: ross.abutalabs.com "thinking-machines-lab/batch_invariant_ops", "When to
+ * avoid" (mm is covered) and "Use cases" (matrix multiplication gives the same output
+ * for different batch sizes).
+ *
+ *   A  device, bf16, [M, K], leading dimension lda >= K (elements)
+ *   B  device, bf16, [K, N] with ldb >= N (BI_B_KN) or [N, K] with ldb >= K (BI_B_NK)
+ *   C  device, [M, N], leading dimension ldc >= N, element type c_dtype (BI_BF16 or BI_F32)
+ *   C[i][j] = round_{c_dtype}( sum_{k ascending} A[i][k] * B(k, j) ), products and sums in fp32.
+ *   K = 0 writes zeros.
+ * Alignment: A, B, C base addresses 16-byte aligned; lda, ldb multiples of 8 elements;
+ *   ldc a multiple of 8 (bf16) or 4 (f32) elements.  Otherwise BI_ERR_ALIGNMENT.
+ * Limits: M, N, K <= 2^31 - 1; otherwise BI_ERR_UNSUPPORTED.
+ */
+bi_status bi_matmul(const void *A, int64_t lda, const void *B, int64_t ldb, bi_b_layout b_layout,
+                    void *C, int64_t ldc, bi_dtype c_dtype, int64_t M, int64_t N, int64_t K,
+                    void *stream);
+
+/*
+ * bi_addmm -- C = input + A . B  (torch.addmm with alpha = beta = 1).
+ * Passage: ross.abutalabs.com "thinking-machines-lab/batch_invariant_ops", "When to
+ * avoid" (addmm is covered).
+ *
+ *   input  device, bf16.  ld_input == 0: a bias vector [N] added to every row.
+ *          ld_input >= N: a matrix [M, N] (e.g. a residual) with that leading dimension,
+ *          which must be a multiple of 8; base 16-byte aligned.
+ *   The input is widened to fp32 and added to the fp32 accumulator once, after the last
+ *   product, before the single rounding to c_dtype.  All else as bi_matmul.
+ */
+bi_status bi_addmm(const void *input, int64_t ld_input, const void *A, int64_t lda, const void *B,
+                   int64_t ldb, bi_b_layout b_layout, void *C, int64_t ldc, bi_dtype c_dtype,
+                   int64_t M, int64_t N, int64_t K, void *stream);
+
+/*
+ * bi_rmsnorm -- y = x * r * w,  r = 1 / sqrt( sum_j x_j^2 / H + eps ), per row.
+ * Passage: readhandoff.com agent-run-reproducibility-pinning, "What does temperature
+ * zero actually guarantee?" and the FAQ (RMSNorm is one of the kernels whose result
+ * depends on the batch by default).
+ *
+ *   x  device, bf16, [M, H] contiguous;  w device, bf16, [H];  y device, bf16, [M, H].
+ *   fp32 arithmetic inside; one rounding of (x * r) * w to bf16.  eps >= 0.
+ *   x, w, y 16-byte aligned when H is a multiple of 8 (the vector path), else any alignment.
+ */
+bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H, float eps,
+                     void *stream);
+
+/*
+ * bi_mean -- y_i = ( sum_j x_ij ) / H, per row (torch.mean over the last dimension).
+ * Passage: ross.abutalabs.com "thinking-machines-lab/batch_invariant_ops", "When to
+ * avoid" (mean is covered); trustbutveri.fyi "Evidence & limits", Evidence (SGLang
+ * integrated the mean kernel).
+ *
+ *   x  device, fp32, [M, H] contiguous;  y device, fp32, [M].
+ *   fp32 sum in a fixed tree, then one IEEE division by H.
+ *   x 16-byte aligned when H is a multiple of 4 (the vector path).
+ */
+bi_status bi_mean(const float *x, float *y, int64_t M, int64_t H, void *stream);
+
+/*
+ * bi_log_softmax -- y_j = (x_j - m) - log( sum_k exp(x_k - m) ),  m = max_k x_k, per row.
+ * Passage: ross.abutalabs.com "thinking-machines-lab/batch_invariant_ops", "When to
+ * avoid" (log_softmax is covered); trustbutveri.fyi "Evidence & limits", Evidence.
+ *
+ *   x  device, [M, V] contiguous, x_dtype BI_F32 or BI_BF16 (bf16 is widened exactly);
+ *   y  device, fp32, [M, V].
+ *   Per-thread running (max, sum) pairs merged through a fixed tree; the row is read
+ *   twice (once for the statistics, once to write y).
+ *   x and y 16-byte aligned when V is a multiple of 8 (bf16) / 4 (f32), the vector path.
+ */
+bi_status bi_log_softmax(const void *x, bi_dtype x_dtype, float *y, int64_t M, int64_t V,
+                         void *stream);
+
+/*
+ * bi_silu_mul -- h_ij = silu(g_ij) * u_ij with g = gu[:, 0:F], u = gu[:, F:2F],
+ * silu(g) = g / (1 + exp(-g)).  Elementwise glue of a gated MLP (no reduction, so
+ * batch-invariant by construction); not an operation the pages name.
+ *
+ *   gu device, bf16, [M, 2F] contiguous;  h device, bf16, [M, F].
+ *   fp32 inside, one rounding to bf16.  16-byte aligned when F is a multiple of 8.
+ */
+bi_status bi_silu_mul(const void *gu, void *h, int64_t M, int64_t F, void *stream);
+
+/*
+ * bi_get_device_status -- synchronise `stream`, then read and clear the current
+ * device's status word.  *out receives BI_OK or the first error a kernel recorded
+ * since the last read (BI_ERR_TIMEOUT for a bounded wait that ran out).
+ * Returns BI_ERR_CUDA if the synchronisation or the read fails.
+ */
+bi_status bi_get_device_status(void *stream, int32_t *out);
+
+/*
+ * bi_selftest_wait_timeout -- launch one block that waits on a shared-memory
+ * barrier nothing will complete, through the same bounded wait the GEMM uses,
+ * with the given limit (nanoseconds, 1000 .. 10^10).  The wait gives up, records
+ * BI_ERR_TIMEOUT in the status word and the kernel returns normally; the device
+ * context stays usable.  For testing the failure path without a GPU fault.
+ */
+bi_status bi_selftest_wait_timeout(int64_t limit_ns, void *stream);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *bi_status_string(bi_status status);
+
+/*
+ * bi_gemm_config -- report the single tile configuration every bi_matmul / bi_addmm
+ * call uses: output tile bm x bn, K-slice bk per pipeline stage, number of stages,
+ * and the K step of one tensor-core instruction.  Any pointer may be NULL.
+ */
+void bi_gemm_config(int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int32_t *mma_k);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t bi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BI_H */

@@ -1,0 +1,250 @@
+"""Python binding of libbi.so: the C ABI of include/bi.h, one function per entry point.
+
+Argument marshalling only.  Each function checks device, dtype and layout of the
+torch tensors it is given, allocates the output with torch when none is passed,
+and calls the C entry point of the same name with raw device pointers, leading
+dimensions and the current CUDA stream.  Every step of the computation runs in
+libbi.so's kernels; there is no fallback.  If libbi.so is missing or a call fails
+the function raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbi.so")
+
+BI_OK, BI_ERR_INVALID_ARG, BI_ERR_UNSUPPORTED, BI_ERR_ALIGNMENT, BI_ERR_CUDA, BI_ERR_TIMEOUT = range(6)
+BI_BF16, BI_F32 = 0, 1
+BI_B_KN, BI_B_NK = 0, 1
+
+# Every entry point declared in include/bi.h, with its ctypes signature.
+_i64, _p, _i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int32
+SIGNATURES = {
+    "bi_matmul": (ctypes.c_int, [_p, _i64, _p, _i64, ctypes.c_int, _p, _i64, ctypes.c_int,
+                                 _i64, _i64, _i64, _p]),
+    "bi_addmm": (ctypes.c_int, [_p, _i64, _p, _i64, _p, _i64, ctypes.c_int, _p, _i64, ctypes.c_int,
+                                _i64, _i64, _i64, _p]),
+    "bi_rmsnorm": (ctypes.c_int, [_p, _p, _p, _i64, _i64, ctypes.c_float, _p]),
+    "bi_mean": (ctypes.c_int, [_p, _p, _i64, _i64, _p]),
+    "bi_log_softmax": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p]),
+    "bi_silu_mul": (ctypes.c_int, [_p, _p, _i64, _i64, _p]),
+    "bi_get_device_status": (ctypes.c_int, [_p, ctypes.POINTER(_i32)]),
+    "bi_selftest_wait_timeout": (ctypes.c_int, [_i64, _p]),
+    "bi_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "bi_gemm_config": (None, [ctypes.POINTER(_i32)] * 5),
+    "bi_version": (ctypes.c_int32, []),
+}
+
+_lib = None
+
+
+class BiError(RuntimeError):
+    def __init__(self, name: str, status: int):
+        super().__init__(f"{name} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libbi.so (once) and attach the ctypes signatures."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"libbi.so not found at {path}: build it with __graft_entry__.build() or "
+                "invariant_bi_matmul_02_b200/csrc/build.py")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().bi_status_string(int(status)).decode()
+
+
+def _check(name: str, status: int):
+    if status != BI_OK:
+        raise BiError(name, status)
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _need_cuda(t: torch.Tensor, name: str, dtypes):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
+
+
+def _ld(t: torch.Tensor, name: str) -> int:
+    """Leading dimension of a 2-D tensor with unit-stride rows."""
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D")
+    if t.shape[1] > 1 and t.stride(1) != 1:
+        raise ValueError(f"{name} rows must be contiguous")
+    return t.stride(0) if t.shape[0] > 1 else max(t.stride(0), t.shape[1])
+
+
+def _contig(t: torch.Tensor, name: str):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+_DT = {torch.bfloat16: BI_BF16, torch.float32: BI_F32}
+
+
+def _gemm_shapes(a, b, b_layout):
+    if b_layout not in ("kn", "nk"):
+        raise ValueError("b_layout must be 'kn' ([K, N]) or 'nk' ([N, K])")
+    M, K = a.shape
+    if b_layout == "kn":
+        Kb, N = b.shape
+    else:
+        N, Kb = b.shape
+    if Kb != K:
+        raise ValueError(f"inner dimensions differ: A has K={K}, B has K={Kb}")
+    return M, N, K
+
+
+def bi_matmul(a: torch.Tensor, b: torch.Tensor, b_layout: str = "nk", out: torch.Tensor | None = None,
+              out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+    """C = A . B (b_layout 'kn': B [K, N]; 'nk': B [N, K], i.e. C = A . B^T)."""
+    _need_cuda(a, "A", (torch.bfloat16,))
+    _need_cuda(b, "B", (torch.bfloat16,))
+    M, N, K = _gemm_shapes(a, b, b_layout)
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    _need_cuda(out, "C", (torch.bfloat16, torch.float32))
+    if tuple(out.shape) != (M, N):
+        raise ValueError("C must be [M, N]")
+    st = load().bi_matmul(a.data_ptr(), _ld(a, "A"), b.data_ptr(), _ld(b, "B"),
+                          BI_B_KN if b_layout == "kn" else BI_B_NK, out.data_ptr(), _ld(out, "C"),
+                          _DT[out.dtype], M, N, K, _stream(stream))
+    _check("bi_matmul", st)
+    return out
+
+
+def bi_addmm(input: torch.Tensor, a: torch.Tensor, b: torch.Tensor, b_layout: str = "nk",
+             out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
+             stream=None) -> torch.Tensor:
+    """C = input + A . B; input is a bias [N] or a matrix [M, N] (bf16)."""
+    _need_cuda(a, "A", (torch.bfloat16,))
+    _need_cuda(b, "B", (torch.bfloat16,))
+    _need_cuda(input, "input", (torch.bfloat16,))
+    M, N, K = _gemm_shapes(a, b, b_layout)
+    if input.dim() == 1:
+        if input.shape[0] != N:
+            raise ValueError("bias must have N entries")
+        if input.stride(0) != 1:
+            raise ValueError("bias must be contiguous")
+        ld_in = 0
+    else:
+        if tuple(input.shape) != (M, N):
+            raise ValueError("input must be [N] or [M, N]")
+        ld_in = _ld(input, "input")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    _need_cuda(out, "C", (torch.bfloat16, torch.float32))
+    if tuple(out.shape) != (M, N):
+        raise ValueError("C must be [M, N]")
+    st = load().bi_addmm(input.data_ptr(), ld_in, a.data_ptr(), _ld(a, "A"), b.data_ptr(), _ld(b, "B"),
+                         BI_B_KN if b_layout == "kn" else BI_B_NK, out.data_ptr(), _ld(out, "C"),
+                         _DT[out.dtype], M, N, K, _stream(stream))
+    _check("bi_addmm", st)
+    return out
+
+
+def bi_rmsnorm(x: torch.Tensor, w: torch.Tensor, eps: float = 1e-6, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """y = x / sqrt(mean(x^2) + eps) * w over the last dimension (bf16)."""
+    _need_cuda(x, "x", (torch.bfloat16,))
+    _need_cuda(w, "w", (torch.bfloat16,))
+    _contig(x, "x")
+    _contig(w, "w")
+    M, H = x.shape
+    if tuple(w.shape) != (H,):
+        raise ValueError("w must be [H]")
+    if out is None:
+        out = torch.empty_like(x)
+    _need_cuda(out, "y", (torch.bfloat16,))
+    _contig(out, "y")
+    _check("bi_rmsnorm", load().bi_rmsnorm(x.data_ptr(), w.data_ptr(), out.data_ptr(), M, H,
+                                           float(eps), _stream(stream)))
+    return out
+
+
+def bi_mean(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y_i = mean_j x_ij (fp32)."""
+    _need_cuda(x, "x", (torch.float32,))
+    _contig(x, "x")
+    M, H = x.shape
+    if out is None:
+        out = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _need_cuda(out, "y", (torch.float32,))
+    _contig(out, "y")
+    _check("bi_mean", load().bi_mean(x.data_ptr(), out.data_ptr(), M, H, _stream(stream)))
+    return out
+
+
+def bi_log_softmax(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """log_softmax over the last dimension; x fp32 or bf16, y fp32."""
+    _need_cuda(x, "x", (torch.float32, torch.bfloat16))
+    _contig(x, "x")
+    M, V = x.shape
+    if out is None:
+        out = torch.empty((M, V), dtype=torch.float32, device=x.device)
+    _need_cuda(out, "y", (torch.float32,))
+    _contig(out, "y")
+    _check("bi_log_softmax", load().bi_log_softmax(x.data_ptr(), _DT[x.dtype], out.data_ptr(), M, V,
+                                                   _stream(stream)))
+    return out
+
+
+def bi_silu_mul(gu: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """h = silu(gu[:, :F]) * gu[:, F:] (bf16)."""
+    _need_cuda(gu, "gu", (torch.bfloat16,))
+    _contig(gu, "gu")
+    M, F2 = gu.shape
+    if F2 % 2:
+        raise ValueError("gu must have 2F columns")
+    F = F2 // 2
+    if out is None:
+        out = torch.empty((M, F), dtype=torch.bfloat16, device=gu.device)
+    _need_cuda(out, "h", (torch.bfloat16,))
+    _contig(out, "h")
+    _check("bi_silu_mul", load().bi_silu_mul(gu.data_ptr(), out.data_ptr(), M, F, _stream(stream)))
+    return out
+
+
+def bi_get_device_status(stream=None) -> int:
+    """Synchronise the stream, then read and clear the device status word."""
+    v = _i32(0)
+    _check("bi_get_device_status", load().bi_get_device_status(_stream(stream), ctypes.byref(v)))
+    return int(v.value)
+
+
+def bi_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    _check("bi_selftest_wait_timeout", load().bi_selftest_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+def bi_gemm_config() -> dict:
+    vals = [_i32(0) for _ in range(5)]
+    load().bi_gemm_config(*[ctypes.byref(v) for v in vals])
+    return dict(zip(("bm", "bn", "bk", "stages", "mma_k"), (int(v.value) for v in vals)))
+
+
+def bi_version() -> int:
+    return int(load().bi_version())

@@ -1,0 +1,356 @@
+// bi.cu -- host side of libbi.so: argument checks, TMA tensor-map encoding and
+// stream-ordered launches behind the C ABI declared in include/bi.h.
+//
+// The library allocates no device memory.  Per device it caches the SM count, the
+// address of its status word and the GEMM kernel's shared-memory attribute.  No
+// launch decision depends on M except the grid size (how many CTAs share the tile
+// list, or how many rows there are), which never changes a row's arithmetic.
+#include "bi.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "rowops.cuh"
+
+// Per-device status word: 0, or the first error a kernel recorded (BI_ERR_TIMEOUT).
+__device__ int32_t g_bi_status = 0;
+
+namespace {
+
+constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s per device-side wait
+constexpr int kMaxDevices = 64;
+constexpr int64_t kI32Max = 2147483647;
+
+struct DeviceState {
+    bool ready = false;
+    int sms = 0;
+    int32_t *status = nullptr;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bi_status device_state(DeviceState **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return BI_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState &d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return BI_ERR_CUDA;
+        void *sym = nullptr;
+        if (cudaGetSymbolAddress(&sym, g_bi_status) != cudaSuccess) return BI_ERR_CUDA;
+        d.status = static_cast<int32_t *>(sym);
+        if (cudaFuncSetAttribute(bi::gemm_bf16_tcgen05_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 bi::kGemmSmem) != cudaSuccess)
+            return BI_ERR_CUDA;
+        d.ready = true;
+    }
+    *out = &d;
+    return BI_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor map over a row-major matrix: `inner` contiguous elements per row,
+// `outer` rows `ld` elements apart, box inner x outer, 128-byte swizzle, zero fill.
+bi_status encode_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint64_t ld,
+                     uint32_t box_inner, uint32_t box_outer)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return BI_ERR_CUDA;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {ld * 2};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? BI_OK : BI_ERR_CUDA;
+}
+
+bi_status launched() { return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA; }
+
+bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, const void *A, int64_t lda,
+                      const void *B, int64_t ldb, int b_layout, void *C, int64_t ldc, int c_dtype,
+                      int64_t M, int64_t N, int64_t K, void *stream)
+{
+    if (M < 0 || N < 0 || K < 0) return BI_ERR_INVALID_ARG;
+    if (b_layout != BI_B_KN && b_layout != BI_B_NK) return BI_ERR_INVALID_ARG;
+    if (c_dtype != BI_BF16 && c_dtype != BI_F32) return BI_ERR_INVALID_ARG;
+    if (M > kI32Max || N > kI32Max || K > kI32Max) return BI_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return BI_OK;
+    if (!C || ldc < N) return BI_ERR_INVALID_ARG;
+    if (addend_mode != bi::kAddNone) {
+        if (!input || ld_input < 0 || (ld_input != 0 && ld_input < N)) return BI_ERR_INVALID_ARG;
+        if (!aligned16(input) || ld_input % 8 != 0) return BI_ERR_ALIGNMENT;
+    }
+    const bool c_f32 = c_dtype == BI_F32;
+    if (!aligned16(C) || ldc % (c_f32 ? 4 : 8) != 0) return BI_ERR_ALIGNMENT;
+    if (K > 0) {
+        if (!A || !B) return BI_ERR_INVALID_ARG;
+        if (lda < K || ldb < (b_layout == BI_B_KN ? N : K)) return BI_ERR_INVALID_ARG;
+        if (!aligned16(A) || !aligned16(B) || lda % 8 != 0 || ldb % 8 != 0) return BI_ERR_ALIGNMENT;
+    }
+
+    DeviceState *dev = nullptr;
+    bi_status st = device_state(&dev);
+    if (st != BI_OK) return st;
+
+    bi::GemmParams p{};
+    p.M = (int32_t)M;
+    p.N = (int32_t)N;
+    p.K = (int32_t)K;
+    p.m_blocks = (int32_t)((M + bi::kBM - 1) / bi::kBM);
+    p.n_blocks = (int32_t)((N + bi::kBN - 1) / bi::kBN);
+    p.k_blocks = (int32_t)((K + bi::kBK - 1) / bi::kBK);
+    p.b_mn_major = b_layout == BI_B_KN ? 1 : 0;
+    p.c_f32 = c_f32 ? 1 : 0;
+    p.addend_mode = addend_mode;
+    p.ldc = ldc;
+    p.ld_addend = ld_input;
+    p.C = C;
+    p.addend = static_cast<const __nv_bfloat16 *>(input);
+    p.status = dev->status;
+    p.wait_limit_ns = kWaitLimitNs;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    if (K == 0) {
+        const int64_t total = M * N;
+        int64_t blocks = (total + 255) / 256;
+        if (blocks > (int64_t)dev->sms * 16) blocks = (int64_t)dev->sms * 16;
+        bi::gemm_k0_fill_kernel<<<(unsigned)blocks, 256, 0, s>>>(p);
+        return launched();
+    }
+
+    const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
+    if (tiles > kI32Max) return BI_ERR_UNSUPPORTED;
+
+    CUtensorMap tm_a, tm_b;
+    st = encode_map(&tm_a, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda, bi::kBK, bi::kBM);
+    if (st != BI_OK) return st;
+    if (b_layout == BI_B_NK)
+        st = encode_map(&tm_b, B, (uint64_t)K, (uint64_t)N, (uint64_t)ldb, bi::kBK, bi::kBN);
+    else
+        st = encode_map(&tm_b, B, (uint64_t)N, (uint64_t)K, (uint64_t)ldb, 64, bi::kBK);
+    if (st != BI_OK) return st;
+
+    const int grid = (int)(tiles < dev->sms ? tiles : dev->sms);
+    bi::gemm_bf16_tcgen05_kernel<<<grid, bi::kGemmThreads, bi::kGemmSmem, s>>>(tm_a, tm_b, p);
+    return launched();
+}
+
+__global__ void selftest_wait_kernel(int32_t *status, uint64_t limit_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        bi::mbar_init(&bar, 1);
+        abort_flag = 0;
+        bi::fence_mbar_init();
+    }
+    __syncthreads();
+    // Phase 0 of `bar` never completes: nothing arrives on it.
+    if (threadIdx.x == 0) bi::wait_bounded(&bar, 0, &abort_flag, status, limit_ns);
+    __syncthreads();
+}
+
+inline unsigned elementwise_blocks(int64_t work, int sms)
+{
+    int64_t blocks = (work + 255) / 256;
+    const int64_t cap = (int64_t)sms * 8;
+    return (unsigned)(blocks < 1 ? 1 : (blocks > cap ? cap : blocks));
+}
+
+}  // namespace
+
+extern "C" {
+
+bi_status bi_matmul(const void *A, int64_t lda, const void *B, int64_t ldb, bi_b_layout b_layout,
+                    void *C, int64_t ldc, bi_dtype c_dtype, int64_t M, int64_t N, int64_t K,
+                    void *stream)
+{
+    return gemm_common(nullptr, 0, bi::kAddNone, A, lda, B, ldb, b_layout, C, ldc, c_dtype, M, N, K,
+                       stream);
+}
+
+bi_status bi_addmm(const void *input, int64_t ld_input, const void *A, int64_t lda, const void *B,
+                   int64_t ldb, bi_b_layout b_layout, void *C, int64_t ldc, bi_dtype c_dtype,
+                   int64_t M, int64_t N, int64_t K, void *stream)
+{
+    return gemm_common(input, ld_input, ld_input == 0 ? bi::kAddBias : bi::kAddMatrix, A, lda, B, ldb,
+                       b_layout, C, ldc, c_dtype, M, N, K, stream);
+}
+
+bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H, float eps,
+                     void *stream)
+{
+    if (M < 0 || H < 0 || !(eps >= 0.0f)) return BI_ERR_INVALID_ARG;
+    if (M > kI32Max || H > kI32Max) return BI_ERR_UNSUPPORTED;
+    if (M == 0) return BI_OK;
+    if (H == 0 || !x || !w || !y) return BI_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int T = bi::rmsnorm_threads(H);
+    if (H % 8 == 0) {
+        if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return BI_ERR_ALIGNMENT;
+        const int64_t cpt = (H / 8 + T - 1) / T;
+        const uint4 *xv = static_cast<const uint4 *>(x);
+        const uint4 *wv = static_cast<const uint4 *>(w);
+        uint4 *yv = static_cast<uint4 *>(y);
+        switch (cpt) {
+        case 1: bi::rmsnorm_vec_kernel<1><<<(unsigned)M, T, 0, s>>>(xv, wv, yv, H, eps); break;
+        case 2: bi::rmsnorm_vec_kernel<2><<<(unsigned)M, T, 0, s>>>(xv, wv, yv, H, eps); break;
+        case 3: bi::rmsnorm_vec_kernel<3><<<(unsigned)M, T, 0, s>>>(xv, wv, yv, H, eps); break;
+        case 4: bi::rmsnorm_vec_kernel<4><<<(unsigned)M, T, 0, s>>>(xv, wv, yv, H, eps); break;
+        default:
+            bi::rmsnorm_scalar_kernel<<<(unsigned)M, T, 0, s>>>(
+                static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w),
+                static_cast<__nv_bfloat16 *>(y), H, eps);
+        }
+    } else {
+        bi::rmsnorm_scalar_kernel<<<(unsigned)M, T, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w),
+            static_cast<__nv_bfloat16 *>(y), H, eps);
+    }
+    return launched();
+}
+
+bi_status bi_mean(const float *x, float *y, int64_t M, int64_t H, void *stream)
+{
+    if (M < 0 || H < 0) return BI_ERR_INVALID_ARG;
+    if (M > kI32Max || H > kI32Max) return BI_ERR_UNSUPPORTED;
+    if (M == 0) return BI_OK;
+    if (H == 0 || !x || !y) return BI_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int T = bi::mean_threads(H);
+    if (H % 4 == 0) {
+        if (!aligned16(x)) return BI_ERR_ALIGNMENT;
+        bi::mean_vec_kernel<<<(unsigned)M, T, 0, s>>>(reinterpret_cast<const float4 *>(x), y, H);
+    } else {
+        bi::mean_scalar_kernel<<<(unsigned)M, T, 0, s>>>(x, y, H);
+    }
+    return launched();
+}
+
+bi_status bi_log_softmax(const void *x, bi_dtype x_dtype, float *y, int64_t M, int64_t V, void *stream)
+{
+    if (M < 0 || V < 0) return BI_ERR_INVALID_ARG;
+    if (x_dtype != BI_BF16 && x_dtype != BI_F32) return BI_ERR_INVALID_ARG;
+    if (M > kI32Max || V > kI32Max) return BI_ERR_UNSUPPORTED;
+    if (M == 0) return BI_OK;
+    if (V == 0 || !x || !y) return BI_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int T = bi::log_softmax_threads(V);
+    const bool bf16 = x_dtype == BI_BF16;
+    const int per = bf16 ? 8 : 4;
+    if (V % per == 0) {
+        if (!aligned16(x) || !aligned16(y)) return BI_ERR_ALIGNMENT;
+        const uint4 *xv = static_cast<const uint4 *>(x);
+        float4 *yv = reinterpret_cast<float4 *>(y);
+        if (bf16)
+            bi::log_softmax_vec_kernel<true><<<(unsigned)M, T, 0, s>>>(xv, yv, V);
+        else
+            bi::log_softmax_vec_kernel<false><<<(unsigned)M, T, 0, s>>>(xv, yv, V);
+    } else {
+        if (bf16)
+            bi::log_softmax_scalar_kernel<true><<<(unsigned)M, T, 0, s>>>(x, y, V);
+        else
+            bi::log_softmax_scalar_kernel<false><<<(unsigned)M, T, 0, s>>>(x, y, V);
+    }
+    return launched();
+}
+
+bi_status bi_silu_mul(const void *gu, void *h, int64_t M, int64_t F, void *stream)
+{
+    if (M < 0 || F < 0) return BI_ERR_INVALID_ARG;
+    if (M > kI32Max || F > kI32Max) return BI_ERR_UNSUPPORTED;
+    if (M == 0 || F == 0) return BI_OK;
+    if (!gu || !h) return BI_ERR_INVALID_ARG;
+    DeviceState *dev = nullptr;
+    bi_status st = device_state(&dev);
+    if (st != BI_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (F % 8 == 0) {
+        if (!aligned16(gu) || !aligned16(h)) return BI_ERR_ALIGNMENT;
+        const int64_t work = M * (F / 8);
+        bi::silu_mul_vec_kernel<<<elementwise_blocks(work, dev->sms), 256, 0, s>>>(
+            static_cast<const uint4 *>(gu), static_cast<uint4 *>(h), M, F);
+    } else {
+        bi::silu_mul_scalar_kernel<<<elementwise_blocks(M * F, dev->sms), 256, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(gu), static_cast<__nv_bfloat16 *>(h), M, F);
+    }
+    return launched();
+}
+
+bi_status bi_get_device_status(void *stream, int32_t *out)
+{
+    if (!out) return BI_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return BI_ERR_CUDA;
+    int32_t v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_bi_status, sizeof v) != cudaSuccess) return BI_ERR_CUDA;
+    const int32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_bi_status, &zero, sizeof zero) != cudaSuccess) return BI_ERR_CUDA;
+    *out = v;
+    return BI_OK;
+}
+
+bi_status bi_selftest_wait_timeout(int64_t limit_ns, void *stream)
+{
+    if (limit_ns < 1000 || limit_ns > 10000000000ll) return BI_ERR_INVALID_ARG;
+    DeviceState *dev = nullptr;
+    bi_status st = device_state(&dev);
+    if (st != BI_OK) return st;
+    selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev->status,
+                                                                          (uint64_t)limit_ns);
+    return launched();
+}
+
+const char *bi_status_string(bi_status status)
+{
+    switch (status) {
+    case BI_OK: return "BI_OK";
+    case BI_ERR_INVALID_ARG: return "BI_ERR_INVALID_ARG";
+    case BI_ERR_UNSUPPORTED: return "BI_ERR_UNSUPPORTED";
+    case BI_ERR_ALIGNMENT: return "BI_ERR_ALIGNMENT";
+    case BI_ERR_CUDA: return "BI_ERR_CUDA";
+    case BI_ERR_TIMEOUT: return "BI_ERR_TIMEOUT";
+    }
+    return "BI_ERR_UNKNOWN";
+}
+
+void bi_gemm_config(int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int32_t *mma_k)
+{
+    if (bm) *bm = bi::kBM;
+    if (bn) *bn = bi::kBN;
+    if (bk) *bk = bi::kBK;
+    if (stages) *stages = bi::kStages;
+    if (mma_k) *mma_k = bi::kMmaK;
+}
+
+int32_t bi_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,379 @@
+// rowops.cuh -- one-block-per-row reductions (RMSNorm, mean, log_softmax) and the
+// elementwise SiLU-times-up glue.
+//
+// Batch invariance: a row is reduced by one thread block whose size, and whose
+// assignment of elements to threads, depend only on the row length.  Each thread
+// folds its elements in a fixed sequence; the per-thread partials meet in a fixed
+// xor-butterfly over the warp and then a fixed butterfly over the warp partials.
+// Nothing in a row's arithmetic depends on M, on the block's index or on timing, and
+// no atomics are used.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace bi {
+
+#define kNegInf (-__builtin_huge_valf())
+
+// --------------------------------------------------------------- fixed-order trees
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Sum over the block; every thread returns the same bits.  `red` holds >= 32 floats.
+__device__ __forceinline__ float block_sum(float v, float *red)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    v = warp_sum(v);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float t = lane < nwarps ? red[lane] : 0.0f;
+    t = warp_sum(t);
+    __syncthreads();  // `red` may be reused by the caller
+    return t;
+}
+
+// (max, sum of exp(x - max)) pairs.  The merge is symmetric in its two arguments
+// (no contracted multiply-adds), so both lanes of a butterfly pair hold equal bits.
+struct MaxSum {
+    float m, s;
+};
+
+__device__ __forceinline__ MaxSum merge(MaxSum a, MaxSum b)
+{
+    const float m = fmaxf(a.m, b.m);
+    if (m == kNegInf) return {m, 0.0f};
+    const float s = __fadd_rn(__fmul_rn(a.s, __expf(a.m - m)), __fmul_rn(b.s, __expf(b.m - m)));
+    return {m, s};
+}
+
+__device__ __forceinline__ MaxSum warp_merge(MaxSum v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        MaxSum w{__shfl_xor_sync(0xffffffffu, v.m, o), __shfl_xor_sync(0xffffffffu, v.s, o)};
+        v = merge(v, w);
+    }
+    return v;
+}
+
+__device__ __forceinline__ MaxSum block_merge(MaxSum v, float *red_m, float *red_s)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    v = warp_merge(v);
+    if (lane == 0) {
+        red_m[warp] = v.m;
+        red_s[warp] = v.s;
+    }
+    __syncthreads();
+    MaxSum t = lane < nwarps ? MaxSum{red_m[lane], red_s[lane]} : MaxSum{kNegInf, 0.0f};
+    t = warp_merge(t);
+    __syncthreads();
+    return t;
+}
+
+// Running (max, sum) update with a group of values already reduced to their max `gm`.
+__device__ __forceinline__ void rescale_to(MaxSum &acc, float gm)
+{
+    if (gm > acc.m) {
+        acc.s = acc.m == kNegInf ? 0.0f : acc.s * __expf(acc.m - gm);
+        acc.m = gm;
+    }
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&p);
+}
+
+// --------------------------------------------------------------- block-size rules
+// Functions of the row length only.
+
+__host__ __device__ inline int round_up32(long long v) { return (int)((v + 31) / 32 * 32); }
+
+__host__ __device__ inline int clamp_threads(long long v)
+{
+    int t = round_up32(v);
+    return t < 32 ? 32 : (t > 1024 ? 1024 : t);
+}
+
+// RMSNorm, bf16 rows: aim for two 16-byte chunks per thread.
+__host__ inline int rmsnorm_threads(long long H) { return clamp_threads((H / 8 + 1) / 2); }
+// mean, fp32 rows: aim for four 16-byte chunks per thread.
+__host__ inline int mean_threads(long long H) { return clamp_threads((H / 4 + 3) / 4); }
+// log_softmax: long rows, a full block.
+__host__ inline int log_softmax_threads(long long V) { return clamp_threads((V + 7) / 8); }
+
+// --------------------------------------------------------------- RMSNorm
+
+// Vector path: H % 8 == 0, row held in registers as CPT 16-byte chunks per thread.
+// Chunk c of a row belongs to thread c % T, as its (c / T)-th chunk.
+template <int CPT>
+__global__ void __launch_bounds__(1024) rmsnorm_vec_kernel(const uint4 *__restrict__ x,
+                                                          const uint4 *__restrict__ w,
+                                                          uint4 *__restrict__ y, int64_t H,
+                                                          float eps)
+{
+    __shared__ float red[32];
+    const int64_t nch = H / 8;
+    const int T = blockDim.x;
+    const uint4 *xr = x + (int64_t)blockIdx.x * nch;
+    uint4 *yr = y + (int64_t)blockIdx.x * nch;
+
+    uint4 v[CPT];
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int64_t c = threadIdx.x + (int64_t)i * T;
+        v[i] = c < nch ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const uint32_t q[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float a = bf16lo(q[k]), b = bf16hi(q[k]);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+        }
+    }
+    ss = block_sum(ss, red);
+    const float r = rsqrtf(ss / (float)H + eps);
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int64_t c = threadIdx.x + (int64_t)i * T;
+        if (c < nch) {
+            const uint4 wv = __ldg(w + c);
+            const uint32_t q[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+            const uint32_t g[4] = {wv.x, wv.y, wv.z, wv.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                o[k] = pack_bf16x2(__fmul_rn(__fmul_rn(bf16lo(q[k]), r), bf16lo(g[k])),
+                                   __fmul_rn(__fmul_rn(bf16hi(q[k]), r), bf16hi(g[k])));
+            yr[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+// Scalar path for any H: element j belongs to thread j % T; the row is read twice.
+__global__ void __launch_bounds__(1024) rmsnorm_scalar_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                             const __nv_bfloat16 *__restrict__ w,
+                                                             __nv_bfloat16 *__restrict__ y,
+                                                             int64_t H, float eps)
+{
+    __shared__ float red[32];
+    const __nv_bfloat16 *xr = x + (int64_t)blockIdx.x * H;
+    __nv_bfloat16 *yr = y + (int64_t)blockIdx.x * H;
+    float ss = 0.0f;
+    for (int64_t j = threadIdx.x; j < H; j += blockDim.x) {
+        const float a = __bfloat162float(xr[j]);
+        ss = fmaf(a, a, ss);
+    }
+    ss = block_sum(ss, red);
+    const float r = rsqrtf(ss / (float)H + eps);
+    for (int64_t j = threadIdx.x; j < H; j += blockDim.x)
+        yr[j] = __float2bfloat16_rn(
+            __fmul_rn(__fmul_rn(__bfloat162float(xr[j]), r), __bfloat162float(w[j])));
+}
+
+// --------------------------------------------------------------- mean
+
+// Vector path: H % 4 == 0.  Chunk c (4 floats) belongs to thread c % T; each thread
+// keeps four running sums (one per float4 lane) and folds them as (s0+s1)+(s2+s3).
+__global__ void __launch_bounds__(1024) mean_vec_kernel(const float4 *__restrict__ x,
+                                                       float *__restrict__ y, int64_t H)
+{
+    __shared__ float red[32];
+    const int64_t nch = H / 4;
+    const float4 *xr = x + (int64_t)blockIdx.x * nch;
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    int64_t c = threadIdx.x;
+    const int T = blockDim.x;
+    for (; c + 3 * (int64_t)T < nch; c += 4 * (int64_t)T) {
+        float4 a = __ldg(xr + c), b = __ldg(xr + c + T), d = __ldg(xr + c + 2 * T),
+               e = __ldg(xr + c + 3 * T);
+        s0 += a.x; s1 += a.y; s2 += a.z; s3 += a.w;
+        s0 += b.x; s1 += b.y; s2 += b.z; s3 += b.w;
+        s0 += d.x; s1 += d.y; s2 += d.z; s3 += d.w;
+        s0 += e.x; s1 += e.y; s2 += e.z; s3 += e.w;
+    }
+    for (; c < nch; c += T) {
+        float4 a = __ldg(xr + c);
+        s0 += a.x; s1 += a.y; s2 += a.z; s3 += a.w;
+    }
+    float s = __fadd_rn(__fadd_rn(s0, s1), __fadd_rn(s2, s3));
+    s = block_sum(s, red);
+    if (threadIdx.x == 0) y[blockIdx.x] = s / (float)H;
+}
+
+__global__ void __launch_bounds__(1024) mean_scalar_kernel(const float *__restrict__ x,
+                                                          float *__restrict__ y, int64_t H)
+{
+    __shared__ float red[32];
+    const float *xr = x + (int64_t)blockIdx.x * H;
+    float s = 0.f;
+    for (int64_t j = threadIdx.x; j < H; j += blockDim.x) s += xr[j];
+    s = block_sum(s, red);
+    if (threadIdx.x == 0) y[blockIdx.x] = s / (float)H;
+}
+
+// --------------------------------------------------------------- log_softmax
+
+template <bool BF16>
+struct LsmTraits;
+
+template <>
+struct LsmTraits<true> {  // 8 bf16 per 16-byte chunk
+    static constexpr int kPer = 8;
+    __device__ static void unpack(const uint4 &u, float (&v)[8])
+    {
+        v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+        v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+    }
+};
+
+template <>
+struct LsmTraits<false> {  // 4 fp32 per 16-byte chunk
+    static constexpr int kPer = 4;
+    __device__ static void unpack(const uint4 &u, float (&v)[4])
+    {
+        v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+        v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+    }
+};
+
+template <int P>
+__device__ __forceinline__ void lsm_accumulate(MaxSum &acc, const float (&v)[P])
+{
+    float gm = v[0];
+#pragma unroll
+    for (int k = 1; k < P; ++k) gm = fmaxf(gm, v[k]);
+    rescale_to(acc, gm);
+    if (acc.m != kNegInf) {
+#pragma unroll
+        for (int k = 0; k < P; ++k) acc.s += __expf(v[k] - acc.m);
+    }
+}
+
+// Vector path (V a multiple of the chunk width).  Chunk c belongs to thread c % T and
+// is visited in increasing c.  Pass 1 builds the row's (max, sum); pass 2 re-reads the
+// row and writes y = (x - max) - log(sum) as fp32.
+template <bool BF16>
+__global__ void __launch_bounds__(1024, 1) log_softmax_vec_kernel(const uint4 *__restrict__ x,
+                                                                 float4 *__restrict__ y,
+                                                                 int64_t V)
+{
+    __shared__ float red_m[32], red_s[32];
+    constexpr int P = LsmTraits<BF16>::kPer;
+    const int64_t nch = V / P;
+    const int T = blockDim.x;
+    const uint4 *xr = x + (int64_t)blockIdx.x * nch;
+
+    MaxSum acc{kNegInf, 0.0f};
+    int64_t c = threadIdx.x;
+    for (; c + 3 * (int64_t)T < nch; c += 4 * (int64_t)T) {
+        const uint4 u0 = __ldg(xr + c), u1 = __ldg(xr + c + T), u2 = __ldg(xr + c + 2 * T),
+                    u3 = __ldg(xr + c + 3 * T);
+        float v[P];
+        LsmTraits<BF16>::unpack(u0, v); lsm_accumulate(acc, v);
+        LsmTraits<BF16>::unpack(u1, v); lsm_accumulate(acc, v);
+        LsmTraits<BF16>::unpack(u2, v); lsm_accumulate(acc, v);
+        LsmTraits<BF16>::unpack(u3, v); lsm_accumulate(acc, v);
+    }
+    for (; c < nch; c += T) {
+        float v[P];
+        LsmTraits<BF16>::unpack(__ldg(xr + c), v);
+        lsm_accumulate(acc, v);
+    }
+    const MaxSum row = block_merge(acc, red_m, red_s);
+    const float m = row.m, ls = __logf(row.s);
+
+    float4 *yr = y + (int64_t)blockIdx.x * (V / 4);
+    for (int64_t c2 = threadIdx.x; c2 < nch; c2 += T) {
+        float v[P];
+        LsmTraits<BF16>::unpack(__ldg(xr + c2), v);
+#pragma unroll
+        for (int k = 0; k < P; k += 4)
+            __stcs(yr + c2 * (P / 4) + k / 4,
+                   make_float4((v[k] - m) - ls, (v[k + 1] - m) - ls, (v[k + 2] - m) - ls,
+                               (v[k + 3] - m) - ls));
+    }
+}
+
+// Scalar path for any V: element j belongs to thread j % T.
+template <bool BF16>
+__global__ void __launch_bounds__(1024, 1) log_softmax_scalar_kernel(const void *__restrict__ xv,
+                                                                    float *__restrict__ y,
+                                                                    int64_t V)
+{
+    __shared__ float red_m[32], red_s[32];
+    const int64_t base = (int64_t)blockIdx.x * V;
+    auto load = [&](int64_t j) -> float {
+        if (BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(xv)[base + j]);
+        return reinterpret_cast<const float *>(xv)[base + j];
+    };
+    MaxSum acc{kNegInf, 0.0f};
+    for (int64_t j = threadIdx.x; j < V; j += blockDim.x) {
+        float v[1] = {load(j)};
+        lsm_accumulate(acc, v);
+    }
+    const MaxSum row = block_merge(acc, red_m, red_s);
+    const float m = row.m, ls = __logf(row.s);
+    for (int64_t j = threadIdx.x; j < V; j += blockDim.x) y[base + j] = (load(j) - m) - ls;
+}
+
+// --------------------------------------------------------------- SiLU * up
+
+__device__ __forceinline__ float silu_mul1(float g, float u)
+{
+    return __fmul_rn(g / (1.0f + __expf(-g)), u);
+}
+
+// F % 8 == 0: thread handles 8 outputs (one 16-byte chunk of h) per step.
+__global__ void __launch_bounds__(256) silu_mul_vec_kernel(const uint4 *__restrict__ gu,
+                                                          uint4 *__restrict__ h, int64_t M,
+                                                          int64_t F)
+{
+    const int64_t fch = F / 8;
+    const int64_t total = M * fch;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = e / fch, c = e % fch;
+        const uint4 g = __ldg(gu + i * 2 * fch + c);
+        const uint4 u = __ldg(gu + i * 2 * fch + fch + c);
+        const uint32_t gq[4] = {g.x, g.y, g.z, g.w}, uq[4] = {u.x, u.y, u.z, u.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            o[k] = pack_bf16x2(silu_mul1(bf16lo(gq[k]), bf16lo(uq[k])),
+                               silu_mul1(bf16hi(gq[k]), bf16hi(uq[k])));
+        h[e] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+__global__ void __launch_bounds__(256) silu_mul_scalar_kernel(const __nv_bfloat16 *__restrict__ gu,
+                                                             __nv_bfloat16 *__restrict__ h,
+                                                             int64_t M, int64_t F)
+{
+    const int64_t total = M * F;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = e / F, j = e % F;
+        h[e] = __float2bfloat16_rn(silu_mul1(__bfloat162float(gu[i * 2 * F + j]),
+                                             __bfloat162float(gu[i * 2 * F + F + j])));
+    }
+}
+
+}  // namespace bi

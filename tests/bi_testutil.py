@@ -1,0 +1,75 @@
+"""Helpers shared by the GPU parity and invariance tests.
+
+Tolerances (written here once, used by every parity test):
+* bf16 outputs:        |gpu - ref| <= 2^-7 |ref| + 1e-3
+* fp32 log_softmax:    |gpu - ref| <= 1e-4
+* fp32 mean:           |gpu - ref| <= (ceil(log2 H) + 2) 2^-24 sum|x| / H + 2^-24 |ref|
+  (the error bound of a tree-shaped fp32 sum of depth ceil(log2 H) + 2, then one
+  correctly rounded division)
+"""
+import math
+
+import numpy as np
+import torch
+
+from invariant_bi_matmul_02_b200 import inputs
+
+BF16_REL = 2.0 ** -7
+BF16_ABS = 1e-3
+LSM_ABS = 1e-4
+U32 = 2.0 ** -24
+
+
+def to_np64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def assert_bf16_close(gpu: torch.Tensor, ref: np.ndarray, what: str = ""):
+    g = to_np64(gpu)
+    err = np.abs(g - ref)
+    bound = BF16_REL * np.abs(ref) + BF16_ABS
+    bad = err > bound
+    if bad.any():
+        idx = np.argwhere(bad)[0]
+        raise AssertionError(
+            f"{what}: {int(bad.sum())} of {bad.size} entries out of tolerance; first at {tuple(idx)}: "
+            f"gpu={g[tuple(idx)]!r} ref={ref[tuple(idx)]!r}")
+
+
+def assert_lsm_close(gpu: torch.Tensor, ref: np.ndarray, what: str = ""):
+    g = to_np64(gpu)
+    err = np.abs(g - ref)
+    worst = float(err.max()) if err.size else 0.0
+    assert worst <= LSM_ABS, f"{what}: max |err| {worst} > {LSM_ABS}"
+
+
+def assert_mean_close(gpu: torch.Tensor, ref: np.ndarray, x: np.ndarray, what: str = ""):
+    H = x.shape[1]
+    g = to_np64(gpu)
+    depth = math.ceil(math.log2(max(H, 2))) + 2
+    bound = depth * U32 * np.abs(x.astype(np.float64)).sum(axis=1) / H + U32 * np.abs(ref)
+    err = np.abs(g - ref)
+    assert np.all(err <= bound), f"{what}: worst excess {float((err - bound).max())}"
+
+
+def bits16(t: torch.Tensor) -> torch.Tensor:
+    return t.contiguous().view(torch.int16)
+
+
+def bits32(t: torch.Tensor) -> torch.Tensor:
+    return t.contiguous().view(torch.int32)
+
+
+def same_bits(a: torch.Tensor, b: torch.Tensor) -> bool:
+    if a.dtype != b.dtype or a.shape != b.shape:
+        return False
+    view = bits16 if a.element_size() == 2 else bits32
+    return bool(torch.equal(view(a), view(b)))
+
+
+def bf16_bits_np(t: torch.Tensor) -> np.ndarray:
+    return inputs.bf16_bits(t)
+
+
+# The M values of the GEMM sweep (powers of two up to 2048 plus the odd sizes).
+M_SWEEP = [1, 2, 3, 4, 8, 16, 32, 64, 77, 128, 256, 512, 1000, 1024, 2048]

@@ -1,0 +1,106 @@
+"""CPU-only checks of the C ABI: libbi.so loads, exports every entry point the header
+declares, and rejects bad arguments on the host before touching a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from invariant_bi_matmul_02_b200 import binding
+from invariant_bi_matmul_02_b200.csrc import build as libbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bi.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bi_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    libbuild.build()
+    return binding.load()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("bi_matmul", "bi_addmm", "bi_rmsnorm", "bi_mean", "bi_log_softmax", "bi_silu_mul",
+              "bi_get_device_status", "bi_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/bi.h but not exported"
+    assert set(declared_functions()) == set(binding.SIGNATURES), "binding and header disagree"
+
+
+def test_status_strings_and_config(lib):
+    assert binding.status_string(binding.BI_OK) == "BI_OK"
+    assert binding.status_string(binding.BI_ERR_TIMEOUT) == "BI_ERR_TIMEOUT"
+    assert binding.status_string(99) == "BI_ERR_UNKNOWN"
+    cfg = binding.bi_gemm_config()
+    assert cfg["bm"] == 128 and cfg["bk"] == 64 and cfg["mma_k"] == 16
+    assert cfg["bn"] in (64, 128, 192, 256) and cfg["stages"] >= 2
+    assert binding.bi_version() >= 100
+
+
+NULL = None
+
+
+def test_host_validation_without_a_gpu(lib):
+    I = binding.BI_ERR_INVALID_ARG
+    U = binding.BI_ERR_UNSUPPORTED
+    A = binding.BI_ERR_ALIGNMENT
+    # negative sizes, bad enums, null pointers
+    assert lib.bi_matmul(NULL, 8, NULL, 8, 1, NULL, 8, 0, -1, 8, 8, NULL) == I
+    assert lib.bi_matmul(NULL, 8, NULL, 8, 7, NULL, 8, 0, 1, 8, 8, NULL) == I
+    assert lib.bi_matmul(NULL, 8, NULL, 8, 1, NULL, 8, 5, 1, 8, 8, NULL) == I
+    assert lib.bi_matmul(NULL, 8, NULL, 8, 1, NULL, 8, 0, 1, 8, 8, NULL) == I
+    assert lib.bi_matmul(NULL, 8, NULL, 8, 1, NULL, 8, 0, 1 << 31, 8, 8, NULL) == U
+    # leading dimension too small, misaligned pointers / leading dims
+    fake = 0x10000
+    assert lib.bi_matmul(fake, 4, fake, 8, 1, fake, 8, 0, 2, 8, 8, NULL) == I
+    assert lib.bi_matmul(fake + 2, 8, fake, 8, 1, fake, 8, 0, 2, 8, 8, NULL) == A
+    assert lib.bi_matmul(fake, 12, fake, 8, 1, fake, 8, 0, 2, 8, 8, NULL) == A
+    assert lib.bi_matmul(fake, 8, fake, 8, 1, fake, 12, 0, 2, 8, 8, NULL) == A
+    assert lib.bi_addmm(NULL, 0, fake, 8, fake, 8, 1, fake, 8, 0, 2, 8, 8, NULL) == I
+    assert lib.bi_addmm(fake, 4, fake, 8, fake, 8, 1, fake, 8, 0, 2, 8, 8, NULL) == I
+    # M = 0 is a no-op that succeeds without a device
+    assert lib.bi_matmul(NULL, 8, NULL, 8, 1, NULL, 8, 0, 0, 8, 8, NULL) == binding.BI_OK
+    assert lib.bi_rmsnorm(NULL, NULL, NULL, 0, 8, ctypes.c_float(1e-6), NULL) == binding.BI_OK
+    # row ops
+    assert lib.bi_rmsnorm(NULL, NULL, NULL, 2, 8, ctypes.c_float(1e-6), NULL) == I
+    assert lib.bi_rmsnorm(fake, fake, fake, 2, 8, ctypes.c_float(-1.0), NULL) == I
+    assert lib.bi_rmsnorm(fake + 2, fake, fake, 2, 8, ctypes.c_float(1e-6), NULL) == A
+    assert lib.bi_mean(NULL, NULL, 2, 8, NULL) == I
+    assert lib.bi_mean(fake + 4, fake, 2, 8, NULL) == A
+    assert lib.bi_log_softmax(fake, 9, fake, 2, 8, NULL) == I
+    assert lib.bi_log_softmax(fake + 4, 1, fake, 2, 8, NULL) == A
+    assert lib.bi_silu_mul(NULL, NULL, 2, 8, NULL) == I
+    assert lib.bi_selftest_wait_timeout(10, NULL) == I
+    v = ctypes.c_int32(0)
+    assert lib.bi_get_device_status(NULL, None) == I
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    a = torch.zeros(2, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.bi_matmul(a, a, "nk")
+    with pytest.raises(ValueError):
+        binding.bi_mean(a.float())
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    saved = binding._lib
+    binding._lib = None
+    try:
+        with pytest.raises(RuntimeError, match="libbi.so not found"):
+            binding.load(str(tmp_path / "libbi.so"))
+    finally:
+        binding._lib = saved
