@@ -1,0 +1,667 @@
+#!/usr/bin/env python
+"""Benchmark of the batch-invariant hot path on B200.
+
+One *step* is one pass of every kernel of the path over a batch of M token rows
+(default 1024) shaped like a Qwen3-8B layer plus its LM head:
+
+    h1   = bi_rmsnorm(x, g_attn)                      [M, 4096]    bf16
+    q    = bi_addmm(b_q, h1, W_q)                     [M, 4096]    bias N(0, 0.01)
+    k, v = bi_matmul(h1, W_k), bi_matmul(h1, W_v)     [M, 1024] x 2
+    o    = bi_addmm(x, q, W_o)                        [M, 4096]    residual add
+    h2   = bi_rmsnorm(o, g_mlp)
+    gu   = bi_matmul(h2, W_gu)                        [M, 24576]   gate | up
+    a    = bi_silu_mul(gu)                            [M, 12288]
+    y    = bi_addmm(o, a, W_down)                     [M, 4096]    residual add
+    hf   = bi_rmsnorm(y, g_final)
+    lg   = bi_matmul(hf, W_lm)                        [M, 151936]  bf16 logits
+    lp   = bi_log_softmax(lg)                         [M, 151936]  fp32
+    ce   = bi_mean(lp)                                [M]          mean log-prob (= -H(uniform, p))
+
+(attention itself is not one of the batch-invariant reduction kernels; q stands
+in for its output).  Weights are nn.Linear-style [N, K] bf16 N(0, 0.02), RMSNorm
+gains 1 + N(0, 0.1), activations N(0, 1), all seeded.  The working set (~3 GB)
+is far larger than the 126 MB L2, so no flush is needed between steps.
+
+Printed: ONE JSON line on rank 0.  `value` = GEMM FLOPs of all ranks' steps /
+max-over-ranks device time (TFLOP/s).  `--impl reference` times the fp64 CPU
+oracle on a bounded sample of the same step instead (rank 0 only).
+`--sweep` prints per-kernel M sweeps (not part of the JSON contract).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "bi_matmul TFLOP/s & row-op GB/s vs M (bitwise batch-invariant), % roofline"
+WORKLOAD = "qwen3_8b_layer_plus_lm_head_logprobs"
+HIDDEN, KV, FFN, VOCAB = 4096, 1024, 12288, 151936
+EPS = 1e-6
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# (name, K, N) of the GEMM launches of one step, in order.
+GEMMS = [("q", HIDDEN, HIDDEN), ("k", HIDDEN, KV), ("v", HIDDEN, KV), ("o", HIDDEN, HIDDEN),
+         ("gate_up", HIDDEN, 2 * FFN), ("down", FFN, HIDDEN), ("lm_head", HIDDEN, VOCAB)]
+OPS = ["rms1", "q", "k", "v", "o", "rms2", "gate_up", "silu_mul", "down", "rms3", "lm_head",
+       "log_softmax", "mean"]
+
+
+def gemm_flops_per_row() -> int:
+    return sum(2 * K * N for _, K, N in GEMMS)
+
+
+def row_op_bytes_per_row() -> dict:
+    """Algorithmic HBM bytes per row of each row op (read inputs once, write outputs once)."""
+    return {
+        "rms1": 2 * HIDDEN + 2 * HIDDEN, "rms2": 2 * HIDDEN + 2 * HIDDEN, "rms3": 2 * HIDDEN + 2 * HIDDEN,
+        "silu_mul": 2 * (2 * FFN) + 2 * FFN,
+        "log_softmax": 2 * VOCAB + 4 * VOCAB,
+        "mean": 4 * VOCAB + 4,
+    }
+
+
+def gemm_bytes(M: int, K: int, N: int, extra_in: int = 0) -> int:
+    return 2 * (M * K + K * N + M * N) + extra_in
+
+
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_gemm_lm_head.json")
+GEMM_SOURCES = [os.path.join(ROOT, "invariant_bi_matmul_02_b200", "csrc", n)
+                for n in ("gemm.cuh", "ptx.cuh")]
+
+
+def gemm_source_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for p in GEMM_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(rows: int):
+    """DRAM bytes per LM-head launch from the committed ncu summary, or None when the
+    capture is missing, was taken on another row count, or predates the GEMM source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    if d.get("gemm_source_sha") != gemm_source_sha() or int(d.get("rows", -1)) != rows:
+        return None
+    return int(d["dram_bytes_per_launch"])
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- workload
+
+def make_weights() -> dict:
+    """The step's weights on the host (bf16), drawn from fixed seeds; identical on every rank."""
+    from invariant_bi_matmul_02_b200 import inputs
+    return {
+        "W_q": inputs.weight_normal(11, (HIDDEN, HIDDEN)),
+        "W_k": inputs.weight_normal(12, (KV, HIDDEN)),
+        "W_v": inputs.weight_normal(13, (KV, HIDDEN)),
+        "W_o": inputs.weight_normal(14, (HIDDEN, HIDDEN)),
+        "W_gu": inputs.weight_normal(15, (2 * FFN, HIDDEN)),
+        "W_down": inputs.weight_normal(16, (HIDDEN, FFN)),
+        "W_lm": inputs.weight_normal(17, (VOCAB, HIDDEN)),
+        "g_attn": inputs.gain(18, HIDDEN),
+        "g_mlp": inputs.gain(19, HIDDEN),
+        "g_final": inputs.gain(20, HIDDEN),
+        "b_q": inputs.bias(21, HIDDEN),
+    }
+
+
+class Workload:
+    """Weights (shared by all ranks) and this rank's rows, resident on the device."""
+
+    def __init__(self, rows: int, row0: int, device):
+        import torch
+        from invariant_bi_matmul_02_b200 import inputs
+        self.M = rows
+        self.host = make_weights()
+        self.x_host = inputs.rows_normal(10, row0, rows, HIDDEN)
+        self.dev = {k: v.to(device) for k, v in self.host.items()}
+        self.x = self.x_host.to(device)
+        e = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device=device)
+        M = rows
+        self.buf = {
+            "h1": e(M, HIDDEN), "q": e(M, HIDDEN), "k": e(M, KV), "v": e(M, KV), "o": e(M, HIDDEN),
+            "h2": e(M, HIDDEN), "gu": e(M, 2 * FFN), "a": e(M, FFN), "y": e(M, HIDDEN),
+            "hf": e(M, HIDDEN), "lg": e(M, VOCAB), "lp": e(M, VOCAB, dt=torch.float32),
+            "ce": e(M, dt=torch.float32),
+        }
+
+
+def run_step(wl: Workload, x, marks=None):
+    """One pass of the hot path; `marks` (list of CUDA events, len(OPS)+1) brackets each op."""
+    from invariant_bi_matmul_02_b200 import binding as bi
+    W, B = wl.dev, wl.buf
+
+    def mark(i):
+        if marks is not None:
+            marks[i].record()
+
+    mark(0)
+    bi.bi_rmsnorm(x, W["g_attn"], EPS, out=B["h1"]); mark(1)
+    bi.bi_addmm(W["b_q"], B["h1"], W["W_q"], "nk", out=B["q"]); mark(2)
+    bi.bi_matmul(B["h1"], W["W_k"], "nk", out=B["k"]); mark(3)
+    bi.bi_matmul(B["h1"], W["W_v"], "nk", out=B["v"]); mark(4)
+    bi.bi_addmm(x, B["q"], W["W_o"], "nk", out=B["o"]); mark(5)
+    bi.bi_rmsnorm(B["o"], W["g_mlp"], EPS, out=B["h2"]); mark(6)
+    bi.bi_matmul(B["h2"], W["W_gu"], "nk", out=B["gu"]); mark(7)
+    bi.bi_silu_mul(B["gu"], out=B["a"]); mark(8)
+    bi.bi_addmm(B["o"], B["a"], W["W_down"], "nk", out=B["y"]); mark(9)
+    bi.bi_rmsnorm(B["y"], W["g_final"], EPS, out=B["hf"]); mark(10)
+    bi.bi_matmul(B["hf"], W["W_lm"], "nk", out=B["lg"]); mark(11)
+    bi.bi_log_softmax(B["lg"], out=B["lp"]); mark(12)
+    bi.bi_mean(B["lp"], out=B["ce"]); mark(13)
+    return B["ce"]
+
+
+LAUNCHES_PER_STEP = len(OPS)
+
+
+# ----------------------------------------------------------------------------- oracle leg
+
+def oracle_step_rows(host: dict, x_rows, nthreads: int):
+    """The same step in fp64 on the CPU oracle for a few rows (bf16 rounding between
+    stages, as the device stores bf16 intermediates).  Returns the per-row mean log-prob."""
+    import numpy as np
+    import torch
+    from invariant_bi_matmul_02_b200 import inputs
+    from oracle import oracle
+
+    b = inputs.bf16_bits
+    to_bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16)
+    h1 = to_bf16(oracle.rmsnorm(b(x_rows), b(host["g_attn"]), EPS, nthreads))
+    q = to_bf16(oracle.addmm(b(host["b_q"]), b(h1), b(host["W_q"]), "nk", nthreads))
+    oracle.matmul(b(h1), b(host["W_k"]), "nk", nthreads)
+    oracle.matmul(b(h1), b(host["W_v"]), "nk", nthreads)
+    o = to_bf16(oracle.addmm(b(x_rows), b(q), b(host["W_o"]), "nk", nthreads))
+    h2 = to_bf16(oracle.rmsnorm(b(o), b(host["g_mlp"]), EPS, nthreads))
+    gu = to_bf16(oracle.matmul(b(h2), b(host["W_gu"]), "nk", nthreads))
+    a = to_bf16(oracle.silu_mul(b(gu), nthreads))
+    y = to_bf16(oracle.addmm(b(o), b(a), b(host["W_down"]), "nk", nthreads))
+    hf = to_bf16(oracle.rmsnorm(b(y), b(host["g_final"]), EPS, nthreads))
+    lg = to_bf16(oracle.matmul(b(hf), b(host["W_lm"]), "nk", nthreads))
+    lp = oracle.log_softmax(b(lg), nthreads).astype(np.float32)
+    return oracle.mean(lp, nthreads)
+
+
+def cpu_baseline(host: dict, x_host, budget_s: float = 15.0) -> dict:
+    """Time the oracle on a bounded sample of the step (rank 0, N = 1)."""
+    from oracle import oracle as orc
+    cores = os.cpu_count() or 1
+    orc.max_threads()
+    t0 = time.perf_counter()
+    oracle_step_rows(host, x_host[:1], cores)
+    t1 = time.perf_counter() - t0
+    rows = max(1, min(x_host.shape[0], int(budget_s / max(t1, 1e-3))))
+    t0 = time.perf_counter()
+    oracle_step_rows(host, x_host[:rows], cores)
+    dt = time.perf_counter() - t0
+    return {"value": rows * gemm_flops_per_row() / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{rows} of {x_host.shape[0]} rows through the whole step in fp64 "
+                      f"({dt:.1f} s, after a 1-row calibration of {t1:.2f} s)"}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- main arms
+
+def physical_gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            return int(vis.split(",")[local_rank])
+        except (ValueError, IndexError):
+            return local_rank
+    return local_rank
+
+
+def run_bi(args):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=device)
+
+    from invariant_bi_matmul_02_b200.shard import weak_rows
+    M = args.rows
+    wl = Workload(M, weak_rows(M, rank)[0], device)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        run_step(wl, wl.x)
+    torch.cuda.synchronize()
+
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(len(OPS) + 1)]
+             for _ in range(args.steps)]
+    sampler = ClockSampler(physical_gpu_index(local_rank)) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)  # let nvidia-smi attach before the timed region
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(args.steps):
+        run_step(wl, wl.x, marks[s])
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    barrier()
+    elapsed_ms = start.elapsed_time(end)
+    per_op = {op: 0.0 for op in OPS}
+    for s in range(args.steps):
+        for i, op in enumerate(OPS):
+            per_op[op] += marks[s][i].elapsed_time(marks[s][i + 1])
+    per_op = {k: v / args.steps for k, v in per_op.items()}
+
+    # end to end through the public API: pinned host input in, per-row result out, every step
+    x_pinned = wl.x_host.pin_memory()
+    ce_pinned = torch.empty(M, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(wl.x)
+    e2e_steps = max(1, min(args.steps, 100))
+    for _ in range(2):
+        x_dev.copy_(x_pinned, non_blocking=True)
+        ce_pinned.copy_(run_step(wl, x_dev), non_blocking=True)
+        stream.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_pinned, non_blocking=True)
+        ce_pinned.copy_(run_step(wl, x_dev), non_blocking=True)
+        stream.synchronize()  # the host reads the step's result
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    from invariant_bi_matmul_02_b200 import binding as bi
+    status = bi.bi_get_device_status()
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms, e2e_ms, float(status)], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, e2e_ms, status = float(t[0]), float(t[1]), int(t[2])
+
+    flops_step = gemm_flops_per_row() * M
+    value = world * flops_step * args.steps / (elapsed_ms / 1e3) / 1e12
+    e2e_value = world * flops_step * e2e_steps / (e2e_ms / 1e3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    long_run = elapsed_ms > 2000.0
+    peak_tf = peaks["bf16_tflops_sustained" if long_run else "bf16_tflops"]
+    lm_ms = per_op["lm_head"]
+    lm_flops = 2 * M * HIDDEN * VOCAB
+    achieved = lm_flops / (lm_ms / 1e3) / 1e12
+    gemm_ms = sum(per_op[n] for n, _, _ in GEMMS)
+    row_bytes = row_op_bytes_per_row()
+    row_gbs = {op: round(b * M / (per_op[op] / 1e3) / 1e9, 1) for op, b in row_bytes.items()}
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(wl.host, wl.x_host, args.cpu_budget)
+        line = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(elapsed_ms / args.steps, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "rows_per_gpu": M, "global_rows": M * world,
+                       "hidden": HIDDEN, "kv_out": KV, "ffn": FFN, "vocab": VOCAB,
+                       "accumulate": "fp32", "parallelism": f"replicas x{world} (rows sharded)",
+                       "l2": "working set ~3 GB > 126 MB L2; no flush",
+                       "gemm_tile": bi.bi_gemm_config()},
+            "roofline": {"kernel": "bi_matmul LM head launch [%d x 4096] x [4096 x 151936]" % M,
+                         "bound": "tensor", "achieved": round(achieved, 1), "peak": peak_tf,
+                         "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
+                         "traffic": measured_traffic(M),
+                         "algorithmic_bytes": gemm_bytes(M, HIDDEN, VOCAB),
+                         "peak_source": f"{peak_src} {'bf16_tflops_sustained' if long_run else 'bf16_tflops'}"},
+            "gemm_all_launches_tflops": round(flops_step / (gemm_ms / 1e3) / 1e12, 1),
+            "row_ops_gbs": row_gbs,
+            "row_ops_hbm_peak_gbs": peaks["hbm_gbs"],
+            "breakdown_ms": {k: round(v, 4) for k, v in per_op.items()},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": int(wl.x.numel() * 2), "d2h_bytes_per_step": int(M * 4),
+                    "steps": e2e_steps},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clocks,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if status != 0:
+        raise SystemExit(f"device status word set: {status}")
+
+
+def run_reference(args):
+    """The fp64 CPU oracle, timed on the host cores: each step is one row through the step."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import torch  # noqa: F401
+    from invariant_bi_matmul_02_b200 import inputs
+    M = args.rows
+    hw = make_weights()
+    cores = os.cpu_count() or 1
+    x = inputs.rows_normal(10, 0, max(args.steps + args.warmup, 1), HIDDEN)
+    for i in range(args.warmup):
+        oracle_step_rows(hw, x[i:i + 1], cores)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        r = args.warmup + s
+        oracle_step_rows(hw, x[r:r + 1], cores)
+    dt = time.perf_counter() - t0
+    value = args.steps * gemm_flops_per_row() / dt / 1e12
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / max(args.steps, 1) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "rows_per_gpu": M, "hidden": HIDDEN, "kv_out": KV,
+                   "ffn": FFN, "vocab": VOCAB, "sample_rows_per_step": 1},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"1 of {M} rows through the whole step per timed step, fp64"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- sweep mode
+
+SWEEP_M = [1, 2, 3, 4, 8, 16, 32, 64, 77, 128, 256, 512, 1000, 1024, 2048]
+SWEEP_SHAPES = [("q/o", HIDDEN, HIDDEN), ("k/v", HIDDEN, KV), ("gate/up", HIDDEN, FFN),
+                ("down", FFN, HIDDEN), ("lm_head", HIDDEN, VOCAB)]
+
+
+def _timed(fn, flush, reps):
+    import torch
+    times = []
+    for _ in range(reps):
+        flush()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        e.synchronize()
+        times.append(s.elapsed_time(e))
+    return statistics.median(times)
+
+
+def run_sweep(args):
+    """Per-kernel M sweeps: bi kernels vs torch defaults, L2 flushed before every rep.
+    Also counts, for torch's defaults, rows whose bits differ from their M = 1 result."""
+    import torch
+    import torch.nn.functional as F
+    from invariant_bi_matmul_02_b200 import binding as bi
+    from invariant_bi_matmul_02_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    peaks, src = load_peaks()
+    scratch = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush = lambda: scratch.fill_(1.0)
+    reps = max(5, min(args.steps, 30))
+    out = {"peaks": peaks, "peak_source": src, "gemm": [], "rows": []}
+    print(f"peaks ({src}): {peaks}")
+    print(f"{'shape':9s} {'M':>5s} {'bi us':>9s} {'bi TF/s':>8s} {'%pk':>6s} {'GB/s':>7s} "
+          f"{'torch us':>9s} {'torch TF/s':>10s} {'torch rows != M=1':>18s}")
+    for name, K, N in SWEEP_SHAPES:
+        if args.sweep_shapes and name not in args.sweep_shapes.split(","):
+            continue
+        w = inputs.weight_normal(40, (N, K)).to(dev)
+        pool = inputs.rows_normal(41, 0, max(SWEEP_M), K).to(dev)
+        ref_torch = F.linear(pool[:64], w)  # torch's own rows computed at M = 64 ...
+        ref1 = torch.cat([F.linear(pool[i:i + 1], w) for i in range(64)])  # ... and at M = 1
+        for M in SWEEP_M:
+            a = pool[:M]
+            c = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            t_bi = _timed(lambda: bi.bi_matmul(a, w, "nk", out=c), flush, reps)
+            t_t = _timed(lambda: torch.mm(a, w.t(), out=c), flush, reps)
+            fl = 2 * M * N * K
+            by = gemm_bytes(M, K, N)
+            rows_cmp = min(M, 64)
+            tc = F.linear(a, w)[:rows_cmp]
+            diff = int((tc.view(torch.int16) != ref1[:rows_cmp].view(torch.int16)).any(dim=1).sum())
+            rec = {"shape": name, "K": K, "N": N, "M": M, "bi_us": t_bi * 1e3,
+                   "bi_tflops": fl / t_bi / 1e9, "bi_frac_tensor": fl / t_bi / 1e9 / peaks["bf16_tflops"],
+                   "bi_gbs": by / t_bi / 1e6, "bi_frac_hbm": by / t_bi / 1e6 / peaks["hbm_gbs"],
+                   "torch_us": t_t * 1e3, "torch_tflops": fl / t_t / 1e9,
+                   "torch_rows_differing_from_m1": diff, "rows_compared": rows_cmp}
+            out["gemm"].append(rec)
+            print(f"{name:9s} {M:5d} {t_bi*1e3:9.1f} {rec['bi_tflops']:8.1f} "
+                  f"{100*rec['bi_frac_tensor']:5.1f}% {rec['bi_gbs']:7.0f} {t_t*1e3:9.1f} "
+                  f"{rec['torch_tflops']:10.1f} {diff:>10d}/{rows_cmp}", flush=True)
+        del w, pool, ref_torch, ref1
+        torch.cuda.empty_cache()
+    if not args.sweep_shapes or "rows" in args.sweep_shapes.split(","):
+        print(f"{'op':12s} {'M':>6s} {'bi us':>9s} {'GB/s':>8s} {'%HBM':>6s} {'torch us':>9s} {'torch GB/s':>10s}")
+        g = inputs.gain(42, HIDDEN).to(dev)
+        for M in [1, 8, 64, 148, 256, 1024, 4096, 8192, 16384, 3, 77, 1000]:
+            x = inputs.rows_normal_outliers(43, 0, M, HIDDEN, torch.bfloat16).to(dev)
+            xf = x.float()
+            y = torch.empty_like(x)
+            ym = torch.empty(M, dtype=torch.float32, device=dev)
+            for op, fn, tfn, by in (
+                ("rmsnorm", lambda: bi.bi_rmsnorm(x, g, EPS, out=y),
+                 lambda: F.rms_norm(x, (HIDDEN,), g, EPS), 4 * HIDDEN * M),
+                ("mean", lambda: bi.bi_mean(xf, out=ym), lambda: xf.mean(-1), (4 * HIDDEN + 4) * M)):
+                t_bi = _timed(fn, flush, reps)
+                t_t = _timed(tfn, flush, reps)
+                out["rows"].append({"op": op, "M": M, "bi_us": t_bi * 1e3, "bi_gbs": by / t_bi / 1e6,
+                                    "bi_frac_hbm": by / t_bi / 1e6 / peaks["hbm_gbs"],
+                                    "torch_us": t_t * 1e3, "torch_gbs": by / t_t / 1e6})
+                print(f"{op:12s} {M:6d} {t_bi*1e3:9.1f} {by/t_bi/1e6:8.0f} "
+                      f"{100*by/t_bi/1e6/peaks['hbm_gbs']:5.1f}% {t_t*1e3:9.1f} {by/t_t/1e6:10.0f}",
+                      flush=True)
+        for M in [1, 8, 64, 256, 1024]:
+            x = inputs.rows_normal(44, 0, M, VOCAB, std=1.3).to(dev)
+            y = torch.empty(M, VOCAB, dtype=torch.float32, device=dev)
+            by = 6 * VOCAB * M
+            t_bi = _timed(lambda: bi.bi_log_softmax(x, out=y), flush, reps)
+            t_t = _timed(lambda: torch.log_softmax(x.float(), -1), flush, reps)
+            out["rows"].append({"op": "log_softmax", "M": M, "bi_us": t_bi * 1e3, "bi_gbs": by / t_bi / 1e6,
+                                "bi_frac_hbm": by / t_bi / 1e6 / peaks["hbm_gbs"],
+                                "torch_us": t_t * 1e3, "torch_gbs": by / t_t / 1e6})
+            print(f"{'log_softmax':12s} {M:6d} {t_bi*1e3:9.1f} {by/t_bi/1e6:8.0f} "
+                  f"{100*by/t_bi/1e6/peaks['hbm_gbs']:5.1f}% {t_t*1e3:9.1f} {by/t_t/1e6:10.0f}",
+                  flush=True)
+    if args.sweep_out:
+        with open(args.sweep_out, "w") as f:
+            json.dump(out, f, indent=1)
+
+
+# ----------------------------------------------------------------------------- single-kernel cases
+
+KERNEL_CASES = {
+    # name: (description, bytes in + out) -- inputs larger than L2, a few hundred MB on the device
+    "gemm_gate_up": "bi_matmul M=1024 K=4096 N=24576 (B [N, K])",
+    "gemm_lm_head": "bi_matmul M=1024 K=4096 N=151936 (B [N, K])",
+    "gemm_qo_m256": "bi_matmul M=256 K=4096 N=4096 (B [N, K])",
+    "rmsnorm": "bi_rmsnorm M=16384 H=4096 bf16",
+    "mean": "bi_mean M=16384 H=4096 fp32",
+    "log_softmax": "bi_log_softmax M=1024 V=151936 bf16 -> fp32",
+    "silu_mul": "bi_silu_mul M=1024 F=12288",
+}
+
+
+def run_kernel_case(args):
+    """Launch one kernel `warmup + steps` times on a fixed case (for profiler captures);
+    prints the mean device time of the timed launches."""
+    import torch
+    from invariant_bi_matmul_02_b200 import binding as bi
+    from invariant_bi_matmul_02_b200 import inputs
+    dev = torch.device("cuda", 0)
+    name = args.kernel_case
+    if name.startswith("gemm"):
+        M, K, N = {"gemm_gate_up": (1024, HIDDEN, 2 * FFN), "gemm_lm_head": (1024, HIDDEN, VOCAB),
+                   "gemm_qo_m256": (256, HIDDEN, HIDDEN)}[name]
+        a = inputs.rows_normal(50, 0, M, K).to(dev)
+        w = inputs.weight_normal(51, (N, K)).to(dev)
+        c = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        fn = lambda: bi.bi_matmul(a, w, "nk", out=c)
+        work, unit = 2 * M * N * K, "TFLOP/s"
+    elif name in ("rmsnorm", "mean"):
+        x = inputs.rows_normal_outliers(52, 0, 16384, HIDDEN, torch.bfloat16).to(dev)
+        if name == "rmsnorm":
+            g = inputs.gain(53, HIDDEN).to(dev)
+            y = torch.empty_like(x)
+            fn = lambda: bi.bi_rmsnorm(x, g, EPS, out=y)
+            work = 4 * HIDDEN * 16384
+        else:
+            xf = x.float()
+            y = torch.empty(16384, dtype=torch.float32, device=dev)
+            fn = lambda: bi.bi_mean(xf, out=y)
+            work = (4 * HIDDEN + 4) * 16384
+        unit = "GB/s"
+    elif name == "log_softmax":
+        x = inputs.rows_normal(54, 0, 1024, VOCAB, std=1.3).to(dev)
+        y = torch.empty(1024, VOCAB, dtype=torch.float32, device=dev)
+        fn = lambda: bi.bi_log_softmax(x, out=y)
+        work, unit = 6 * VOCAB * 1024, "GB/s"
+    elif name == "silu_mul":
+        gu = inputs.rows_normal(55, 0, 1024, 2 * FFN, std=2.0).to(dev)
+        h = torch.empty(1024, FFN, dtype=torch.bfloat16, device=dev)
+        fn = lambda: bi.bi_silu_mul(gu, out=h)
+        work, unit = 6 * FFN * 1024, "GB/s"
+    else:
+        raise SystemExit(f"unknown kernel case {name}; choose from {sorted(KERNEL_CASES)}")
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / args.steps
+    rate = work / (ms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
+    print(json.dumps({"kernel_case": name, "what": KERNEL_CASES[name], "launches": args.warmup + args.steps,
+                      "mean_ms": ms, "rate": rate, "unit": unit,
+                      "status": bi.bi_get_device_status()}), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--rows", type=int, default=1024, help="token rows per GPU per step")
+    ap.add_argument("--impl", choices=["bi", "reference"], default="bi")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="per-kernel M sweeps (table, not JSON line)")
+    ap.add_argument("--sweep-shapes", default="", help="comma list of sweep groups (q/o,k/v,...,rows)")
+    ap.add_argument("--sweep-out", default="", help="write the sweep as JSON to this path")
+    ap.add_argument("--kernel-case", default="", help="launch one kernel on a fixed case: "
+                    + ", ".join(sorted(KERNEL_CASES)))
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.sweep:
+        run_sweep(args)
+        return
+    if args.kernel_case:
+        run_kernel_case(args)
+        return
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_bi(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -300,16 +300,28 @@ __global__ void __launch_bounds__(1024, 1) log_softmax_vec_kernel(const uint4 *_
     const MaxSum row = block_merge(acc, red_m, red_s);
     const float m = row.m, ls = __logf(row.s);
 
+    // Pass 2: four chunks in flight per thread; y is streamed out (evict-first) so the
+    // rows still to be re-read keep their place in L2.
     float4 *yr = y + (int64_t)blockIdx.x * (V / 4);
-    for (int64_t c2 = threadIdx.x; c2 < nch; c2 += T) {
+    auto emit = [&](int64_t cc, const uint4 &u) {
         float v[P];
-        LsmTraits<BF16>::unpack(__ldg(xr + c2), v);
+        LsmTraits<BF16>::unpack(u, v);
 #pragma unroll
         for (int k = 0; k < P; k += 4)
-            __stcs(yr + c2 * (P / 4) + k / 4,
+            __stcs(yr + cc * (P / 4) + k / 4,
                    make_float4((v[k] - m) - ls, (v[k + 1] - m) - ls, (v[k + 2] - m) - ls,
                                (v[k + 3] - m) - ls));
+    };
+    int64_t c2 = threadIdx.x;
+    for (; c2 + 3 * (int64_t)T < nch; c2 += 4 * (int64_t)T) {
+        const uint4 u0 = __ldg(xr + c2), u1 = __ldg(xr + c2 + T), u2 = __ldg(xr + c2 + 2 * T),
+                    u3 = __ldg(xr + c2 + 3 * T);
+        emit(c2, u0);
+        emit(c2 + T, u1);
+        emit(c2 + 2 * T, u2);
+        emit(c2 + 3 * T, u3);
     }
+    for (; c2 < nch; c2 += T) emit(c2, __ldg(xr + c2));
 }
 
 // Scalar path for any V: element j belongs to thread j % T.
