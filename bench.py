@@ -75,7 +75,7 @@ def gemm_bytes(M: int, K: int, N: int, extra_in: int = 0) -> int:
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_gemm_lm_head.json")
 GEMM_SOURCES = [os.path.join(ROOT, "invariant_bi_matmul_02_b200", "csrc", n)
-                for n in ("gemm.cuh", "ptx.cuh")]
+                for n in ("gemm.cuh", "gemm_pair.cuh", "ptx.cuh")]
 
 
 def gemm_source_sha() -> str:

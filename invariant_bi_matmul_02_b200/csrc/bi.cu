@@ -15,6 +15,7 @@
 #include <mutex>
 
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "ptx.cuh"
 #include "rowops.cuh"
 
@@ -30,6 +31,7 @@ constexpr int64_t kI32Max = 2147483647;
 struct DeviceState {
     bool ready = false;
     int sms = 0;
+    int gemm_clusters = 0;  // CTA pairs of the GEMM that fit on the device at once
     int32_t *status = nullptr;
 };
 
@@ -51,10 +53,26 @@ bi_status device_state(DeviceState **out)
         void *sym = nullptr;
         if (cudaGetSymbolAddress(&sym, g_bi_status) != cudaSuccess) return BI_ERR_CUDA;
         d.status = static_cast<int32_t *>(sym);
-        if (cudaFuncSetAttribute(bi::gemm_bf16_tcgen05_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 bi::kGemmSmem) != cudaSuccess)
+        if (cudaFuncSetAttribute(bi::gemm_bf16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 bi::kPairSmem) != cudaSuccess)
             return BI_ERR_CUDA;
+        {
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3(2 * d.sms, 1, 1);
+            cfg.blockDim = dim3(bi::kGemmThreads, 1, 1);
+            cfg.dynamicSmemBytes = bi::kPairSmem;
+            cudaLaunchAttribute attr{};
+            attr.id = cudaLaunchAttributeClusterDimension;
+            attr.val.clusterDim.x = 2;
+            attr.val.clusterDim.y = 1;
+            attr.val.clusterDim.z = 1;
+            cfg.attrs = &attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, bi::gemm_bf16_pair_kernel, &cfg) != cudaSuccess || n < 1)
+                return BI_ERR_CUDA;
+            d.gemm_clusters = n;
+        }
         d.ready = true;
     }
     *out = &d;
@@ -125,8 +143,8 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
     p.M = (int32_t)M;
     p.N = (int32_t)N;
     p.K = (int32_t)K;
-    p.m_blocks = (int32_t)((M + bi::kBM - 1) / bi::kBM);
-    p.n_blocks = (int32_t)((N + bi::kBN - 1) / bi::kBN);
+    p.m_blocks = (int32_t)((M + bi::kPairBM - 1) / bi::kPairBM);
+    p.n_blocks = (int32_t)((N + bi::kPairBN - 1) / bi::kPairBN);
     p.k_blocks = (int32_t)((K + bi::kBK - 1) / bi::kBK);
     p.b_mn_major = b_layout == BI_B_KN ? 1 : 0;
     p.c_f32 = c_f32 ? 1 : 0;
@@ -148,19 +166,21 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
     }
 
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
+    const uint32_t b_rows_box = bi::kHalfBN;
     if (tiles > kI32Max) return BI_ERR_UNSUPPORTED;
 
     CUtensorMap tm_a, tm_b;
     st = encode_map(&tm_a, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda, bi::kBK, bi::kBM);
     if (st != BI_OK) return st;
     if (b_layout == BI_B_NK)
-        st = encode_map(&tm_b, B, (uint64_t)K, (uint64_t)N, (uint64_t)ldb, bi::kBK, bi::kBN);
+        st = encode_map(&tm_b, B, (uint64_t)K, (uint64_t)N, (uint64_t)ldb, bi::kBK, b_rows_box);
     else
         st = encode_map(&tm_b, B, (uint64_t)N, (uint64_t)K, (uint64_t)ldb, 64, bi::kBK);
     if (st != BI_OK) return st;
 
-    const int grid = (int)(tiles < dev->sms ? tiles : dev->sms);
-    bi::gemm_bf16_tcgen05_kernel<<<grid, bi::kGemmThreads, bi::kGemmSmem, s>>>(tm_a, tm_b, p);
+    const int64_t pairs = dev->gemm_clusters;
+    const int grid = 2 * (int)(tiles < pairs ? tiles : pairs);
+    bi::gemm_bf16_pair_kernel<<<grid, bi::kGemmThreads, bi::kPairSmem, s>>>(tm_a, tm_b, p);
     return launched();
 }
 
@@ -344,10 +364,10 @@ const char *bi_status_string(bi_status status)
 
 void bi_gemm_config(int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int32_t *mma_k)
 {
-    if (bm) *bm = bi::kBM;
-    if (bn) *bn = bi::kBN;
+    if (bm) *bm = bi::kPairBM;
+    if (bn) *bn = bi::kPairBN;
+    if (stages) *stages = bi::kPStages;
     if (bk) *bk = bi::kBK;
-    if (stages) *stages = bi::kStages;
     if (mma_k) *mma_k = bi::kMmaK;
 }
 

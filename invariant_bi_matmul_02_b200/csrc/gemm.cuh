@@ -1,29 +1,5 @@
-// gemm.cuh -- the batch-invariant bf16 GEMM for sm_100a: C = A . B (+ input).
-//
-// One tile configuration for every call: a 128 x BN output tile per CTA, K sliced
-// 64 at a time into a ring of shared-memory stages by TMA, multiplied by tcgen05.mma
-// (M = 128, N = BN, K = 16 per instruction) into an fp32 accumulator in tensor
-// memory, and read back by four epilogue warps.  Each output element therefore sums
-// its K products in one order that depends only on K: 16-wide tensor-core steps in
-// ascending K, the first overwriting the accumulator.  The tile shape, the K slicing
-// and the instruction sequence never change with M, N or the position of a row in
-// the batch; there is no split-K or stream-K, so no partial sums ever meet across
-// CTAs.  Rows past M and columns past N/K are zero-filled by TMA and never stored.
-//
-// Persistent schedule: gridDim.x CTAs (at most one per SM) walk the tile list with
-// stride gridDim.x.  The tensor-memory accumulator is double-buffered, so the
-// epilogue of one tile overlaps the main loop of the next.  Which CTA computes a tile
-// does not affect its arithmetic.
-//
-// Warp roles (192 threads):
-//   warp 0      TMA producer (one lane)
-//   warp 1      TMEM owner + MMA issuer (one lane)
-//   warps 2..5  epilogue: TMEM -> registers -> (+ bias / residual) -> global
-//
-// Every wait on an mbarrier is bounded.  A wait that runs out records a timeout in
-// the device status word and raises a shared abort flag; every role then leaves its
-// loop, outstanding TMA loads and MMAs are drained (again with a bound), TMEM is
-// freed and the kernel returns.
+// gemm.cuh -- pieces shared by the GEMM kernel: launch parameters, the bounded
+// mbarrier wait, ring-index arithmetic and the epilogue's addend/store helpers.
 #pragma once
 
 #include <cstdint>
@@ -32,33 +8,15 @@
 
 #include "ptx.cuh"
 
-#ifndef BI_GEMM_BN
-#define BI_GEMM_BN 256
-#endif
-
 namespace bi {
 
-constexpr int kBM = 128;
-constexpr int kBN = BI_GEMM_BN;
-constexpr int kBK = 64;          // one 128-byte swizzle row of bf16
-constexpr int kMmaK = 16;        // K of one tcgen05.mma kind::f16
-constexpr int kGemmThreads = 192;
-constexpr int kABytes = kBM * kBK * 2;
-constexpr int kBBytes = kBN * kBK * 2;
-constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kBM = 128;          // rows of C per CTA (one TMEM lane per row)
+constexpr int kBK = 64;           // K per pipeline stage: one 128-byte swizzle row of bf16
+constexpr int kMmaK = 16;         // K of one tcgen05.mma kind::f16
+constexpr int kGemmThreads = 192; // warp 0 TMA, warp 1 TMEM/MMA, warps 2..5 epilogue
 constexpr int kSmemBudget = 227 * 1024;
 constexpr int kSmemMisc = 1024 /*alignment slack*/ + 512 /*barriers, flags*/;
-constexpr int kStagesRaw = (kSmemBudget - kSmemMisc) / kStageBytes;
-constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-constexpr int kGemmSmem = kStages * kStageBytes + kSmemMisc;
 constexpr uint32_t pow2_at_least(uint32_t v, uint32_t p = 32) { return p >= v ? p : pow2_at_least(v, p * 2); }
-constexpr uint32_t kTmemCols = pow2_at_least(2 * kBN);
-
-static_assert(kBN % 32 == 0 && kBN >= 32 && kBN <= 256, "tile N must be a multiple of 32 in [32, 256]");
-static_assert(kBN % 64 == 0, "the [K, N] operand is loaded as 64-column boxes");
-static_assert(kStages >= 2, "need at least two pipeline stages");
-static_assert(kTmemCols <= 512, "accumulators must fit in tensor memory");
-static_assert(kGemmSmem > 114 * 1024, "one CTA per SM keeps the TMEM allocation uncontended");
 
 enum AddendMode : int { kAddNone = 0, kAddBias = 1, kAddMatrix = 2 };
 
@@ -162,192 +120,6 @@ __device__ __forceinline__ void store_row_chunk(const GemmParams &p, int64_t row
         } else {
             for (int j = 0; j < 32 && col0 + j < p.N; ++j) dst[j] = __float2bfloat16_rn(v[j]);
         }
-    }
-}
-
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tm_a,
-                             const __grid_constant__ CUtensorMap tm_b, const GemmParams p)
-{
-    extern __shared__ uint8_t smem_raw[];
-    // 128-byte swizzle atoms need 1024-byte aligned stage buffers (shared-window offset).
-    uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    uint8_t *sA = smem;
-    uint8_t *sB = smem + kStages * kABytes;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sB + kStages * kBBytes);
-    uint64_t *empty = full + kStages;
-    uint64_t *tfull = empty + kStages;   // [2] accumulator ready for the epilogue
-    uint64_t *tempty = tfull + 2;        // [2] accumulator drained by the epilogue
-    uint64_t *drain = tempty + 2;        // [1] used only when aborting
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4 * 32);
-        }
-        mbar_init(drain, 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
-        prefetch_tensor_map(&tm_a);
-        prefetch_tensor_map(&tm_b);
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_holder, kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    const uint32_t tmem_base = *tmem_holder;
-
-    const int num_tiles = p.m_blocks * p.n_blocks;
-    const uint64_t lim = p.wait_limit_ns;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            // ---------------------------------------------------------- TMA producer
-            uint32_t stage = 0, phase = 0;
-            uint32_t filled = 0;        // bit s: stage s has a load whose landing is unobserved
-            uint32_t fill_parity = 0;   // bit s: parity of that load's phase
-            bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-                const int m0 = (tile % p.m_blocks) * kBM;
-                const int n0 = (tile / p.m_blocks) * kBN;
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
-                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&full[stage], kStageBytes);
-                    tma_load_2d(sA + stage * kABytes, &tm_a, &full[stage], kb * kBK, m0);
-                    uint8_t *dstB = sB + stage * kBBytes;
-                    if (p.b_mn_major) {
-                        // [K, N] operand: kBN/64 boxes of 64 columns x 64 k-rows each.
-#pragma unroll
-                        for (int g = 0; g < kBN / 64; ++g)
-                            tma_load_2d(dstB + g * (64 * kBK * 2), &tm_b, &full[stage], n0 + g * 64,
-                                        kb * kBK);
-                    } else {
-                        tma_load_2d(dstB, &tm_b, &full[stage], kb * kBK, n0);
-                    }
-                    filled |= 1u << stage;
-                    fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
-                    advance(stage, phase, kStages);
-                }
-            }
-            if (ok) {
-                // Tail: wait until the MMA warp has released every stage, so no
-                // tensor-core read or barrier arrival is still in flight at exit.
-                for (int s = 0; s < kStages; ++s) {
-                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim)) break;
-                    advance(stage, phase, kStages);
-                }
-            } else {
-                // Abort: let every issued TMA load land before the CTA's shared memory goes away.
-                for (int s = 0; s < kStages; ++s) {
-                    if (!(filled >> s & 1u)) continue;
-                    const uint32_t a = smem_addr(&full[s]);
-                    const uint32_t par = fill_parity >> s & 1u;
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(a, par) && global_timer_ns() - t0 < lim) {
-                    }
-                }
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------------------------------------------------- MMA issuer
-            const uint32_t idesc = mma_idesc_bf16(kBM, kBN, p.b_mn_major ? 1u : 0u);
-            uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-                if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, lim)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + acc * kBN;
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
-                    if (!wait_bounded(&full[stage], phase, abort_flag, p.status, lim)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    const uint32_t a_base = smem_addr(sA + stage * kABytes);
-                    const uint32_t b_base = smem_addr(sB + stage * kBBytes);
-#pragma unroll
-                    for (int kk = 0; kk < kBK / kMmaK; ++kk) {
-                        const uint64_t a_desc = sw128_desc(a_base + kk * (kMmaK * 2), 16, 1024);
-                        const uint64_t b_desc =
-                            p.b_mn_major ? sw128_desc(b_base + kk * (kMmaK * 128), 64 * kBK * 2, 1024)
-                                         : sw128_desc(b_base + kk * (kMmaK * 2), 16, 1024);
-                        tc_mma_bf16(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
-                    }
-                    tc_commit(&empty[stage]);
-                    advance(stage, phase, kStages);
-                }
-                if (!ok) break;
-                tc_commit(&tfull[acc]);
-                advance(acc, acc_phase, 2);
-            }
-            if (!ok) {
-                // Abort: wait for every MMA already issued before TMEM is released.
-                tc_commit(drain);
-                const uint32_t a = smem_addr(drain);
-                const uint64_t t0 = global_timer_ns();
-                while (!mbar_try_wait(a, 0) && global_timer_ns() - t0 < lim) {
-                }
-            }
-        }
-    } else {
-        // -------------------------------------------------------------- epilogue
-        const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 are this warp's
-        const int row_in_tile = quarter * 32 + lane;
-        uint32_t acc = 0, acc_phase = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            // All lanes take the same branch: tcgen05.ld below is warp-collective.
-            const bool ready = wait_bounded(&tfull[acc], acc_phase, abort_flag, p.status, lim);
-            if (!__all_sync(0xffffffffu, ready)) break;
-            tc_fence_after_sync();
-            const int64_t row = (int64_t)(tile % p.m_blocks) * kBM + row_in_tile;
-            const int64_t n0 = (int64_t)(tile / p.m_blocks) * kBN;
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kBN;
-#pragma unroll 1
-            for (int c = 0; c < kBN / 32; ++c) {
-                uint32_t r[32];
-                tmem_load_32x32(t_row + c * 32, r);
-                tmem_wait_ld();
-                const int64_t col0 = n0 + c * 32;
-                if (row < p.M && col0 < p.N) {
-                    float v[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-                    const bool full_chunk = col0 + 32 <= p.N;
-                    add_addend(p, row, col0, full_chunk, v);
-                    store_row_chunk(p, row, col0, full_chunk, v);
-                }
-            }
-            tc_fence_before_sync();
-            mbar_arrive(&tempty[acc]);
-            advance(acc, acc_phase, 2);
-        }
-    }
-
-    tc_fence_before_sync();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after_sync();
-        tmem_dealloc(tmem_base, kTmemCols);
     }
 }
 

@@ -1,0 +1,238 @@
+// gemm_pair.cuh -- the batch-invariant bf16 GEMM: tcgen05 on CTA pairs (cta_group::2).
+//
+// One tile configuration for every call: a CTA pair (a 2-CTA cluster on one TPC)
+// owns a 256 x kPairBN output tile.  Each CTA stages, per 64-wide K slice, its own 128
+// rows of A and its own kPairBN/2 rows (columns of C) of B; the leader CTA issues
+// tcgen05.mma.cta_group::2 (M = 256, N = kPairBN, K = 16), which reads both CTAs'
+// shared memory and accumulates each CTA's 128 x kPairBN half of the tile in fp32 in
+// that CTA's tensor memory.  Per output element the order is the same as for any
+// single tcgen05 MMA: the first 16-wide K step overwrites the accumulator, every later
+// step adds in ascending K.  It depends only on K -- not on M, N, the row's position,
+// or which pair computes the tile.  No split-K, no stream-K, no tile switch.
+//
+// Pipeline, per CTA pair:
+//   full[s]   (leader)  armed by the leader's producer with both CTAs' bytes; both
+//                       CTAs' TMA loads complete on it.
+//   empty[s]  (both)    the leader's MMA commit, multicast to both CTAs, frees stage s.
+//   tfull[b]  (both)    the leader's commit after a tile's last MMA: accumulator b ready.
+//   tempty[b] (leader)  one arrival per epilogue warp of both CTAs: accumulator b drained.
+// TMA loads are plain tiled loads (no cluster multicast); only the tcgen05.commit
+// arrivals are multicast.
+//
+// Warp roles (192 threads per CTA): warp 0 TMA producer lane, warp 1 TMEM owner (both
+// CTAs) and MMA issuer (leader only), warps 2..5 epilogue.  Every wait is bounded.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+#ifndef BI_GEMM_PAIR_BN
+#define BI_GEMM_PAIR_BN 256  // the one tile width every call uses; other values exist for experiments only
+#endif
+
+namespace bi {
+
+constexpr int kPairBM = 256;                   // rows of C per CTA pair
+constexpr int kPairBN = BI_GEMM_PAIR_BN;       // columns of C per CTA pair
+constexpr int kHalfBN = kPairBN / 2;           // B rows staged by each CTA
+constexpr int kPABytes = 128 * kBK * 2;        // A slice per CTA
+constexpr int kPBBytes = kHalfBN * kBK * 2;    // B slice per CTA
+constexpr int kPStageBytes = kPABytes + kPBBytes;
+constexpr int kPStagesRaw = (kSmemBudget - kSmemMisc) / kPStageBytes;
+constexpr int kPStages = kPStagesRaw > 12 ? 12 : kPStagesRaw;
+constexpr int kPairSmem = kPStages * kPStageBytes + kSmemMisc;
+constexpr uint32_t kPairTmemCols = pow2_at_least(2 * kPairBN);
+
+static_assert(kPairBN % 128 == 0 && kPairBN <= 256, "pair tile N must be 128 or 256");
+static_assert(kPStages >= 2, "need at least two pipeline stages");
+static_assert(kPairTmemCols <= 512, "accumulators must fit in tensor memory");
+static_assert(kPairSmem > 114 * 1024, "one CTA per SM keeps the TMEM allocation uncontended");
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
+                          const __grid_constant__ CUtensorMap tm_b, const GemmParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + kPStages * kPABytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sB + kPStages * kPBBytes);
+    uint64_t *empty = full + kPStages;
+    uint64_t *tfull = empty + kPStages;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 2 * 4);  // one arrival per epilogue warp of both CTAs
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensor_map(&tm_a);
+        prefetch_tensor_map(&tm_b);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_holder, kPairTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_holder;
+
+    const int m_blocks = (p.M + kPairBM - 1) / kPairBM;
+    const int n_blocks = (p.N + kPairBN - 1) / kPairBN;
+    const int num_tiles = m_blocks * n_blocks;
+    const int first = (int)cluster_id_x(), stride = (int)num_clusters_x();
+    const uint64_t lim = p.wait_limit_ns;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- TMA producer (both CTAs)
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int tile = first; ok && tile < num_tiles; tile += stride) {
+                const int m0 = (tile % m_blocks) * kPairBM + 128 * (int)rank;
+                const int nh0 = (tile / m_blocks) * kPairBN + kHalfBN * (int)rank;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kPStageBytes);
+                    const uint32_t bar = map_to_rank(smem_addr(&full[stage]), 0);
+                    tma_load_2d_pair(sA + stage * kPABytes, &tm_a, bar, kb * kBK, m0);
+                    uint8_t *dstB = sB + stage * kPBBytes;
+                    if (p.b_mn_major) {
+#pragma unroll
+                        for (int g = 0; g < kHalfBN / 64; ++g)
+                            tma_load_2d_pair(dstB + g * (64 * kBK * 2), &tm_b, bar, nh0 + g * 64, kb * kBK);
+                    } else {
+                        tma_load_2d_pair(dstB, &tm_b, bar, kb * kBK, nh0);
+                    }
+                    advance(stage, phase, kPStages);
+                }
+            }
+            if (ok) {
+                // Tail: every stage released by the leader's MMA, so no multicast arrival
+                // is still on its way to this CTA when it exits.
+                for (int s = 0; s < kPStages; ++s) {
+                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim)) break;
+                    advance(stage, phase, kPStages);
+                }
+            } else {
+                // Abort: loads already issued complete on the leader's barrier, which this
+                // CTA cannot observe; give them a bounded grace period to land.
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 2000000ull) {
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ---------------------------------------------------------- MMA issuer (leader)
+            const uint32_t idesc = mma_idesc_bf16(kPairBM, kPairBN, p.b_mn_major ? 1u : 0u);
+            uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+            bool ok = true;
+            for (int tile = first; ok && tile < num_tiles; tile += stride) {
+                if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, lim)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + acc * kPairBN;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!wait_bounded(&full[stage], phase, abort_flag, p.status, lim)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_base = smem_addr(sA + stage * kPABytes);
+                    const uint32_t b_base = smem_addr(sB + stage * kPBBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / kMmaK; ++kk) {
+                        const uint64_t a_desc = sw128_desc(a_base + kk * (kMmaK * 2), 16, 1024);
+                        const uint64_t b_desc =
+                            p.b_mn_major ? sw128_desc(b_base + kk * (kMmaK * 128), 64 * kBK * 2, 1024)
+                                         : sw128_desc(b_base + kk * (kMmaK * 2), 16, 1024);
+                        tc_mma_bf16_pair(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    tc_commit_pair_mc(&empty[stage], 0x3);
+                    advance(stage, phase, kPStages);
+                }
+                if (!ok) break;
+                tc_commit_pair_mc(&tfull[acc], 0x3);
+                advance(acc, acc_phase, 2);
+            }
+            if (!ok) {
+                tc_commit_pair_mc(drain, 0x1);
+                const uint32_t a = smem_addr(drain);
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(a, 0) && global_timer_ns() - t0 < lim) {
+                }
+            }
+        }
+    } else {
+        // -------------------------------------------------------------- epilogue (both CTAs)
+        const int quarter = warp & 3;
+        const int row_in_half = quarter * 32 + lane;
+        const uint32_t tempty_leader0 = map_to_rank(smem_addr(&tempty[0]), 0);
+        uint32_t acc = 0, acc_phase = 0;
+        for (int tile = first; tile < num_tiles; tile += stride) {
+            const bool ready = wait_bounded(&tfull[acc], acc_phase, abort_flag, p.status, lim);
+            if (!__all_sync(0xffffffffu, ready)) break;
+            tc_fence_after_sync();
+            const int64_t row = (int64_t)(tile % m_blocks) * kPairBM + 128 * rank + row_in_half;
+            const int64_t n0 = (int64_t)(tile / m_blocks) * kPairBN;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kPairBN;
+#pragma unroll 1
+            for (int c = 0; c < kPairBN / 32; ++c) {
+                uint32_t r[32];
+                tmem_load_32x32(t_row + c * 32, r);
+                tmem_wait_ld();
+                const int64_t col0 = n0 + c * 32;
+                if (row < p.M && col0 < p.N) {
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+                    const bool full_chunk = col0 + 32 <= p.N;
+                    add_addend(p, row, col0, full_chunk, v);
+                    store_row_chunk(p, row, col0, full_chunk, v);
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * sizeof(uint64_t));
+            advance(acc, acc_phase, 2);
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    cluster_sync_all();  // no CTA leaves while its peer may still signal its barriers
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc_pair(tmem_base, kPairTmemCols);
+    }
+}
+
+}  // namespace bi

@@ -44,8 +44,8 @@ def test_status_strings_and_config(lib):
     assert binding.status_string(binding.BI_ERR_TIMEOUT) == "BI_ERR_TIMEOUT"
     assert binding.status_string(99) == "BI_ERR_UNKNOWN"
     cfg = binding.bi_gemm_config()
-    assert cfg["bm"] == 128 and cfg["bk"] == 64 and cfg["mma_k"] == 16
-    assert cfg["bn"] in (64, 128, 192, 256) and cfg["stages"] >= 2
+    assert cfg["bm"] == 256 and cfg["bk"] == 64 and cfg["mma_k"] == 16  # a CTA pair's tile
+    assert cfg["bn"] in (128, 256) and cfg["stages"] >= 2
     assert binding.bi_version() >= 100
 
 
