@@ -73,6 +73,11 @@ bi_status device_state(DeviceState **out)
                 return BI_ERR_CUDA;
             d.gemm_clusters = n;
         }
+        if (cudaFuncSetAttribute(bi::log_softmax_stream_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kLsmSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(bi::log_softmax_stream_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kLsmSmem) != cudaSuccess)
+            return BI_ERR_CUDA;
         d.ready = true;
     }
     *out = &d;
@@ -289,12 +294,16 @@ bi_status bi_log_softmax(const void *x, bi_dtype x_dtype, float *y, int64_t M, i
     const int per = bf16 ? 8 : 4;
     if (V % per == 0) {
         if (!aligned16(x) || !aligned16(y)) return BI_ERR_ALIGNMENT;
-        const uint4 *xv = static_cast<const uint4 *>(x);
-        float4 *yv = reinterpret_cast<float4 *>(y);
+        DeviceState *dev = nullptr;
+        bi_status st = device_state(&dev);
+        if (st != BI_OK) return st;
+        const uint8_t *xb = static_cast<const uint8_t *>(x);
         if (bf16)
-            bi::log_softmax_vec_kernel<true><<<(unsigned)M, T, 0, s>>>(xv, yv, V);
+            bi::log_softmax_stream_kernel<true><<<(unsigned)M, bi::kLsmThreads, bi::kLsmSmem, s>>>(
+                xb, y, V, dev->status, kWaitLimitNs);
         else
-            bi::log_softmax_vec_kernel<false><<<(unsigned)M, T, 0, s>>>(xv, yv, V);
+            bi::log_softmax_stream_kernel<false><<<(unsigned)M, bi::kLsmThreads, bi::kLsmSmem, s>>>(
+                xb, y, V, dev->status, kWaitLimitNs);
     } else {
         if (bf16)
             bi::log_softmax_scalar_kernel<true><<<(unsigned)M, T, 0, s>>>(x, y, V);

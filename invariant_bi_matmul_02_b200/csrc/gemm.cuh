@@ -34,35 +34,6 @@ struct GemmParams {
     uint64_t wait_limit_ns;
 };
 
-// Bounded wait on (bar, parity).  Returns false if the wait ran out (after recording
-// the timeout and raising the abort flag) or if another role already aborted.
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                             int32_t *status, uint64_t limit_ns)
-{
-    const uint32_t a = smem_addr(bar);
-    if (mbar_try_wait(a, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    for (;;) {
-#pragma unroll 1
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(a, parity)) return true;
-        if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > limit_ns) {
-            *reinterpret_cast<volatile int32_t *>(status) = 5;  // BI_ERR_TIMEOUT
-            *abort_flag = 1;
-            return false;
-        }
-    }
-}
-
-__device__ __forceinline__ void advance(uint32_t &idx, uint32_t &phase, uint32_t n)
-{
-    if (++idx == n) {
-        idx = 0;
-        phase ^= 1u;
-    }
-}
-
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float(b16 << 16); }
 
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi)

@@ -302,3 +302,51 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint64_t *bar, uint16_t cta_ma
 }
 
 }  // namespace bi
+
+namespace bi {
+
+// 1-D bulk copy global -> this CTA's shared memory, completion (bytes) on `bar`.
+// Addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+}  // namespace bi
+
+namespace bi {
+
+// Bounded wait on (bar, parity).  Returns false if the wait ran out (after recording
+// the timeout and raising the abort flag) or if another role already aborted.
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                             int32_t *status, uint64_t limit_ns)
+{
+    const uint32_t a = smem_addr(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(a, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+            *reinterpret_cast<volatile int32_t *>(status) = 5;  // BI_ERR_TIMEOUT
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void advance(uint32_t &idx, uint32_t &phase, uint32_t n)
+{
+    if (++idx == n) {
+        idx = 0;
+        phase ^= 1u;
+    }
+}
+
+}  // namespace bi

@@ -12,6 +12,8 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include "ptx.cuh"
+
 namespace bi {
 
 #define kNegInf (-__builtin_huge_valf())
@@ -112,7 +114,7 @@ __host__ __device__ inline int clamp_threads(long long v)
 __host__ inline int rmsnorm_threads(long long H) { return clamp_threads((H / 8 + 1) / 2); }
 // mean, fp32 rows: aim for four 16-byte chunks per thread.
 __host__ inline int mean_threads(long long H) { return clamp_threads((H / 4 + 3) / 4); }
-// log_softmax: long rows, a full block.
+// log_softmax, scalar path (rows whose length breaks the 16-byte vector rule).
 __host__ inline int log_softmax_threads(long long V) { return clamp_threads((V + 7) / 8); }
 
 // --------------------------------------------------------------- RMSNorm
@@ -231,29 +233,6 @@ __global__ void __launch_bounds__(1024) mean_scalar_kernel(const float *__restri
 
 // --------------------------------------------------------------- log_softmax
 
-template <bool BF16>
-struct LsmTraits;
-
-template <>
-struct LsmTraits<true> {  // 8 bf16 per 16-byte chunk
-    static constexpr int kPer = 8;
-    __device__ static void unpack(const uint4 &u, float (&v)[8])
-    {
-        v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
-        v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
-    }
-};
-
-template <>
-struct LsmTraits<false> {  // 4 fp32 per 16-byte chunk
-    static constexpr int kPer = 4;
-    __device__ static void unpack(const uint4 &u, float (&v)[4])
-    {
-        v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
-        v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
-    }
-};
-
 template <int P>
 __device__ __forceinline__ void lsm_accumulate(MaxSum &acc, const float (&v)[P])
 {
@@ -265,63 +244,6 @@ __device__ __forceinline__ void lsm_accumulate(MaxSum &acc, const float (&v)[P])
 #pragma unroll
         for (int k = 0; k < P; ++k) acc.s += __expf(v[k] - acc.m);
     }
-}
-
-// Vector path (V a multiple of the chunk width).  Chunk c belongs to thread c % T and
-// is visited in increasing c.  Pass 1 builds the row's (max, sum); pass 2 re-reads the
-// row and writes y = (x - max) - log(sum) as fp32.
-template <bool BF16>
-__global__ void __launch_bounds__(1024, 1) log_softmax_vec_kernel(const uint4 *__restrict__ x,
-                                                                 float4 *__restrict__ y,
-                                                                 int64_t V)
-{
-    __shared__ float red_m[32], red_s[32];
-    constexpr int P = LsmTraits<BF16>::kPer;
-    const int64_t nch = V / P;
-    const int T = blockDim.x;
-    const uint4 *xr = x + (int64_t)blockIdx.x * nch;
-
-    MaxSum acc{kNegInf, 0.0f};
-    int64_t c = threadIdx.x;
-    for (; c + 3 * (int64_t)T < nch; c += 4 * (int64_t)T) {
-        const uint4 u0 = __ldg(xr + c), u1 = __ldg(xr + c + T), u2 = __ldg(xr + c + 2 * T),
-                    u3 = __ldg(xr + c + 3 * T);
-        float v[P];
-        LsmTraits<BF16>::unpack(u0, v); lsm_accumulate(acc, v);
-        LsmTraits<BF16>::unpack(u1, v); lsm_accumulate(acc, v);
-        LsmTraits<BF16>::unpack(u2, v); lsm_accumulate(acc, v);
-        LsmTraits<BF16>::unpack(u3, v); lsm_accumulate(acc, v);
-    }
-    for (; c < nch; c += T) {
-        float v[P];
-        LsmTraits<BF16>::unpack(__ldg(xr + c), v);
-        lsm_accumulate(acc, v);
-    }
-    const MaxSum row = block_merge(acc, red_m, red_s);
-    const float m = row.m, ls = __logf(row.s);
-
-    // Pass 2: four chunks in flight per thread; y is streamed out (evict-first) so the
-    // rows still to be re-read keep their place in L2.
-    float4 *yr = y + (int64_t)blockIdx.x * (V / 4);
-    auto emit = [&](int64_t cc, const uint4 &u) {
-        float v[P];
-        LsmTraits<BF16>::unpack(u, v);
-#pragma unroll
-        for (int k = 0; k < P; k += 4)
-            __stcs(yr + cc * (P / 4) + k / 4,
-                   make_float4((v[k] - m) - ls, (v[k + 1] - m) - ls, (v[k + 2] - m) - ls,
-                               (v[k + 3] - m) - ls));
-    };
-    int64_t c2 = threadIdx.x;
-    for (; c2 + 3 * (int64_t)T < nch; c2 += 4 * (int64_t)T) {
-        const uint4 u0 = __ldg(xr + c2), u1 = __ldg(xr + c2 + T), u2 = __ldg(xr + c2 + 2 * T),
-                    u3 = __ldg(xr + c2 + 3 * T);
-        emit(c2, u0);
-        emit(c2 + T, u1);
-        emit(c2 + 2 * T, u2);
-        emit(c2 + 3 * T, u3);
-    }
-    for (; c2 < nch; c2 += T) emit(c2, __ldg(xr + c2));
 }
 
 // Scalar path for any V: element j belongs to thread j % T.
@@ -345,6 +267,118 @@ __global__ void __launch_bounds__(1024, 1) log_softmax_scalar_kernel(const void 
     const float m = row.m, ls = __logf(row.s);
     for (int64_t j = threadIdx.x; j < V; j += blockDim.x) y[base + j] = (load(j) - m) - ls;
 }
+
+// --------------------------------------------------------------- log_softmax, streamed rows
+
+// Vector path of log_softmax on long rows.  One block of kLsmThreads threads per row,
+// two blocks per SM.  The row streams through a ring of kLsmStages shared-memory chunks of
+// kLsmChunk bytes, each filled by one 1-D bulk copy that completes on its own mbarrier;
+// pass 1 builds the row's (max, sum of exp), pass 2 streams the row again and writes
+// y = (x - max) - log(sum).
+//
+// Element order (fixed by V alone): the row is cut into chunks of kLsmChunk bytes; a chunk
+// into groups of 4 elements; thread t owns groups t, t + T, t + 2T, ... of every chunk and
+// folds them in that order, chunk after chunk.  Consecutive threads read consecutive
+// shared-memory words and write consecutive 16-byte pieces of y.
+constexpr int kLsmThreads = 512;
+constexpr int kLsmChunk = 16384;
+constexpr int kLsmStages = 6;
+
+template <bool BF16>
+__global__ void __launch_bounds__(kLsmThreads, 2)
+    log_softmax_stream_kernel(const uint8_t *__restrict__ x, float *__restrict__ y, int64_t V,
+                              int32_t *status, uint64_t wait_limit_ns)
+{
+    constexpr int kElem = BF16 ? 2 : 4;
+    constexpr int kPerChunk = kLsmChunk / kElem;      // elements per chunk
+    constexpr int kGroups = kPerChunk / 4;            // groups of 4 elements per chunk
+    extern __shared__ __align__(128) uint8_t lsm_smem[];
+    uint8_t(*ring)[kLsmChunk] = reinterpret_cast<uint8_t(*)[kLsmChunk]>(lsm_smem);
+    __shared__ uint64_t full[kLsmStages];
+    __shared__ float red_m[32], red_s[32];
+    __shared__ int abort_flag_s;
+    volatile int *abort_flag = &abort_flag_s;
+
+    const int64_t row_bytes = V * kElem;
+    const int nchunks = (int)((row_bytes + kLsmChunk - 1) / kLsmChunk);
+    const uint8_t *xr = x + (int64_t)blockIdx.x * row_bytes;
+    float *yr = y + (int64_t)blockIdx.x * V;
+    const int tid = threadIdx.x;
+
+    if (tid == 0) {
+        for (int s = 0; s < kLsmStages; ++s) mbar_init(&full[s], 1);
+        abort_flag_s = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // Chunk q (0 .. 2*nchunks-1: both passes) goes to stage q % S with parity (q / S) & 1.
+    auto issue = [&](int q) {
+        const int c = q < nchunks ? q : q - nchunks;
+        const int64_t off = (int64_t)c * kLsmChunk;
+        const uint32_t bytes = (uint32_t)(row_bytes - off < kLsmChunk ? row_bytes - off : kLsmChunk);
+        mbar_arrive_expect_tx(&full[q % kLsmStages], bytes);
+        bulk_load(ring[q % kLsmStages], xr + off, bytes, &full[q % kLsmStages]);
+    };
+    const int total = 2 * nchunks;
+    int issued = 0;
+    if (tid == 0)
+        for (; issued < kLsmStages && issued < total; ++issued) issue(issued);
+
+    MaxSum acc{kNegInf, 0.0f};
+    float m = 0.0f, ls = 0.0f;
+    int q = 0;
+    for (; q < total; ++q) {
+        const int stage = q % kLsmStages;
+        const bool landed = wait_bounded(&full[stage], (uint32_t)(q / kLsmStages) & 1u, abort_flag,
+                                         status, wait_limit_ns);
+        if (!__syncthreads_and(landed ? 1 : 0)) break;
+        const int c = q < nchunks ? q : q - nchunks;
+        const int64_t e0 = (int64_t)c * kPerChunk;  // first element of this chunk
+        const uint8_t *buf = ring[stage];
+        if (q == nchunks) {
+            const MaxSum row = block_merge(acc, red_m, red_s);
+            m = row.m;
+            ls = __logf(row.s);
+        }
+        for (int g = tid; g < kGroups; g += kLsmThreads) {
+            const int64_t e = e0 + 4 * (int64_t)g;
+            if (e >= V) break;
+            float v[4];
+            if (BF16) {
+                const uint2 u = *reinterpret_cast<const uint2 *>(buf + 8 * g);
+                v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+            } else {
+                const float4 f = *reinterpret_cast<const float4 *>(buf + 16 * g);
+                v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+            }
+            if (q < nchunks) {
+                lsm_accumulate(acc, v);
+            } else {
+                __stcs(reinterpret_cast<float4 *>(yr + e),
+                       make_float4((v[0] - m) - ls, (v[1] - m) - ls, (v[2] - m) - ls, (v[3] - m) - ls));
+            }
+        }
+        __syncthreads();  // every thread is done with this stage
+        if (tid == 0 && issued < total) {
+            fence_proxy_async_smem();  // order the reads above before the copy that overwrites
+            issue(issued++);
+        }
+    }
+    if (q < total && tid == 0) {
+        // A wait ran out: let the copies still in flight (chunks q .. issued-1, one per
+        // stage) land before the block's shared memory goes away.
+        for (int r = q; r < issued; ++r) {
+            const uint32_t a = smem_addr(&full[r % kLsmStages]);
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(a, (uint32_t)(r / kLsmStages) & 1u) &&
+                   global_timer_ns() - t0 < wait_limit_ns) {
+            }
+        }
+    }
+}
+
+constexpr int kLsmSmem = kLsmStages * kLsmChunk;
 
 // --------------------------------------------------------------- SiLU * up
 

@@ -211,7 +211,7 @@ def test_addmm_residual_invariance_positions():
     w = weight(235, N, K, "nk").to(DEV)
     ref = torch.cat([bi.bi_addmm(resid[i:i + 1], pool[i:i + 1], w) for i in range(512)])
     for M in (2, 3, 77, 128, 129, 256, 512):
-        for r in (0, 127, 128, M - 1):
+        for r in (0, 127, 128, 255, 256, M - 1):
             if r >= M:
                 continue
             idx = torch.arange(M, device=DEV)
