@@ -51,8 +51,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (name, K, N) of the GEMM launches of one step, in order.
 GEMMS = [("q", HIDDEN, HIDDEN), ("k", HIDDEN, KV), ("v", HIDDEN, KV), ("o", HIDDEN, HIDDEN),
          ("gate_up", HIDDEN, 2 * FFN), ("down", FFN, HIDDEN), ("lm_head", HIDDEN, VOCAB)]
-OPS = ["rms1", "q", "k", "v", "o", "rms2", "gate_up", "silu_mul", "down", "rms3", "lm_head",
-       "log_softmax", "mean"]
+OPS_UNFUSED = ["rms1", "q", "k", "v", "o", "rms2", "gate_up", "silu_mul", "down", "rms3", "lm_head",
+               "log_softmax", "mean"]
+OPS_FUSED = ["rms1", "q", "k", "v", "o", "rms2", "gate_up_silu", "down", "rms3", "lm_head",
+             "log_softmax", "mean"]
 
 
 def gemm_flops_per_row() -> int:
@@ -131,10 +133,12 @@ def make_weights() -> dict:
 class Workload:
     """Weights (shared by all ranks) and this rank's rows, resident on the device."""
 
-    def __init__(self, rows: int, row0: int, device):
+    def __init__(self, rows: int, row0: int, device, fused_mlp: bool = True):
         import torch
         from invariant_bi_matmul_02_b200 import inputs
         self.M = rows
+        self.fused = fused_mlp
+        self.ops = OPS_FUSED if fused_mlp else OPS_UNFUSED
         self.host = make_weights()
         self.x_host = inputs.rows_normal(10, row0, rows, HIDDEN)
         self.dev = {k: v.to(device) for k, v in self.host.items()}
@@ -158,24 +162,33 @@ def run_step(wl: Workload, x, marks=None):
         if marks is not None:
             marks[i].record()
 
+    i = 0
+
+    def step_done():
+        nonlocal i
+        i += 1
+        mark(i)
+
     mark(0)
-    bi.bi_rmsnorm(x, W["g_attn"], EPS, out=B["h1"]); mark(1)
-    bi.bi_addmm(W["b_q"], B["h1"], W["W_q"], "nk", out=B["q"]); mark(2)
-    bi.bi_matmul(B["h1"], W["W_k"], "nk", out=B["k"]); mark(3)
-    bi.bi_matmul(B["h1"], W["W_v"], "nk", out=B["v"]); mark(4)
-    bi.bi_addmm(x, B["q"], W["W_o"], "nk", out=B["o"]); mark(5)
-    bi.bi_rmsnorm(B["o"], W["g_mlp"], EPS, out=B["h2"]); mark(6)
-    bi.bi_matmul(B["h2"], W["W_gu"], "nk", out=B["gu"]); mark(7)
-    bi.bi_silu_mul(B["gu"], out=B["a"]); mark(8)
-    bi.bi_addmm(B["o"], B["a"], W["W_down"], "nk", out=B["y"]); mark(9)
-    bi.bi_rmsnorm(B["y"], W["g_final"], EPS, out=B["hf"]); mark(10)
-    bi.bi_matmul(B["hf"], W["W_lm"], "nk", out=B["lg"]); mark(11)
-    bi.bi_log_softmax(B["lg"], out=B["lp"]); mark(12)
-    bi.bi_mean(B["lp"], out=B["ce"]); mark(13)
+    bi.bi_rmsnorm(x, W["g_attn"], EPS, out=B["h1"]); step_done()
+    bi.bi_addmm(W["b_q"], B["h1"], W["W_q"], "nk", out=B["q"]); step_done()
+    bi.bi_matmul(B["h1"], W["W_k"], "nk", out=B["k"]); step_done()
+    bi.bi_matmul(B["h1"], W["W_v"], "nk", out=B["v"]); step_done()
+    bi.bi_addmm(x, B["q"], W["W_o"], "nk", out=B["o"]); step_done()
+    bi.bi_rmsnorm(B["o"], W["g_mlp"], EPS, out=B["h2"]); step_done()
+    if wl.fused:
+        bi.bi_matmul_silu_mul(B["h2"], W["W_gu"], "nk", out=B["a"]); step_done()
+    else:
+        bi.bi_matmul(B["h2"], W["W_gu"], "nk", out=B["gu"]); step_done()
+        bi.bi_silu_mul(B["gu"], out=B["a"]); step_done()
+    bi.bi_addmm(B["o"], B["a"], W["W_down"], "nk", out=B["y"]); step_done()
+    bi.bi_rmsnorm(B["y"], W["g_final"], EPS, out=B["hf"]); step_done()
+    bi.bi_matmul(B["hf"], W["W_lm"], "nk", out=B["lg"]); step_done()
+    bi.bi_log_softmax(B["lg"], out=B["lp"]); step_done()
+    bi.bi_mean(B["lp"], out=B["ce"]); step_done()
     return B["ce"]
 
 
-LAUNCHES_PER_STEP = len(OPS)
 
 
 # ----------------------------------------------------------------------------- oracle leg
@@ -300,7 +313,8 @@ def run_bi(args):
 
     from invariant_bi_matmul_02_b200.shard import weak_rows
     M = args.rows
-    wl = Workload(M, weak_rows(M, rank)[0], device)
+    wl = Workload(M, weak_rows(M, rank)[0], device, fused_mlp=args.mlp == "fused")
+    OPS = wl.ops
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -373,9 +387,11 @@ def run_bi(args):
     lm_ms = per_op["lm_head"]
     lm_flops = 2 * M * HIDDEN * VOCAB
     achieved = lm_flops / (lm_ms / 1e3) / 1e12
-    gemm_ms = sum(per_op[n] for n, _, _ in GEMMS)
+    gemm_ms = sum(per_op[n] for n in ("q", "k", "v", "o", "gate_up", "gate_up_silu", "down", "lm_head")
+                  if n in per_op)
     row_bytes = row_op_bytes_per_row()
-    row_gbs = {op: round(b * M / (per_op[op] / 1e3) / 1e9, 1) for op, b in row_bytes.items()}
+    row_gbs = {op: round(b * M / (per_op[op] / 1e3) / 1e9, 1) for op, b in row_bytes.items()
+               if op in per_op}
 
     if rank == 0:
         cpu = None
@@ -397,6 +413,8 @@ def run_bi(args):
             "config": {"workload": WORKLOAD, "rows_per_gpu": M, "global_rows": M * world,
                        "hidden": HIDDEN, "kv_out": KV, "ffn": FFN, "vocab": VOCAB,
                        "accumulate": "fp32", "parallelism": f"replicas x{world} (rows sharded)",
+                       "mlp": "gate/up GEMM with SiLU*up in its epilogue" if wl.fused
+                              else "gate/up GEMM, then bi_silu_mul",
                        "l2": "working set ~3 GB > 126 MB L2; no flush",
                        "gemm_tile": bi.bi_gemm_config()},
             "roofline": {"kernel": "bi_matmul LM head launch [%d x 4096] x [4096 x 151936]" % M,
@@ -413,7 +431,7 @@ def run_bi(args):
             "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(wl.x.numel() * 2), "d2h_bytes_per_step": int(M * 4),
                     "steps": e2e_steps},
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches": len(OPS) * args.steps,
             "clocks": clocks,
             "device_status": status,
         }
@@ -570,6 +588,7 @@ KERNEL_CASES = {
     "gemm_gate_up": "bi_matmul M=1024 K=4096 N=24576 (B [N, K])",
     "gemm_lm_head": "bi_matmul M=1024 K=4096 N=151936 (B [N, K])",
     "gemm_qo_m256": "bi_matmul M=256 K=4096 N=4096 (B [N, K])",
+    "gemm_gate_up_silu": "bi_matmul_silu_mul M=1024 K=4096 F=12288 (B [2F, K])",
     "rmsnorm": "bi_rmsnorm M=16384 H=4096 bf16",
     "mean": "bi_mean M=16384 H=4096 fp32",
     "log_softmax": "bi_log_softmax M=1024 V=151936 bf16 -> fp32",
@@ -585,7 +604,13 @@ def run_kernel_case(args):
     from invariant_bi_matmul_02_b200 import inputs
     dev = torch.device("cuda", 0)
     name = args.kernel_case
-    if name.startswith("gemm"):
+    if name == "gemm_gate_up_silu":
+        a = inputs.rows_normal(50, 0, 1024, HIDDEN).to(dev)
+        w = inputs.weight_normal(51, (2 * FFN, HIDDEN)).to(dev)
+        h = torch.empty(1024, FFN, dtype=torch.bfloat16, device=dev)
+        fn = lambda: bi.bi_matmul_silu_mul(a, w, "nk", out=h)
+        work, unit = 2 * 1024 * 2 * FFN * HIDDEN, "TFLOP/s"
+    elif name.startswith("gemm"):
         M, K, N = {"gemm_gate_up": (1024, HIDDEN, 2 * FFN), "gemm_lm_head": (1024, HIDDEN, VOCAB),
                    "gemm_qo_m256": (256, HIDDEN, HIDDEN)}[name]
         a = inputs.rows_normal(50, 0, M, K).to(dev)
@@ -641,6 +666,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--rows", type=int, default=1024, help="token rows per GPU per step")
     ap.add_argument("--impl", choices=["bi", "reference"], default="bi")
+    ap.add_argument("--mlp", choices=["fused", "unfused"], default="fused",
+                    help="gate/up + SiLU*up as one fused GEMM (default) or GEMM then bi_silu_mul")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="per-kernel M sweeps (table, not JSON line)")

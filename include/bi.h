@@ -101,6 +101,26 @@ bi_status bi_addmm(const void *input, int64_t ld_input, const void *A, int64_t l
                    int64_t M, int64_t N, int64_t K, void *stream);
 
 /*
+ * bi_matmul_silu_mul -- H = silu(A . Wg) * (A . Wu): the gate/up projection of a gated MLP
+ * with the SiLU-times-up glue applied in the GEMM's epilogue, so the [M, 2F] gate/up
+ * activations never reach memory.  Elementwise glue after the same batch-invariant
+ * reduction as bi_matmul; not an operation the pages name (the MLP block of the workload).
+ *
+ *   A  device, bf16, [M, K], lda >= K.
+ *   B  device, bf16, the gate and up weights stacked: BI_B_NK: [2F, K] with rows [0, F) the
+ *      gate and rows [F, 2F) the up projection (ldb >= K); BI_B_KN: [K, 2F] with columns
+ *      [0, F) gate and [F, 2F) up (ldb >= 2F).
+ *   H  device, bf16, [M, F], ldh >= F.
+ *   g and u are the fp32 accumulators of bi_matmul (same K order); h = (g / (1 + exp(-g))) * u
+ *   in fp32, one rounding to bf16.  (bi_matmul followed by bi_silu_mul rounds g and u to bf16
+ *   first, so the two paths agree to the bf16 tolerance, not bit for bit.)
+ *   Alignment and limits as bi_matmul; 2F <= 2^31 - 1.  K = 0 writes zeros.
+ */
+bi_status bi_matmul_silu_mul(const void *A, int64_t lda, const void *B, int64_t ldb,
+                             bi_b_layout b_layout, void *H, int64_t ldh, int64_t M, int64_t F,
+                             int64_t K, void *stream);
+
+/*
  * bi_rmsnorm -- y = x * r * w,  r = 1 / sqrt( sum_j x_j^2 / H + eps ), per row.
  * Passage: readhandoff.com agent-run-reproducibility-pinning, "What does temperature
  * zero actually guarantee?" and the FAQ (RMSNorm is one of the kernels whose result

@@ -12,6 +12,7 @@ from .binding import (  # noqa: F401
     bi_get_device_status,
     bi_log_softmax,
     bi_matmul,
+    bi_matmul_silu_mul,
     bi_mean,
     bi_rmsnorm,
     bi_selftest_wait_timeout,

@@ -28,6 +28,8 @@ SIGNATURES = {
                                  _i64, _i64, _i64, _p]),
     "bi_addmm": (ctypes.c_int, [_p, _i64, _p, _i64, _p, _i64, ctypes.c_int, _p, _i64, ctypes.c_int,
                                 _i64, _i64, _i64, _p]),
+    "bi_matmul_silu_mul": (ctypes.c_int, [_p, _i64, _p, _i64, ctypes.c_int, _p, _i64, _i64, _i64, _i64,
+                                          _p]),
     "bi_rmsnorm": (ctypes.c_int, [_p, _p, _p, _i64, _i64, ctypes.c_float, _p]),
     "bi_mean": (ctypes.c_int, [_p, _p, _i64, _i64, _p]),
     "bi_log_softmax": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p]),
@@ -164,6 +166,28 @@ def bi_addmm(input: torch.Tensor, a: torch.Tensor, b: torch.Tensor, b_layout: st
                          BI_B_KN if b_layout == "kn" else BI_B_NK, out.data_ptr(), _ld(out, "C"),
                          _DT[out.dtype], M, N, K, _stream(stream))
     _check("bi_addmm", st)
+    return out
+
+
+def bi_matmul_silu_mul(a: torch.Tensor, b: torch.Tensor, b_layout: str = "nk",
+                       out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """H = silu(A . gate) * (A . up) with B the stacked [gate; up] weight ('nk': [2F, K];
+    'kn': [K, 2F]); the glue runs in the GEMM's epilogue."""
+    _need_cuda(a, "A", (torch.bfloat16,))
+    _need_cuda(b, "B", (torch.bfloat16,))
+    M, N2, K = _gemm_shapes(a, b, b_layout)
+    if N2 % 2:
+        raise ValueError("B must stack gate and up: an even number of output rows")
+    F = N2 // 2
+    if out is None:
+        out = torch.empty((M, F), dtype=torch.bfloat16, device=a.device)
+    _need_cuda(out, "H", (torch.bfloat16,))
+    if tuple(out.shape) != (M, F):
+        raise ValueError("H must be [M, F]")
+    st = load().bi_matmul_silu_mul(a.data_ptr(), _ld(a, "A"), b.data_ptr(), _ld(b, "B"),
+                                   BI_B_KN if b_layout == "kn" else BI_B_NK, out.data_ptr(),
+                                   _ld(out, "H"), M, F, K, _stream(stream))
+    _check("bi_matmul_silu_mul", st)
     return out
 
 

@@ -118,15 +118,18 @@ bi_status encode_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_
 
 bi_status launched() { return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA; }
 
+// N is the number of output columns.  With fuse_silu, B holds 2N rows ([gate; up]) and
+// the output is silu(A . gate^T) * (A . up^T).
 bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, const void *A, int64_t lda,
                       const void *B, int64_t ldb, int b_layout, void *C, int64_t ldc, int c_dtype,
-                      int64_t M, int64_t N, int64_t K, void *stream)
+                      int64_t M, int64_t N, int64_t K, void *stream, int fuse_silu = 0)
 {
     if (M < 0 || N < 0 || K < 0) return BI_ERR_INVALID_ARG;
     if (b_layout != BI_B_KN && b_layout != BI_B_NK) return BI_ERR_INVALID_ARG;
     if (c_dtype != BI_BF16 && c_dtype != BI_F32) return BI_ERR_INVALID_ARG;
-    if (M > kI32Max || N > kI32Max || K > kI32Max) return BI_ERR_UNSUPPORTED;
+    if (M > kI32Max || (fuse_silu ? 2 * N : N) > kI32Max || K > kI32Max) return BI_ERR_UNSUPPORTED;
     if (M == 0 || N == 0) return BI_OK;
+    const int64_t b_rows = fuse_silu ? 2 * N : N;  // extent of B along the output dimension
     if (!C || ldc < N) return BI_ERR_INVALID_ARG;
     if (addend_mode != bi::kAddNone) {
         if (!input || ld_input < 0 || (ld_input != 0 && ld_input < N)) return BI_ERR_INVALID_ARG;
@@ -136,7 +139,7 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
     if (!aligned16(C) || ldc % (c_f32 ? 4 : 8) != 0) return BI_ERR_ALIGNMENT;
     if (K > 0) {
         if (!A || !B) return BI_ERR_INVALID_ARG;
-        if (lda < K || ldb < (b_layout == BI_B_KN ? N : K)) return BI_ERR_INVALID_ARG;
+        if (lda < K || ldb < (b_layout == BI_B_KN ? b_rows : K)) return BI_ERR_INVALID_ARG;
         if (!aligned16(A) || !aligned16(B) || lda % 8 != 0 || ldb % 8 != 0) return BI_ERR_ALIGNMENT;
     }
 
@@ -149,7 +152,8 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
     p.N = (int32_t)N;
     p.K = (int32_t)K;
     p.m_blocks = (int32_t)((M + bi::kPairBM - 1) / bi::kPairBM);
-    p.n_blocks = (int32_t)((N + bi::kPairBN - 1) / bi::kPairBN);
+    p.n_blocks = (int32_t)(fuse_silu ? (N + bi::kHalfBN - 1) / bi::kHalfBN : (N + bi::kPairBN - 1) / bi::kPairBN);
+    p.fuse_silu = fuse_silu;
     p.k_blocks = (int32_t)((K + bi::kBK - 1) / bi::kBK);
     p.b_mn_major = b_layout == BI_B_KN ? 1 : 0;
     p.c_f32 = c_f32 ? 1 : 0;
@@ -162,7 +166,7 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
     p.wait_limit_ns = kWaitLimitNs;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    if (K == 0) {
+    if (K == 0 && !fuse_silu) {
         const int64_t total = M * N;
         int64_t blocks = (total + 255) / 256;
         if (blocks > (int64_t)dev->sms * 16) blocks = (int64_t)dev->sms * 16;
@@ -178,9 +182,9 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
     st = encode_map(&tm_a, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda, bi::kBK, bi::kBM);
     if (st != BI_OK) return st;
     if (b_layout == BI_B_NK)
-        st = encode_map(&tm_b, B, (uint64_t)K, (uint64_t)N, (uint64_t)ldb, bi::kBK, b_rows_box);
+        st = encode_map(&tm_b, B, (uint64_t)K, (uint64_t)b_rows, (uint64_t)ldb, bi::kBK, b_rows_box);
     else
-        st = encode_map(&tm_b, B, (uint64_t)N, (uint64_t)K, (uint64_t)ldb, 64, bi::kBK);
+        st = encode_map(&tm_b, B, (uint64_t)b_rows, (uint64_t)K, (uint64_t)ldb, 64, bi::kBK);
     if (st != BI_OK) return st;
 
     const int64_t pairs = dev->gemm_clusters;
@@ -229,6 +233,17 @@ bi_status bi_addmm(const void *input, int64_t ld_input, const void *A, int64_t l
 {
     return gemm_common(input, ld_input, ld_input == 0 ? bi::kAddBias : bi::kAddMatrix, A, lda, B, ldb,
                        b_layout, C, ldc, c_dtype, M, N, K, stream);
+}
+
+bi_status bi_matmul_silu_mul(const void *A, int64_t lda, const void *B, int64_t ldb,
+                             bi_b_layout b_layout, void *H, int64_t ldh, int64_t M, int64_t F, int64_t K,
+                             void *stream)
+{
+    if (K == 0)  // empty products: silu(0) * 0 = 0
+        return gemm_common(nullptr, 0, bi::kAddNone, A, lda, B, ldb, b_layout, H, ldh, BI_BF16, M, F, 0,
+                           stream, 0);
+    return gemm_common(nullptr, 0, bi::kAddNone, A, lda, B, ldb, b_layout, H, ldh, BI_BF16, M, F, K, stream,
+                       1);
 }
 
 bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H, float eps,

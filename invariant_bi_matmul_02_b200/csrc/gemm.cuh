@@ -26,6 +26,7 @@ struct GemmParams {
     int32_t b_mn_major;     // 1: B stored [K, N] (MN-major operand); 0: B stored [N, K]
     int32_t c_f32;          // 1: C is fp32; 0: C is bf16
     int32_t addend_mode;    // AddendMode
+    int32_t fuse_silu;      // 1: B is [gate; up] (2F rows), C = silu(A.gate^T) * (A.up^T), N = F
     int64_t ldc;
     int64_t ld_addend;
     void *C;
@@ -92,6 +93,16 @@ __device__ __forceinline__ void store_row_chunk(const GemmParams &p, int64_t row
             for (int j = 0; j < 32 && col0 + j < p.N; ++j) dst[j] = __float2bfloat16_rn(v[j]);
         }
     }
+}
+
+// silu(g) * u of one row chunk, fp32 inside, stored as bf16 (columns col0 .. col0+31 of h).
+__device__ __forceinline__ void store_silu_chunk(const GemmParams &p, int64_t row, int64_t col0,
+                                                 const float (&g)[32], const float (&u)[32])
+{
+    float h[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) h[j] = __fmul_rn(g[j] / (1.0f + __expf(-g[j])), u[j]);
+    store_row_chunk(p, row, col0, col0 + 32 <= p.N, h);
 }
 
 // K = 0: the product is empty, so C = input (addmm) or 0.

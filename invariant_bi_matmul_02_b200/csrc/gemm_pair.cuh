@@ -99,8 +99,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_holder;
 
+    // Fused SiLU * up: a pair tile yields kHalfBN columns of h; CTA 0 stages gate rows
+    // n0 .. n0+127 and CTA 1 the up rows F + n0 .. so each CTA's accumulator holds gate in
+    // columns [0, kHalfBN) and up in [kHalfBN, kPairBN) for its 128 rows.
+    const int out_cols = p.fuse_silu ? kHalfBN : kPairBN;
     const int m_blocks = (p.M + kPairBM - 1) / kPairBM;
-    const int n_blocks = (p.N + kPairBN - 1) / kPairBN;
+    const int n_blocks = (p.N + out_cols - 1) / out_cols;
     const int num_tiles = m_blocks * n_blocks;
     const int first = (int)cluster_id_x(), stride = (int)num_clusters_x();
     const uint64_t lim = p.wait_limit_ns;
@@ -112,7 +116,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             bool ok = true;
             for (int tile = first; ok && tile < num_tiles; tile += stride) {
                 const int m0 = (tile % m_blocks) * kPairBM + 128 * (int)rank;
-                const int nh0 = (tile / m_blocks) * kPairBN + kHalfBN * (int)rank;
+                const int nh0 = p.fuse_silu ? (tile / m_blocks) * kHalfBN + (rank ? p.N : 0)
+                                            : (tile / m_blocks) * kPairBN + kHalfBN * (int)rank;
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim)) {
                         ok = false;
@@ -202,10 +207,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             if (!__all_sync(0xffffffffu, ready)) break;
             tc_fence_after_sync();
             const int64_t row = (int64_t)(tile % m_blocks) * kPairBM + 128 * rank + row_in_half;
-            const int64_t n0 = (int64_t)(tile / m_blocks) * kPairBN;
+            const int64_t n0 = (int64_t)(tile / m_blocks) * out_cols;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kPairBN;
 #pragma unroll 1
-            for (int c = 0; c < kPairBN / 32; ++c) {
+            for (int c = 0; p.fuse_silu && c < kHalfBN / 32; ++c) {
+                uint32_t rg[32], ru[32];
+                tmem_load_32x32(t_row + c * 32, rg);
+                tmem_load_32x32(t_row + kHalfBN + c * 32, ru);
+                tmem_wait_ld();
+                const int64_t col0 = n0 + c * 32;
+                if (row < p.M && col0 < p.N) {
+                    float gv[32], uv[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        gv[j] = __uint_as_float(rg[j]);
+                        uv[j] = __uint_as_float(ru[j]);
+                    }
+                    store_silu_chunk(p, row, col0, gv, uv);
+                }
+            }
+#pragma unroll 1
+            for (int c = 0; !p.fuse_silu && c < kPairBN / 32; ++c) {
                 uint32_t r[32];
                 tmem_load_32x32(t_row + c * 32, r);
                 tmem_wait_ld();

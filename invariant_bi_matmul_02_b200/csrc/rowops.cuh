@@ -270,16 +270,24 @@ __global__ void __launch_bounds__(1024, 1) log_softmax_scalar_kernel(const void 
 
 // --------------------------------------------------------------- log_softmax, streamed rows
 
-// Vector path of log_softmax on long rows.  One block of kLsmThreads threads per row,
-// two blocks per SM.  The row streams through a ring of kLsmStages shared-memory chunks of
-// kLsmChunk bytes, each filled by one 1-D bulk copy that completes on its own mbarrier;
-// pass 1 builds the row's (max, sum of exp), pass 2 streams the row again and writes
-// y = (x - max) - log(sum).
+// Vector path of log_softmax.  One block of kLsmThreads threads per row, two blocks per
+// SM.  The row streams through a ring of kLsmStages shared-memory chunks of kLsmChunk
+// bytes, each filled by one 1-D bulk copy that completes on its own mbarrier.  Pass 1
+// builds the row's (max, sum of exp); pass 2 writes y = (x - max) - log(sum), starting
+// with the last chunks of the row, which are still in the ring, and streaming the rest
+// again.  Pass-1 copies ask L2 to keep their lines (they are read again in pass 2),
+// pass-2 copies and the y stores ask it to drop theirs.
 //
 // Element order (fixed by V alone): the row is cut into chunks of kLsmChunk bytes; a chunk
 // into groups of 4 elements; thread t owns groups t, t + T, t + 2T, ... of every chunk and
 // folds them in that order, chunk after chunk.  Consecutive threads read consecutive
 // shared-memory words and write consecutive 16-byte pieces of y.
+//
+// Copy schedule: copy j (j = 0, 1, ...) goes to stage j % S and completes phase j / S of
+// that stage's barrier.  Copies 0 .. n-1 are the n chunks of pass 1; copies n .. n+R-1
+// (R = max(0, n - S)) are chunks 0 .. R-1 again for pass 2.  Chunks R .. n-1 are still in
+// their stages when pass 1 ends and are used by pass 2 without a copy.  A copy is issued
+// once the previous occupant of its stage has been consumed for the last time.
 constexpr int kLsmThreads = 512;
 constexpr int kLsmChunk = 16384;
 constexpr int kLsmStages = 6;
@@ -300,7 +308,9 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
     volatile int *abort_flag = &abort_flag_s;
 
     const int64_t row_bytes = V * kElem;
-    const int nchunks = (int)((row_bytes + kLsmChunk - 1) / kLsmChunk);
+    const int n = (int)((row_bytes + kLsmChunk - 1) / kLsmChunk);
+    const int R = n > kLsmStages ? n - kLsmStages : 0;  // chunks pass 2 must copy again
+    const int copies = n + R;
     const uint8_t *xr = x + (int64_t)blockIdx.x * row_bytes;
     float *yr = y + (int64_t)blockIdx.x * V;
     const int tid = threadIdx.x;
@@ -312,35 +322,32 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
     }
     __syncthreads();
 
-    // Chunk q (0 .. 2*nchunks-1: both passes) goes to stage q % S with parity (q / S) & 1.
-    auto issue = [&](int q) {
-        const int c = q < nchunks ? q : q - nchunks;
+    int issued = 0;  // meaningful in thread 0 only
+    auto issue = [&](int j) {
+        const int c = j < n ? j : j - n;
         const int64_t off = (int64_t)c * kLsmChunk;
         const uint32_t bytes = (uint32_t)(row_bytes - off < kLsmChunk ? row_bytes - off : kLsmChunk);
-        mbar_arrive_expect_tx(&full[q % kLsmStages], bytes);
-        bulk_load(ring[q % kLsmStages], xr + off, bytes, &full[q % kLsmStages]);
+        uint64_t *bar = &full[j % kLsmStages];
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_load_hint(ring[j % kLsmStages], xr + off, bytes, bar,
+                       j < n ? l2_policy_evict_last() : l2_policy_evict_first());
     };
-    const int total = 2 * nchunks;
-    int issued = 0;
     if (tid == 0)
-        for (; issued < kLsmStages && issued < total; ++issued) issue(issued);
+        for (; issued < kLsmStages && issued < n; ++issued) issue(issued);
 
+    // Wait for copy j (all threads agree on the outcome).
+    auto landed = [&](int j) -> bool {
+        const bool ok = wait_bounded(&full[j % kLsmStages], (uint32_t)(j / kLsmStages) & 1u,
+                                     abort_flag, status, wait_limit_ns);
+        return __syncthreads_and(ok ? 1 : 0) != 0;
+    };
+    // Fold or write the chunk held by copy j.
     MaxSum acc{kNegInf, 0.0f};
     float m = 0.0f, ls = 0.0f;
-    int q = 0;
-    for (; q < total; ++q) {
-        const int stage = q % kLsmStages;
-        const bool landed = wait_bounded(&full[stage], (uint32_t)(q / kLsmStages) & 1u, abort_flag,
-                                         status, wait_limit_ns);
-        if (!__syncthreads_and(landed ? 1 : 0)) break;
-        const int c = q < nchunks ? q : q - nchunks;
-        const int64_t e0 = (int64_t)c * kPerChunk;  // first element of this chunk
-        const uint8_t *buf = ring[stage];
-        if (q == nchunks) {
-            const MaxSum row = block_merge(acc, red_m, red_s);
-            m = row.m;
-            ls = __logf(row.s);
-        }
+    auto visit = [&](int j, bool write) {
+        const int c = j < n ? j : j - n;
+        const int64_t e0 = (int64_t)c * kPerChunk;
+        const uint8_t *buf = ring[j % kLsmStages];
         for (int g = tid; g < kGroups; g += kLsmThreads) {
             const int64_t e = e0 + 4 * (int64_t)g;
             if (e >= V) break;
@@ -352,26 +359,53 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
                 const float4 f = *reinterpret_cast<const float4 *>(buf + 16 * g);
                 v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
             }
-            if (q < nchunks) {
+            if (!write) {
                 lsm_accumulate(acc, v);
             } else {
                 __stcs(reinterpret_cast<float4 *>(yr + e),
                        make_float4((v[0] - m) - ls, (v[1] - m) - ls, (v[2] - m) - ls, (v[3] - m) - ls));
             }
         }
+    };
+    // After the last use of copy j's stage, start copy j + S if it exists.
+    auto refill = [&](int j) {
         __syncthreads();  // every thread is done with this stage
-        if (tid == 0 && issued < total) {
+        if (tid == 0 && j + kLsmStages < copies && issued == j + kLsmStages) {
             fence_proxy_async_smem();  // order the reads above before the copy that overwrites
             issue(issued++);
         }
+    };
+
+    bool ok = true;
+    // Pass 1: copies 0 .. n-1.  Stages of the last S chunks are kept for pass 2.
+    for (int j = 0; j < n && ok; ++j) {
+        if (!(ok = landed(j))) break;
+        visit(j, false);
+        if (j + kLsmStages < n) refill(j);
+        else __syncthreads();
     }
-    if (q < total && tid == 0) {
-        // A wait ran out: let the copies still in flight (chunks q .. issued-1, one per
-        // stage) land before the block's shared memory goes away.
-        for (int r = q; r < issued; ++r) {
-            const uint32_t a = smem_addr(&full[r % kLsmStages]);
+    if (ok) {
+        const MaxSum row = block_merge(acc, red_m, red_s);
+        m = row.m;
+        ls = __logf(row.s);
+        // Pass 2, resident chunks R .. n-1 (copies R .. n-1), then copies n .. n+R-1.
+        for (int j = R; j < n; ++j) {
+            visit(j, true);
+            refill(j);
+        }
+        for (int j = n; j < copies && ok; ++j) {
+            if (!(ok = landed(j))) break;
+            visit(j, true);
+            refill(j);
+        }
+    }
+    if (!ok && tid == 0) {
+        // A wait ran out: let every copy already issued land before the block's shared
+        // memory goes away (at most one outstanding copy per stage).
+        for (int j = issued > kLsmStages ? issued - kLsmStages : 0; j < issued; ++j) {
+            const uint32_t a = smem_addr(&full[j % kLsmStages]);
             const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(a, (uint32_t)(r / kLsmStages) & 1u) &&
+            while (!mbar_try_wait(a, (uint32_t)(j / kLsmStages) & 1u) &&
                    global_timer_ns() - t0 < wait_limit_ns) {
             }
         }

@@ -240,6 +240,25 @@ int oracle_silu_mul(const uint16_t *gu, double *h, int64_t M, int64_t F, int nth
     return 0;
 }
 
+/*
+ * The same gated-MLP glue on binary64 inputs: gu is [M, 2F] double (gate columns [0, F),
+ * up columns [F, 2F)), as produced by oracle_matmul without an intermediate rounding.
+ */
+int oracle_silu_mul_f64(const double *gu, double *h, int64_t M, int64_t F, int nthreads)
+{
+    if (M < 0 || F <= 0) return (M == 0 && F >= 0) ? 0 : -1;
+    if (M > 0 && (gu == 0 || h == 0)) return -1;
+#pragma omp parallel for num_threads(threads_or_one(nthreads)) schedule(static)
+    for (int64_t i = 0; i < M; ++i) {
+        for (int64_t j = 0; j < F; ++j) {
+            double g = gu[i * 2 * F + j];
+            double u = gu[i * 2 * F + F + j];
+            h[i * F + j] = g / (1.0 + exp(-g)) * u;
+        }
+    }
+    return 0;
+}
+
 /* Number of OpenMP threads the runtime would use by default (1 without OpenMP). */
 int oracle_max_threads(void)
 {

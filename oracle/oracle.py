@@ -28,7 +28,8 @@ def _lib():
         path = _build.build()
         lib = ctypes.CDLL(path)
         for name in ("oracle_matmul", "oracle_addmm", "oracle_rmsnorm", "oracle_mean_f32",
-                     "oracle_log_softmax_f32", "oracle_log_softmax_bf16", "oracle_silu_mul"):
+                     "oracle_log_softmax_f32", "oracle_log_softmax_bf16", "oracle_silu_mul",
+                     "oracle_silu_mul_f64"):
             getattr(lib, name).restype = ctypes.c_int
         lib.oracle_matmul.argtypes = [_ptr, _i64, _ptr, _i64, ctypes.c_int, _ptr, _i64,
                                       _i64, _i64, _i64, ctypes.c_int]
@@ -39,6 +40,7 @@ def _lib():
         lib.oracle_log_softmax_f32.argtypes = [_ptr, _ptr, _i64, _i64, ctypes.c_int]
         lib.oracle_log_softmax_bf16.argtypes = [_ptr, _ptr, _i64, _i64, ctypes.c_int]
         lib.oracle_silu_mul.argtypes = [_ptr, _ptr, _i64, _i64, ctypes.c_int]
+        lib.oracle_silu_mul_f64.argtypes = [_ptr, _ptr, _i64, _i64, ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -170,3 +172,22 @@ def silu_mul(gu_bits, nthreads=None) -> np.ndarray:
     _check(_lib().oracle_silu_mul(gu.ctypes.data, h.ctypes.data, M, F, _threads(nthreads)),
            "oracle_silu_mul")
     return h
+
+
+def silu_mul_f64(gu, nthreads=None) -> np.ndarray:
+    """h = silu(gate) * up on binary64 gate|up columns (no rounding in between)."""
+    gu = np.ascontiguousarray(_as(gu, np.float64, "gu"))
+    M, F2 = gu.shape
+    if F2 % 2:
+        raise ValueError("gu must have an even number of columns")
+    F = F2 // 2
+    h = np.zeros((M, F), dtype=np.float64)
+    _check(_lib().oracle_silu_mul_f64(gu.ctypes.data, h.ctypes.data, M, F, _threads(nthreads)),
+           "oracle_silu_mul_f64")
+    return h
+
+
+def matmul_silu_mul(a_bits, b_bits, b_layout: str = "nk", nthreads=None) -> np.ndarray:
+    """silu(A . gate) * (A . up) with B = [gate; up] (2F outputs), all in binary64."""
+    return silu_mul_f64(matmul(a_bits, b_bits, b_layout, nthreads), nthreads)
+

@@ -331,6 +331,24 @@ def test_silu_mul_halves_and_linearity_in_up():
     assert not np.allclose(swapped, h)
 
 
+def test_silu_mul_f64_matches_bf16_version_on_exact_inputs():
+    gu = inputs.rows_normal(33, 0, 4, 2 * 96, std=2.0)
+    assert np.array_equal(oracle.silu_mul_f64(gu.double().numpy()), oracle.silu_mul(bits(gu)))
+
+
+def test_matmul_silu_mul_composes_the_definitions():
+    """Fused gate/up + glue: integer A, B make g and u exact, so h is the closed form of exact g, u."""
+    M, K, F = 3, 32, 16
+    a = inputs.rows_int(34, 0, M, K)
+    w = inputs.weight_int(35, (2 * F, K))
+    gu = py_matmul(ints(a).tolist(), ints(w).T.tolist())
+    h = oracle.matmul_silu_mul(bits(a), bits(w), "nk")
+    for i in range(M):
+        for j in range(F):
+            g, u = gu[i][j], gu[i][F + j]
+            assert math.isclose(h[i, j], g / (1 + math.exp(-g)) * u, rel_tol=1e-15, abs_tol=1e-300)
+
+
 def test_oracle_rejects_bad_shapes():
     with pytest.raises(ValueError):
         oracle.matmul(np.zeros((2, 3), np.uint16), np.zeros((4, 5), np.uint16), "kn")
