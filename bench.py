@@ -569,13 +569,16 @@ def run_sweep(args):
             y = torch.empty(M, VOCAB, dtype=torch.float32, device=dev)
             by = 6 * VOCAB * M
             t_bi = _timed(lambda: bi.bi_log_softmax(x, out=y), flush, reps)
-            t_t = _timed(lambda: torch.log_softmax(x.float(), -1), flush, reps)
-            out["rows"].append({"op": "log_softmax", "M": M, "bi_us": t_bi * 1e3, "bi_gbs": by / t_bi / 1e6,
-                                "bi_frac_hbm": by / t_bi / 1e6 / peaks["hbm_gbs"],
-                                "torch_us": t_t * 1e3, "torch_gbs": by / t_t / 1e6})
-            print(f"{'log_softmax':12s} {M:6d} {t_bi*1e3:9.1f} {by/t_bi/1e6:8.0f} "
-                  f"{100*by/t_bi/1e6/peaks['hbm_gbs']:5.1f}% {t_t*1e3:9.1f} {by/t_t/1e6:10.0f}",
-                  flush=True)
+            t_t = _timed(lambda: torch.log_softmax(x, -1, dtype=torch.float32), flush, reps)
+            scr = torch.empty(bi.bi_log_softmax_split_scratch_bytes(M, VOCAB), dtype=torch.uint8, device=dev)
+            t_sp = _timed(lambda: bi.bi_log_softmax_split(x, scr, out=y), flush, reps)
+            for op, t in (("log_softmax", t_bi), ("log_softmax_split", t_sp)):
+                out["rows"].append({"op": op, "M": M, "bi_us": t * 1e3, "bi_gbs": by / t / 1e6,
+                                    "bi_frac_hbm": by / t / 1e6 / peaks["hbm_gbs"],
+                                    "torch_us": t_t * 1e3, "torch_gbs": by / t_t / 1e6})
+                print(f"{op:12s} {M:6d} {t*1e3:9.1f} {by/t/1e6:8.0f} "
+                      f"{100*by/t/1e6/peaks['hbm_gbs']:5.1f}% {t_t*1e3:9.1f} {by/t_t/1e6:10.0f}",
+                      flush=True)
     if args.sweep_out:
         with open(args.sweep_out, "w") as f:
             json.dump(out, f, indent=1)

@@ -44,6 +44,7 @@
 #ifndef BI_H
 #define BI_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -158,6 +159,28 @@ bi_status bi_mean(const float *x, float *y, int64_t M, int64_t H, void *stream);
  */
 bi_status bi_log_softmax(const void *x, bi_dtype x_dtype, float *y, int64_t M, int64_t V,
                          void *stream);
+
+/*
+ * bi_log_softmax_split -- the same y as bi_log_softmax, computed by many blocks per row, for
+ * short batches (decode-time sampling) where one block per row leaves most SMs idle.
+ * Passage: as bi_log_softmax.  The row is cut into chunks of 4096 elements, a cut fixed by V
+ * alone; each chunk is reduced to a (max, sum of exp) partial, and every block of the row
+ * merges the row's partials in one fixed tree before writing its chunk.  The result is
+ * batch-invariant; it is a different fixed order from bi_log_softmax's, so the two agree to
+ * the tolerance, not bit for bit.
+ *
+ *   x, x_dtype, y, M, V as bi_log_softmax; V must be a multiple of 8 (else
+ *   BI_ERR_UNSUPPORTED), x and y 16-byte aligned; M <= 65535.
+ *   scratch  device memory owned by the caller, 16-byte aligned, at least
+ *            bi_log_softmax_split_scratch_bytes(M, V) bytes; overwritten by the call (two
+ *            launches on `stream`), so calls that overlap on the GPU need separate scratch.
+ *   Too small a scratch returns BI_ERR_INVALID_ARG.
+ */
+bi_status bi_log_softmax_split(const void *x, bi_dtype x_dtype, float *y, int64_t M, int64_t V,
+                               void *scratch, size_t scratch_bytes, void *stream);
+
+/* Bytes of scratch bi_log_softmax_split needs for M rows of V elements (0 if M or V <= 0). */
+size_t bi_log_softmax_split_scratch_bytes(int64_t M, int64_t V);
 
 /*
  * bi_silu_mul -- h_ij = silu(g_ij) * u_ij with g = gu[:, 0:F], u = gu[:, F:2F],

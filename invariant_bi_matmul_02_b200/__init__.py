@@ -11,6 +11,8 @@ from .binding import (  # noqa: F401
     bi_gemm_config,
     bi_get_device_status,
     bi_log_softmax,
+    bi_log_softmax_split,
+    bi_log_softmax_split_scratch_bytes,
     bi_matmul,
     bi_matmul_silu_mul,
     bi_mean,

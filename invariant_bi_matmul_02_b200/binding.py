@@ -33,6 +33,8 @@ SIGNATURES = {
     "bi_rmsnorm": (ctypes.c_int, [_p, _p, _p, _i64, _i64, ctypes.c_float, _p]),
     "bi_mean": (ctypes.c_int, [_p, _p, _i64, _i64, _p]),
     "bi_log_softmax": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p]),
+    "bi_log_softmax_split": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p, ctypes.c_size_t, _p]),
+    "bi_log_softmax_split_scratch_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "bi_silu_mul": (ctypes.c_int, [_p, _p, _i64, _i64, _p]),
     "bi_get_device_status": (ctypes.c_int, [_p, ctypes.POINTER(_i32)]),
     "bi_selftest_wait_timeout": (ctypes.c_int, [_i64, _p]),
@@ -234,6 +236,32 @@ def bi_log_softmax(x: torch.Tensor, out: torch.Tensor | None = None, stream=None
     _contig(out, "y")
     _check("bi_log_softmax", load().bi_log_softmax(x.data_ptr(), _DT[x.dtype], out.data_ptr(), M, V,
                                                    _stream(stream)))
+    return out
+
+
+def bi_log_softmax_split_scratch_bytes(M: int, V: int) -> int:
+    return int(load().bi_log_softmax_split_scratch_bytes(int(M), int(V)))
+
+
+def bi_log_softmax_split(x: torch.Tensor, scratch: torch.Tensor | None = None,
+                         out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """log_softmax over the last dimension by many blocks per row (short batches).
+    `scratch` is caller-owned device memory of at least bi_log_softmax_split_scratch_bytes."""
+    _need_cuda(x, "x", (torch.float32, torch.bfloat16))
+    _contig(x, "x")
+    M, V = x.shape
+    if out is None:
+        out = torch.empty((M, V), dtype=torch.float32, device=x.device)
+    _need_cuda(out, "y", (torch.float32,))
+    _contig(out, "y")
+    need = bi_log_softmax_split_scratch_bytes(M, V)
+    if scratch is None:
+        scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    if not scratch.is_cuda:
+        raise ValueError("scratch must be device memory")
+    nbytes = scratch.numel() * scratch.element_size()
+    _check("bi_log_softmax_split", load().bi_log_softmax_split(
+        x.data_ptr(), _DT[x.dtype], out.data_ptr(), M, V, scratch.data_ptr(), nbytes, _stream(stream)))
     return out
 
 

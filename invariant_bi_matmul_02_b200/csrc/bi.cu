@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cstddef>
 #include <cstdint>
 #include <mutex>
 
@@ -324,6 +325,37 @@ bi_status bi_log_softmax(const void *x, bi_dtype x_dtype, float *y, int64_t M, i
             bi::log_softmax_scalar_kernel<true><<<(unsigned)M, T, 0, s>>>(x, y, V);
         else
             bi::log_softmax_scalar_kernel<false><<<(unsigned)M, T, 0, s>>>(x, y, V);
+    }
+    return launched();
+}
+
+size_t bi_log_softmax_split_scratch_bytes(int64_t M, int64_t V)
+{
+    if (M <= 0 || V <= 0) return 0;
+    return (size_t)M * (size_t)bi::split_chunks(V) * sizeof(float2);
+}
+
+bi_status bi_log_softmax_split(const void *x, bi_dtype x_dtype, float *y, int64_t M, int64_t V, void *scratch,
+                               size_t scratch_bytes, void *stream)
+{
+    if (M < 0 || V < 0) return BI_ERR_INVALID_ARG;
+    if (x_dtype != BI_BF16 && x_dtype != BI_F32) return BI_ERR_INVALID_ARG;
+    if (M > 65535 || V > kI32Max) return BI_ERR_UNSUPPORTED;  // rows on grid.y
+    if (M == 0) return BI_OK;
+    if (V == 0 || !x || !y || !scratch) return BI_ERR_INVALID_ARG;
+    if (V % 8 != 0) return BI_ERR_UNSUPPORTED;
+    if (scratch_bytes < bi_log_softmax_split_scratch_bytes(M, V)) return BI_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(scratch)) return BI_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const dim3 grid((unsigned)bi::split_chunks(V), (unsigned)M);
+    const uint8_t *xb = static_cast<const uint8_t *>(x);
+    float2 *part = static_cast<float2 *>(scratch);
+    if (x_dtype == BI_BF16) {
+        bi::log_softmax_split_stats_kernel<true><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, V);
+        bi::log_softmax_split_write_kernel<true><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, y, V);
+    } else {
+        bi::log_softmax_split_stats_kernel<false><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, V);
+        bi::log_softmax_split_write_kernel<false><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, y, V);
     }
     return launched();
 }

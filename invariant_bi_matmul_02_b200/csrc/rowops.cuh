@@ -414,6 +414,94 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
 
 constexpr int kLsmSmem = kLsmStages * kLsmChunk;
 
+// --------------------------------------------------------------- log_softmax, split rows
+
+// Fixed-chunk multi-block variant for short batches.  The row is cut into chunks of
+// kSplitChunk elements (a constant, so the cut depends on V alone); block (c, i) reduces
+// chunk c of row i to a (max, sum of exp) partial, then, in a second launch, every block
+// of row i merges the row's partials in the same fixed tree and writes its chunk of y.
+// Within a chunk, thread t owns the 8-element groups t, t + T, ... in that order.
+// Partials live in caller-provided scratch: one float2 (max, sum) per (row, chunk).
+constexpr int kSplitThreads = 256;
+constexpr int kSplitChunk = 4096;  // elements per chunk
+
+__host__ __device__ inline int64_t split_chunks(int64_t V) { return (V + kSplitChunk - 1) / kSplitChunk; }
+
+template <bool BF16>
+__device__ __forceinline__ void split_load8(const uint8_t *row, int64_t e, float (&v)[8])
+{
+    if (BF16) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(row + 2 * e));
+        v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+        v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+    } else {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(row + 4 * e));
+        const float4 b = __ldg(reinterpret_cast<const float4 *>(row + 4 * e) + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+}
+
+// Launch 1: grid (chunks, M).  V % 8 == 0, x 16-byte aligned.
+template <bool BF16>
+__global__ void __launch_bounds__(kSplitThreads) log_softmax_split_stats_kernel(
+    const uint8_t *__restrict__ x, float2 *__restrict__ partial, int64_t V)
+{
+    __shared__ float red_m[32], red_s[32];
+    constexpr int kElem = BF16 ? 2 : 4;
+    const int64_t nch = split_chunks(V);
+    const int64_t row = blockIdx.y, c = blockIdx.x;
+    const uint8_t *xr = x + row * V * kElem;
+    const int64_t e0 = c * kSplitChunk;
+    MaxSum acc{kNegInf, 0.0f};
+    for (int g = threadIdx.x; g < kSplitChunk / 8; g += kSplitThreads) {
+        const int64_t e = e0 + 8 * (int64_t)g;
+        if (e >= V) break;
+        float v[8];
+        split_load8<BF16>(xr, e, v);
+        lsm_accumulate(acc, v);
+    }
+    const MaxSum part = block_merge(acc, red_m, red_s);
+    if (threadIdx.x == 0) partial[row * nch + c] = make_float2(part.m, part.s);
+}
+
+// Launch 2: grid (chunks, M).  Merge the row's partials (lane l folds chunks l, l+32, ...
+// in order, then a fixed xor butterfly), then write y for this block's chunk.
+template <bool BF16>
+__global__ void __launch_bounds__(kSplitThreads) log_softmax_split_write_kernel(
+    const uint8_t *__restrict__ x, const float2 *__restrict__ partial, float *__restrict__ y, int64_t V)
+{
+    __shared__ float row_stats[2];
+    constexpr int kElem = BF16 ? 2 : 4;
+    const int64_t nch = split_chunks(V);
+    const int64_t row = blockIdx.y, c = blockIdx.x;
+    if (threadIdx.x < 32) {
+        MaxSum acc{kNegInf, 0.0f};
+        for (int64_t k = threadIdx.x; k < nch; k += 32) {
+            const float2 pk = partial[row * nch + k];
+            acc = merge(acc, MaxSum{pk.x, pk.y});
+        }
+        acc = warp_merge(acc);
+        if (threadIdx.x == 0) {
+            row_stats[0] = acc.m;
+            row_stats[1] = __logf(acc.s);
+        }
+    }
+    __syncthreads();
+    const float m = row_stats[0], ls = row_stats[1];
+    const uint8_t *xr = x + row * V * kElem;
+    float *yr = y + row * V;
+    const int64_t e0 = c * kSplitChunk;
+    for (int g = threadIdx.x; g < kSplitChunk / 8; g += kSplitThreads) {
+        const int64_t e = e0 + 8 * (int64_t)g;
+        if (e >= V) break;
+        float v[8];
+        split_load8<BF16>(xr, e, v);
+        float4 *dst = reinterpret_cast<float4 *>(yr + e);
+        __stcs(dst, make_float4((v[0] - m) - ls, (v[1] - m) - ls, (v[2] - m) - ls, (v[3] - m) - ls));
+        __stcs(dst + 1, make_float4((v[4] - m) - ls, (v[5] - m) - ls, (v[6] - m) - ls, (v[7] - m) - ls));
+    }
+}
+
 // --------------------------------------------------------------- SiLU * up
 
 __device__ __forceinline__ float silu_mul1(float g, float u)
