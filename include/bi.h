@@ -183,6 +183,30 @@ bi_status bi_log_softmax_split(const void *x, bi_dtype x_dtype, float *y, int64_
 size_t bi_log_softmax_split_scratch_bytes(int64_t M, int64_t V);
 
 /*
+ * bi_log_softmax_split_noalloc -- bi_log_softmax_split for callers that cannot allocate
+ * device memory at call time: ones working inside a device-memory budget reserved up front
+ * by a pool they do not own, plugins whose host framework controls every allocation, or hot
+ * paths that cannot afford the synchronisation a cudaMalloc implies.  The paper has no
+ * counterpart; this is a library convenience.
+ *
+ * The per-(row, chunk) partials live in a fixed array inside libbi.so's device image (512 KiB,
+ * 65536 partials) instead of caller scratch.  Every GPU that loads the library holds that
+ * array until the process exits; no call allocates or frees anything.
+ *
+ *   x, x_dtype, y, M, V as bi_log_softmax_split (V a multiple of 8, 16-byte aligned x and y,
+ *   M <= 65535).  Limit: M * ceil(V / 4096) <= 65536 (e.g. M <= 1724 rows at V = 151936);
+ *   larger calls return BI_ERR_UNSUPPORTED without launching.
+ *   The result is the same as bi_log_softmax_split's for the same input.
+ *   The first call on a device looks up the array's device address (once per device, with
+ *   that device current); make that first call before capturing any stream.
+ *   All calls on a device share the one array, and it keeps the last call's partials (every
+ *   call overwrites all the partials it reads, so nothing has to start at zero).  Calls that
+ *   overlap on the GPU -- on different streams without ordering between them -- race on it.
+ */
+bi_status bi_log_softmax_split_noalloc(const void *x, bi_dtype x_dtype, float *y, int64_t M,
+                                       int64_t V, void *stream);
+
+/*
  * bi_silu_mul -- h_ij = silu(g_ij) * u_ij with g = gu[:, 0:F], u = gu[:, F:2F],
  * silu(g) = g / (1 + exp(-g)).  Elementwise glue of a gated MLP (no reduction, so
  * batch-invariant by construction); not an operation the pages name.

@@ -35,6 +35,7 @@ SIGNATURES = {
     "bi_log_softmax": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p]),
     "bi_log_softmax_split": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p, ctypes.c_size_t, _p]),
     "bi_log_softmax_split_scratch_bytes": (ctypes.c_size_t, [_i64, _i64]),
+    "bi_log_softmax_split_noalloc": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p]),
     "bi_silu_mul": (ctypes.c_int, [_p, _p, _i64, _i64, _p]),
     "bi_get_device_status": (ctypes.c_int, [_p, ctypes.POINTER(_i32)]),
     "bi_selftest_wait_timeout": (ctypes.c_int, [_i64, _p]),
@@ -262,6 +263,21 @@ def bi_log_softmax_split(x: torch.Tensor, scratch: torch.Tensor | None = None,
     nbytes = scratch.numel() * scratch.element_size()
     _check("bi_log_softmax_split", load().bi_log_softmax_split(
         x.data_ptr(), _DT[x.dtype], out.data_ptr(), M, V, scratch.data_ptr(), nbytes, _stream(stream)))
+    return out
+
+
+def bi_log_softmax_split_noalloc(x: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+    """bi_log_softmax_split with its partials in the library's fixed device array, for callers
+    that cannot allocate device memory when they call it; `out` must be given."""
+    _need_cuda(x, "x", (torch.float32, torch.bfloat16))
+    _contig(x, "x")
+    _need_cuda(out, "y", (torch.float32,))
+    _contig(out, "y")
+    M, V = x.shape
+    if tuple(out.shape) != (M, V):
+        raise ValueError("y must be [M, V]")
+    _check("bi_log_softmax_split_noalloc", load().bi_log_softmax_split_noalloc(
+        x.data_ptr(), _DT[x.dtype], out.data_ptr(), M, V, _stream(stream)))
     return out
 
 

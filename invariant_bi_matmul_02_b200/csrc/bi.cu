@@ -360,6 +360,76 @@ bi_status bi_log_softmax_split(const void *x, bi_dtype x_dtype, float *y, int64_
     return launched();
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// Allocation-free split log_softmax.
+//
+// Some callers cannot hand the library a scratch buffer because they cannot allocate device
+// memory when they call it: code that runs under a memory budget fixed at start-up (every
+// byte already reserved by a pool it does not own), plugins living inside a host framework
+// that controls all device allocation, or callers on a hot path where a cudaMalloc's
+// implicit synchronisation is not acceptable.  For them the partials of the split path live
+// in this file-scope device array.  It has a fixed size and is part of the module image, so
+// every GPU that loads libbi.so holds it until the process exits, and no call allocates.
+namespace {
+
+constexpr int64_t kNoAllocPartials = 65536;  // (row, chunk) partials: 512 KiB per device
+static __device__ __align__(256) float2 g_noalloc_partials[kNoAllocPartials];
+
+std::mutex g_noalloc_mu;
+float2 *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_partials on the current device.  In host code the array's name
+// only stands in for the symbol, so its address is looked up once per device, with that device
+// current, and cached.
+bi_status noalloc_partials(float2 **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BI_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return BI_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_partials) != cudaSuccess || !p) return BI_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<float2 *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return BI_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+bi_status bi_log_softmax_split_noalloc(const void *x, bi_dtype x_dtype, float *y, int64_t M, int64_t V,
+                                       void *stream)
+{
+    if (M < 0 || V < 0) return BI_ERR_INVALID_ARG;
+    if (x_dtype != BI_BF16 && x_dtype != BI_F32) return BI_ERR_INVALID_ARG;
+    if (M > 65535 || V > kI32Max) return BI_ERR_UNSUPPORTED;
+    if (M == 0) return BI_OK;
+    if (V == 0 || !x || !y) return BI_ERR_INVALID_ARG;
+    if (V % 8 != 0) return BI_ERR_UNSUPPORTED;
+    if (M * bi::split_chunks(V) > kNoAllocPartials) return BI_ERR_UNSUPPORTED;  // beyond the fixed array
+    if (!aligned16(x) || !aligned16(y)) return BI_ERR_ALIGNMENT;
+    float2 *part = nullptr;
+    bi_status st = noalloc_partials(&part);
+    if (st != BI_OK) return st;
+    // Launch 1 overwrites every partial that launch 2 reads, so nothing needs clearing.
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const dim3 grid((unsigned)bi::split_chunks(V), (unsigned)M);
+    const uint8_t *xb = static_cast<const uint8_t *>(x);
+    if (x_dtype == BI_BF16) {
+        bi::log_softmax_split_stats_kernel<true><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, V);
+        bi::log_softmax_split_write_kernel<true><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, y, V);
+    } else {
+        bi::log_softmax_split_stats_kernel<false><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, V);
+        bi::log_softmax_split_write_kernel<false><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, y, V);
+    }
+    return launched();
+}
+
 bi_status bi_silu_mul(const void *gu, void *h, int64_t M, int64_t F, void *stream)
 {
     if (M < 0 || F < 0) return BI_ERR_INVALID_ARG;
