@@ -259,6 +259,57 @@ int oracle_silu_mul_f64(const double *gu, double *h, int64_t M, int64_t F, int n
     return 0;
 }
 
+/*
+ * Decode attention (one query token per sequence), grouped-query heads.
+ *   q  [B, Hq, D]          bf16
+ *   k  [B, Lmax, Hkv, D]   bf16 (key cache), v likewise (value cache)
+ *   lens[b] in 1 .. Lmax   tokens of sequence b
+ * Query head h reads kv head h / (Hq / Hkv).  For each (b, h):
+ *   s_t = scale * sum_d q[d] * k[t][d]             t < lens[b]
+ *   p_t = exp(s_t - max_t s_t)
+ *   o_d = (sum_t p_t * v[t][d]) / (sum_t p_t)
+ * (softmax attention; subtracting the maximum does not change the value).
+ * o is [B, Hq, D] double.
+ */
+int oracle_decode_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *lens,
+                            double *o, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t Lmax,
+                            double scale, int nthreads)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Lmax <= 0 || Hq % Hkv) return B == 0 ? 0 : -1;
+    if (B > 0 && (!q || !k || !v || !lens || !o)) return -1;
+    for (int64_t b = 0; b < B; ++b)
+        if (lens[b] < 1 || lens[b] > Lmax) return -1;
+    const int64_t group = Hq / Hkv;
+#pragma omp parallel for num_threads(threads_or_one(nthreads)) schedule(dynamic)
+    for (int64_t bh = 0; bh < B * Hq; ++bh) {
+        const int64_t b = bh / Hq, h = bh % Hq, g = h / group;
+        const int64_t L = lens[b];
+        const uint16_t *qv = q + (b * Hq + h) * D;
+        double m = -INFINITY;
+        for (int64_t t = 0; t < L; ++t) {
+            const uint16_t *kt = k + ((b * Lmax + t) * Hkv + g) * D;
+            double sdot = 0.0;
+            for (int64_t d = 0; d < D; ++d) sdot += bf16_to_double(qv[d]) * bf16_to_double(kt[d]);
+            const double st = scale * sdot;
+            if (st > m) m = st;
+        }
+        double l = 0.0;
+        double *ov = o + (b * Hq + h) * D;
+        for (int64_t d = 0; d < D; ++d) ov[d] = 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            const uint16_t *kt = k + ((b * Lmax + t) * Hkv + g) * D;
+            const uint16_t *vt = v + ((b * Lmax + t) * Hkv + g) * D;
+            double sdot = 0.0;
+            for (int64_t d = 0; d < D; ++d) sdot += bf16_to_double(qv[d]) * bf16_to_double(kt[d]);
+            const double pt = exp(scale * sdot - m);
+            l += pt;
+            for (int64_t d = 0; d < D; ++d) ov[d] += pt * bf16_to_double(vt[d]);
+        }
+        for (int64_t d = 0; d < D; ++d) ov[d] /= l;
+    }
+    return 0;
+}
+
 /* Number of OpenMP threads the runtime would use by default (1 without OpenMP). */
 int oracle_max_threads(void)
 {

@@ -41,6 +41,9 @@ def _lib():
         lib.oracle_log_softmax_bf16.argtypes = [_ptr, _ptr, _i64, _i64, ctypes.c_int]
         lib.oracle_silu_mul.argtypes = [_ptr, _ptr, _i64, _i64, ctypes.c_int]
         lib.oracle_silu_mul_f64.argtypes = [_ptr, _ptr, _i64, _i64, ctypes.c_int]
+        lib.oracle_decode_attention.restype = ctypes.c_int
+        lib.oracle_decode_attention.argtypes = [_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _i64, _i64,
+                                                ctypes.c_double, ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
         _LIB = lib
     return _LIB
@@ -190,4 +193,22 @@ def silu_mul_f64(gu, nthreads=None) -> np.ndarray:
 def matmul_silu_mul(a_bits, b_bits, b_layout: str = "nk", nthreads=None) -> np.ndarray:
     """silu(A . gate) * (A . up) with B = [gate; up] (2F outputs), all in binary64."""
     return silu_mul_f64(matmul(a_bits, b_bits, b_layout, nthreads), nthreads)
+
+
+def decode_attention(q_bits, k_bits, v_bits, lens, scale: float, nthreads=None) -> np.ndarray:
+    """Softmax attention of one query token per sequence over its first lens[b] cached tokens.
+    q [B, Hq, D], k and v [B, Lmax, Hkv, D] as bf16 bits; query head h reads kv head h // (Hq/Hkv)."""
+    q = np.ascontiguousarray(_as(q_bits, np.uint16, "q"))
+    k = np.ascontiguousarray(_as(k_bits, np.uint16, "k"))
+    v = np.ascontiguousarray(_as(v_bits, np.uint16, "v"))
+    lens = np.ascontiguousarray(np.asarray(lens, dtype=np.int32))
+    B, Hq, D = q.shape
+    Bk, Lmax, Hkv, Dk = k.shape
+    if Bk != B or Dk != D or v.shape != k.shape or lens.shape != (B,):
+        raise ValueError("shape mismatch")
+    o = np.zeros((B, Hq, D), dtype=np.float64)
+    _check(_lib().oracle_decode_attention(q.ctypes.data, k.ctypes.data, v.ctypes.data, lens.ctypes.data,
+                                          o.ctypes.data, B, Hq, Hkv, D, Lmax, float(scale),
+                                          _threads(nthreads)), "oracle_decode_attention")
+    return o
 
