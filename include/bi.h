@@ -217,6 +217,42 @@ bi_status bi_log_softmax_split_noalloc(const void *x, bi_dtype x_dtype, float *y
 bi_status bi_silu_mul(const void *gu, void *h, int64_t M, int64_t F, void *stream);
 
 /*
+ * bi_decode_attention -- one decode step of softmax attention with grouped-query heads:
+ * for each sequence b and query head h (reading kv head h / (Hq / Hkv)),
+ *   s_t = scale * q[b,h,:] . k[b,t,g,:],  p = softmax over t < seq_lens[b],  out[b,h,:] = sum_t p_t v[b,t,g,:].
+ * Passage: trustbutveri.fyi "Evidence & limits", Evidence and Limitations (SGLang wrote
+ * batch-invariant attention kernels; an improved attention kernel took the deterministic
+ * Qwen3-8B run from 55 s to 42 s); readhandoff.com agent-run-reproducibility-pinning,
+ * "What does temperature zero actually guarantee?" (attention is not batch-invariant by
+ * default).
+ *
+ * Batch invariance: each sequence's cache is cut into splits of 128 tokens, a cut fixed by
+ * its own length (never by the batch size or the GPU's occupancy, unlike split-KV decoding
+ * that sizes splits to fill the machine).  Per split, scores are fp32 dot products over D in
+ * ascending order, the split's max and sum of exp(s - max) come from fixed trees, and the
+ * weighted value sums run over tokens in ascending order; the splits are then folded in
+ * ascending order.  A sequence's output does not depend on the other sequences in the batch.
+ *
+ *   q        device, bf16, [B, Hq, D];  out device, bf16, [B, Hq, D] (one rounding).
+ *   k_cache, v_cache  device, bf16, [B, Lmax, Hkv, D]; only the first seq_lens[b] tokens of
+ *            sequence b are read.
+ *   seq_lens device, int32, [B], each in 1 .. Lmax.  A value outside is clamped and
+ *            BI_ERR_INVALID_ARG is recorded in the device status word.
+ *   D must be 128 and Hq / Hkv at most 8 (else BI_ERR_UNSUPPORTED); B, Hq, Hkv <= 65535.
+ *   scratch  caller-owned device memory, 16-byte aligned, at least
+ *            bi_decode_attention_scratch_bytes(B, Hq, D, Lmax) bytes; overwritten (two
+ *            launches on `stream`), so overlapping calls need separate scratch.
+ *   q, caches 16-byte aligned; seq_lens 4-byte aligned.
+ */
+bi_status bi_decode_attention(const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *seq_lens, void *out, int64_t B, int64_t Hq, int64_t Hkv,
+                              int64_t D, int64_t Lmax, float scale, void *scratch, size_t scratch_bytes,
+                              void *stream);
+
+/* Bytes of scratch bi_decode_attention needs (0 if any size is <= 0). */
+size_t bi_decode_attention_scratch_bytes(int64_t B, int64_t Hq, int64_t D, int64_t Lmax);
+
+/*
  * bi_get_device_status -- synchronise `stream`, then read and clear the current
  * device's status word.  *out receives BI_OK or the first error a kernel recorded
  * since the last read (BI_ERR_TIMEOUT for a bounded wait that ran out).

@@ -8,6 +8,8 @@ libbi.so is loaded on the first call into ``binding``.
 from .binding import (  # noqa: F401
     BiError,
     bi_addmm,
+    bi_decode_attention,
+    bi_decode_attention_scratch_bytes,
     bi_gemm_config,
     bi_get_device_status,
     bi_log_softmax,

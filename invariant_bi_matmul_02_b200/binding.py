@@ -37,6 +37,9 @@ SIGNATURES = {
     "bi_log_softmax_split_scratch_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "bi_log_softmax_split_noalloc": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p]),
     "bi_silu_mul": (ctypes.c_int, [_p, _p, _i64, _i64, _p]),
+    "bi_decode_attention": (ctypes.c_int, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, ctypes.c_float,
+                                           _p, ctypes.c_size_t, _p]),
+    "bi_decode_attention_scratch_bytes": (ctypes.c_size_t, [_i64, _i64, _i64, _i64]),
     "bi_get_device_status": (ctypes.c_int, [_p, ctypes.POINTER(_i32)]),
     "bi_selftest_wait_timeout": (ctypes.c_int, [_i64, _p]),
     "bi_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -294,6 +297,39 @@ def bi_silu_mul(gu: torch.Tensor, out: torch.Tensor | None = None, stream=None) 
     _need_cuda(out, "h", (torch.bfloat16,))
     _contig(out, "h")
     _check("bi_silu_mul", load().bi_silu_mul(gu.data_ptr(), out.data_ptr(), M, F, _stream(stream)))
+    return out
+
+
+def bi_decode_attention_scratch_bytes(B: int, Hq: int, D: int, Lmax: int) -> int:
+    return int(load().bi_decode_attention_scratch_bytes(int(B), int(Hq), int(D), int(Lmax)))
+
+
+def bi_decode_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                        seq_lens: torch.Tensor, scale: float | None = None,
+                        scratch: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """One decode step: q [B, Hq, D], caches [B, Lmax, Hkv, D] (bf16), seq_lens [B] int32."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need_cuda(t, n, (torch.bfloat16,))
+        _contig(t, n)
+    _need_cuda(seq_lens, "seq_lens", (torch.int32,))
+    _contig(seq_lens, "seq_lens")
+    B, Hq, D = q.shape
+    Bk, Lmax, Hkv, Dk = k_cache.shape
+    if Bk != B or Dk != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(seq_lens.shape) != (B,):
+        raise ValueError("shape mismatch between q, caches and seq_lens")
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    _need_cuda(out, "out", (torch.bfloat16,))
+    if scratch is None:
+        scratch = torch.empty(max(bi_decode_attention_scratch_bytes(B, Hq, D, Lmax), 16), dtype=torch.uint8,
+                              device=q.device)
+    nbytes = scratch.numel() * scratch.element_size()
+    _check("bi_decode_attention", load().bi_decode_attention(
+        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seq_lens.data_ptr(), out.data_ptr(),
+        B, Hq, Hkv, D, Lmax, float(scale), scratch.data_ptr(), nbytes, _stream(stream)))
     return out
 
 

@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "gemm.cuh"
+#include "attention.cuh"
 #include "gemm_pair.cuh"
 #include "ptx.cuh"
 #include "rowops.cuh"
@@ -74,6 +75,9 @@ bi_status device_state(DeviceState **out)
                 return BI_ERR_CUDA;
             d.gemm_clusters = n;
         }
+        if (cudaFuncSetAttribute(bi::decode_attention_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(bi::AttnSmem)) != cudaSuccess)
+            return BI_ERR_CUDA;
         if (cudaFuncSetAttribute(bi::log_softmax_stream_kernel<true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kLsmSmem) != cudaSuccess ||
             cudaFuncSetAttribute(bi::log_softmax_stream_kernel<false>,
@@ -427,6 +431,45 @@ bi_status bi_log_softmax_split_noalloc(const void *x, bi_dtype x_dtype, float *y
         bi::log_softmax_split_stats_kernel<false><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, V);
         bi::log_softmax_split_write_kernel<false><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, y, V);
     }
+    return launched();
+}
+
+size_t bi_decode_attention_scratch_bytes(int64_t B, int64_t Hq, int64_t D, int64_t Lmax)
+{
+    if (B <= 0 || Hq <= 0 || D <= 0 || Lmax <= 0) return 0;
+    const size_t parts = (size_t)B * (size_t)Hq * (size_t)bi::attn_splits(Lmax);
+    return parts * ((size_t)D * sizeof(float) + sizeof(float2));
+}
+
+bi_status bi_decode_attention(const void *q, const void *k_cache, const void *v_cache, const int32_t *seq_lens,
+                              void *out, int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t Lmax, float scale,
+                              void *scratch, size_t scratch_bytes, void *stream)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Lmax <= 0) return B == 0 ? BI_OK : BI_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return BI_ERR_INVALID_ARG;
+    if (D != bi::kAttnD || Hq / Hkv > bi::kAttnMaxGroup) return BI_ERR_UNSUPPORTED;
+    if (B > 65535 || Hkv > 65535 || Hq > 65535 || bi::attn_splits(Lmax) > kI32Max) return BI_ERR_UNSUPPORTED;
+    if (B == 0) return BI_OK;
+    if (!q || !k_cache || !v_cache || !seq_lens || !out || !scratch) return BI_ERR_INVALID_ARG;
+    if (scratch_bytes < bi_decode_attention_scratch_bytes(B, Hq, D, Lmax)) return BI_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(scratch) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+        return BI_ERR_ALIGNMENT;
+    DeviceState *dev = nullptr;
+    bi_status st = device_state(&dev);
+    if (st != BI_OK) return st;
+    const int64_t S = bi::attn_splits(Lmax);
+    float *part_acc = static_cast<float *>(scratch);
+    float2 *part_ms = reinterpret_cast<float2 *>(part_acc + (size_t)B * Hq * S * D);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const auto *qb = static_cast<const __nv_bfloat16 *>(q);
+    const auto *kb = static_cast<const __nv_bfloat16 *>(k_cache);
+    const auto *vb = static_cast<const __nv_bfloat16 *>(v_cache);
+    bi::decode_attention_split_kernel<<<dim3((unsigned)S, (unsigned)Hkv, (unsigned)B), bi::kAttnThreads,
+                                        sizeof(bi::AttnSmem), s>>>(qb, kb, vb, seq_lens, part_ms, part_acc,
+                                                                   (int)Hq, (int)Hkv, Lmax, scale, dev->status);
+    bi::decode_attention_combine_kernel<<<dim3((unsigned)Hq, (unsigned)B), bi::kAttnD, 0, s>>>(
+        part_ms, part_acc, seq_lens, static_cast<__nv_bfloat16 *>(out), (int)Hq, Lmax);
     return launched();
 }
 

@@ -381,3 +381,21 @@ __device__ __forceinline__ void bulk_load_hint(void *dst, const void *src, uint3
 }
 
 }  // namespace bi
+
+namespace bi {
+
+// 16-byte asynchronous copy global -> shared; copies `src_bytes` (0 or 16) and zero-fills
+// the rest of the 16 bytes.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+}  // namespace bi

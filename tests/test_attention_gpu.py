@@ -1,0 +1,100 @@
+"""bi_decode_attention through the C ABI: parity with the fp64 oracle, and batch invariance.
+
+A sequence's output must be bit-identical whether it is decoded alone or inside batches of
+other sequences of other lengths, at any position, whatever the cache's Lmax stride.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bi_testutil import assert_bf16_close, bf16_bits_np, same_bits
+from invariant_bi_matmul_02_b200 import binding as bi
+from invariant_bi_matmul_02_b200 import inputs
+from oracle import oracle
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+D = 128
+
+
+def make(seed, B, Hq, Hkv, Lmax):
+    q = inputs.rows_normal(seed, 0, B * Hq, D).view(B, Hq, D)
+    k = inputs.rows_normal(seed + 1, 0, B * Lmax * Hkv, D).view(B, Lmax, Hkv, D)
+    v = inputs.rows_normal(seed + 2, 0, B * Lmax * Hkv, D).view(B, Lmax, Hkv, D)
+    return q, k, v
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 8), (16, 2), (8, 1)])
+@pytest.mark.parametrize("lens", [[1, 128, 300], [127, 129, 256, 257], [5]])
+def test_attention_parity(Hq, Hkv, lens):
+    B, Lmax = len(lens), max(lens) + 3
+    q, k, v = make(800, B, Hq, Hkv, Lmax)
+    sl = torch.tensor(lens, dtype=torch.int32)
+    o = bi.bi_decode_attention(q.to(DEV), k.to(DEV), v.to(DEV), sl.to(DEV))
+    ref = oracle.decode_attention(bf16_bits_np(q), bf16_bits_np(k), bf16_bits_np(v), sl.numpy(), D ** -0.5)
+    assert_bf16_close(o, ref, f"attention Hq={Hq} Hkv={Hkv} lens={lens}")
+    assert bi.bi_get_device_status() == bi.BI_OK
+
+
+def test_attention_long_sequences_sampled():
+    B, Hq, Hkv, Lmax = 4, 32, 8, 4096
+    q, k, v = make(801, B, Hq, Hkv, Lmax)
+    sl = torch.tensor([4096, 1, 2049, 3000], dtype=torch.int32)
+    o = bi.bi_decode_attention(q.to(DEV), k.to(DEV), v.to(DEV), sl.to(DEV))
+    ref = oracle.decode_attention(bf16_bits_np(q), bf16_bits_np(k), bf16_bits_np(v), sl.numpy(), D ** -0.5)
+    assert_bf16_close(o, ref, "attention Lmax=4096")
+
+
+def test_attention_batch_invariance_over_compositions():
+    P, Hq, Hkv, Lmax = 48, 32, 8, 1024
+    q, k, v = make(802, P, Hq, Hkv, Lmax)
+    lens = torch.tensor(inputs.batch_sizes(803, P, 1, Lmax), dtype=torch.int32)
+    qd, kd, vd, ld = q.to(DEV), k.to(DEV), v.to(DEV), lens.to(DEV)
+    ref = torch.cat([bi.bi_decode_attention(qd[i:i + 1], kd[i:i + 1], vd[i:i + 1], ld[i:i + 1]) for i in range(P)])
+    for t, b in enumerate(inputs.batch_sizes(804, 20, 1, P)):
+        idx = inputs.permutation(805 + t, P)[:b].to(DEV)
+        lmax = int(lens[idx.cpu()].max())
+        # a batch's cache may be allocated with a smaller Lmax: the stride changes, the bits may not
+        kk = kd[idx][:, :lmax].contiguous()
+        vv = vd[idx][:, :lmax].contiguous()
+        o = bi.bi_decode_attention(qd[idx], kk, vv, ld[idx])
+        assert same_bits(o, ref[idx]), f"trial {t}: batch of {b} changed a sequence's output"
+
+
+def test_attention_repeatable_100_runs():
+    B, Hq, Hkv, Lmax = 16, 32, 8, 700
+    q, k, v = make(806, B, Hq, Hkv, Lmax)
+    sl = torch.tensor(inputs.batch_sizes(807, B, 1, Lmax), dtype=torch.int32).to(DEV)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    scratch = torch.empty(bi.bi_decode_attention_scratch_bytes(B, Hq, D, Lmax), dtype=torch.uint8, device=DEV)
+    first = bi.bi_decode_attention(qd, kd, vd, sl, scratch=scratch)
+    for _ in range(100):
+        assert same_bits(bi.bi_decode_attention(qd, kd, vd, sl, scratch=scratch), first)
+
+
+def test_attention_bad_lengths_are_reported():
+    B, Hq, Hkv, Lmax = 2, 8, 2, 64
+    q, k, v = make(808, B, Hq, Hkv, Lmax)
+    sl = torch.tensor([0, 99], dtype=torch.int32, device=DEV)
+    assert bi.bi_get_device_status() == bi.BI_OK
+    bi.bi_decode_attention(q.to(DEV), k.to(DEV), v.to(DEV), sl)
+    assert bi.bi_get_device_status() == bi.BI_ERR_INVALID_ARG
+
+
+def test_attention_argument_errors():
+    q = torch.zeros(2, 8, 64, dtype=torch.bfloat16, device=DEV)
+    kv = torch.zeros(2, 16, 2, 64, dtype=torch.bfloat16, device=DEV)
+    sl = torch.ones(2, dtype=torch.int32, device=DEV)
+    with pytest.raises(bi.BiError) as e:
+        bi.bi_decode_attention(q, kv, kv, sl)  # D = 64: only D = 128 is built
+    assert e.value.status == bi.BI_ERR_UNSUPPORTED
+    q = torch.zeros(2, 6, D, dtype=torch.bfloat16, device=DEV)
+    kv = torch.zeros(2, 16, 4, D, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(bi.BiError) as e:
+        bi.bi_decode_attention(q, kv, kv, sl)  # 6 query heads over 4 kv heads
+    assert e.value.status == bi.BI_ERR_INVALID_ARG
+    q = torch.zeros(2, 8, D, dtype=torch.bfloat16, device=DEV)
+    kv = torch.zeros(2, 16, 2, D, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(bi.BiError) as e:
+        bi.bi_decode_attention(q, kv, kv, sl, scratch=torch.empty(16, dtype=torch.uint8, device=DEV))
+    assert e.value.status == bi.BI_ERR_INVALID_ARG
