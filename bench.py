@@ -662,6 +662,146 @@ def run_kernel_case(args):
                       "status": bi.bi_get_device_status()}), flush=True)
 
 
+# ----------------------------------------------------------------------------- uniqueness experiment
+
+class ToyDecoder:
+    """A random-weight decoder (Qwen-style blocks without position encoding) used to repeat the
+    pages' experiment in miniature: greedy decoding of one prompt inside many different batch
+    compositions.  `impl` "bi" runs every reduction through libbi.so; "torch" uses torch's
+    default kernels for the same arithmetic."""
+
+    HIDDEN, HQ, HKV, HEAD, FFN_T, VOC, LAYERS = 1024, 8, 2, 128, 2816, 32000, 4
+
+    def __init__(self, device, seed: int = 900):
+        import torch
+        from invariant_bi_matmul_02_b200 import inputs
+        H, F = self.HIDDEN, self.FFN_T
+        w = lambda i, shape, std=0.02: inputs.weight_normal(seed + i, shape, std=std).to(device)
+        self.emb = w(0, (self.VOC, H), std=1.0)
+        self.layers = []
+        for l in range(self.LAYERS):
+            b = 10 * (l + 1)
+            self.layers.append(dict(
+                g1=inputs.gain(seed + b, H).to(device), g2=inputs.gain(seed + b + 1, H).to(device),
+                wq=w(b + 2, (self.HQ * self.HEAD, H)), wk=w(b + 3, (self.HKV * self.HEAD, H)),
+                wv=w(b + 4, (self.HKV * self.HEAD, H)), wo=w(b + 5, (H, self.HQ * self.HEAD)),
+                wgu=w(b + 6, (2 * F, H)), wd=w(b + 7, (H, F))))
+        self.gf = inputs.gain(seed + 99, H).to(device)
+        self.wlm = w(98, (self.VOC, H))
+        self.device = device
+
+    def step(self, impl, tokens, kcache, vcache, pos):
+        """One decode step for a batch: tokens [B] -> next tokens [B]; writes position `pos`
+        of every sequence's cache and attends over positions 0..pos."""
+        import torch
+        import torch.nn.functional as Fn
+        from invariant_bi_matmul_02_b200 import binding as bi
+        B = tokens.shape[0]
+        x = self.emb.index_select(0, tokens)
+        lens = torch.full((B,), pos + 1, dtype=torch.int32, device=self.device)
+        for l, L in enumerate(self.layers):
+            if impl == "bi":
+                h = bi.bi_rmsnorm(x, L["g1"], EPS)
+                q, k, v = (bi.bi_matmul(h, L["wq"]), bi.bi_matmul(h, L["wk"]), bi.bi_matmul(h, L["wv"]))
+            else:
+                h = Fn.rms_norm(x, (self.HIDDEN,), L["g1"], EPS)
+                q, k, v = Fn.linear(h, L["wq"]), Fn.linear(h, L["wk"]), Fn.linear(h, L["wv"])
+            kcache[l][:, pos] = k.view(B, self.HKV, self.HEAD)
+            vcache[l][:, pos] = v.view(B, self.HKV, self.HEAD)
+            if impl == "bi":
+                a = bi.bi_decode_attention(q.view(B, self.HQ, self.HEAD), kcache[l], vcache[l], lens)
+                x = bi.bi_addmm(x, a.view(B, -1), L["wo"])
+                m = bi.bi_matmul_silu_mul(bi.bi_rmsnorm(x, L["g2"], EPS), L["wgu"])
+                x = bi.bi_addmm(x, m, L["wd"])
+            else:
+                kk = kcache[l][:, :pos + 1].transpose(1, 2)
+                vv = vcache[l][:, :pos + 1].transpose(1, 2)
+                a = Fn.scaled_dot_product_attention(q.view(B, self.HQ, 1, self.HEAD), kk, vv, enable_gqa=True)
+                x = x + Fn.linear(a.reshape(B, -1), L["wo"])
+                gu = Fn.linear(Fn.rms_norm(x, (self.HIDDEN,), L["g2"], EPS), L["wgu"])
+                g_, u_ = gu.chunk(2, dim=-1)
+                x = x + Fn.linear(Fn.silu(g_) * u_, L["wd"])
+        if impl == "bi":
+            lp = bi.bi_log_softmax(bi.bi_matmul(bi.bi_rmsnorm(x, self.gf, EPS), self.wlm))
+        else:
+            lp = torch.log_softmax(Fn.linear(Fn.rms_norm(x, (self.HIDDEN,), self.gf, EPS), self.wlm), -1,
+                                   dtype=torch.float32)
+        return lp.argmax(-1), lp
+
+    def generate(self, impl, prompts, new_tokens, watch=None, digest=None):
+        """Greedy decoding of a batch of equal-length prompts [B, P]: returns [B, new_tokens].
+        With `watch` (a row index) and `digest` (a hashlib object), the bits of that row's
+        log-prob vector at every step are fed to the digest."""
+        import torch
+        B, P = prompts.shape
+
+        def step(tok, pos):
+            nxt, lp = self.step(impl, tok, kc, vc, pos)
+            if digest is not None:
+                digest.update(lp[watch].contiguous().view(torch.int32).cpu().numpy().tobytes())
+            return nxt
+        T = P + new_tokens
+        kc = [torch.zeros(B, T, self.HKV, self.HEAD, dtype=torch.bfloat16, device=self.device)
+              for _ in range(self.LAYERS)]
+        vc = [torch.zeros_like(kc[0]) for _ in range(self.LAYERS)]
+        out = []
+        tok = prompts[:, 0]
+        for pos in range(T - 1):
+            nxt = step(tok, pos)
+            if pos + 1 < P:
+                tok = prompts[:, pos + 1]
+            else:
+                out.append(nxt)
+                tok = nxt
+        out.append(step(tok, T - 1))
+        return torch.stack(out, 1)[:, -new_tokens:]
+
+
+def uniqueness(trials: int, new_tokens: int = 32, prompt_len: int = 16, max_batch: int = 64, seed: int = 950,
+               device="cuda"):
+    """Decode one fixed prompt greedily inside `trials` random batch compositions (random batch
+    size 1..max_batch, random position, random other prompts) with each implementation, and
+    count the distinct completions of the fixed prompt and the distinct bit patterns of its
+    log-prob vectors over all steps."""
+    import hashlib
+    import torch
+    from invariant_bi_matmul_02_b200 import inputs
+    model = ToyDecoder(device)
+    g = torch.Generator().manual_seed(seed)
+    target = torch.randint(0, ToyDecoder.VOC, (prompt_len,), generator=g)
+    sizes = inputs.batch_sizes(seed, trials, 1, max_batch)
+    result = {}
+    for impl in ("bi", "torch"):
+        seen, bits = {}, set()
+        for t, b in enumerate(sizes):
+            gt = torch.Generator().manual_seed(seed * 1000 + t)
+            others = torch.randint(0, ToyDecoder.VOC, (b, prompt_len), generator=gt)
+            at = int(torch.randint(0, b, (1,), generator=gt))
+            others[at] = target
+            h = hashlib.sha256()
+            comp = model.generate(impl, others.to(device), new_tokens, watch=at, digest=h)[at].tolist()
+            key = tuple(comp)
+            seen[key] = seen.get(key, 0) + 1
+            bits.add(h.hexdigest())
+        result[impl] = {"unique": len(seen), "most_common": max(seen.values()),
+                        "unique_logprob_bits": len(bits), "trials": trials}
+    return result
+
+
+def run_uniqueness(args):
+    import torch
+    t0 = time.perf_counter()
+    res = uniqueness(args.uniqueness)
+    print(json.dumps({"experiment": "greedy completions of one prompt over random batch compositions",
+                      "model": "random-weight 4-layer decoder, hidden 1024, 8 q / 2 kv heads of 128, "
+                               "ffn 2816, vocab 32000",
+                      "new_tokens": 32, "prompt_len": 16, "batch_sizes": "1..64",
+                      "bi": res["bi"], "torch_default": res["torch"],
+                      "seconds": round(time.perf_counter() - t0, 1),
+                      "status": __import__("invariant_bi_matmul_02_b200").bi_get_device_status()}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -676,6 +816,8 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="per-kernel M sweeps (table, not JSON line)")
     ap.add_argument("--sweep-shapes", default="", help="comma list of sweep groups (q/o,k/v,...,rows)")
     ap.add_argument("--sweep-out", default="", help="write the sweep as JSON to this path")
+    ap.add_argument("--uniqueness", type=int, default=0,
+                    help="run the batch-composition uniqueness experiment with this many trials")
     ap.add_argument("--kernel-case", default="", help="launch one kernel on a fixed case: "
                     + ", ".join(sorted(KERNEL_CASES)))
     args = ap.parse_args()
@@ -686,6 +828,9 @@ def main():
         return
     if args.kernel_case:
         run_kernel_case(args)
+        return
+    if args.uniqueness:
+        run_uniqueness(args)
         return
     if args.impl == "reference":
         run_reference(args)
