@@ -5,12 +5,11 @@ One *step* is one pass of every kernel of the path over a batch of M token rows
 (default 1024) shaped like a Qwen3-8B layer plus its LM head:
 
     h1   = bi_rmsnorm(x, g_attn)                      [M, 4096]    bf16
-    q    = bi_addmm(b_q, h1, W_q)                     [M, 4096]    bias N(0, 0.01)
-    k, v = bi_matmul(h1, W_k), bi_matmul(h1, W_v)     [M, 1024] x 2
-    o    = bi_addmm(x, q, W_o)                        [M, 4096]    residual add
+    qkv  = bi_addmm(b_qkv, h1, [W_q; W_k; W_v])       [M, 6144]    bias N(0, 0.01) on q, 0 on k, v
+    o    = bi_addmm(x, q, W_o)                        [M, 4096]    residual add (q = qkv[:, :4096])
     h2   = bi_rmsnorm(o, g_mlp)
-    gu   = bi_matmul(h2, W_gu)                        [M, 24576]   gate | up
-    a    = bi_silu_mul(gu)                            [M, 12288]
+    a    = bi_matmul_silu_mul(h2, [W_g; W_u])         [M, 12288]   SiLU(gate) * up in the epilogue
+                                                                   (--mlp unfused: bi_matmul, then bi_silu_mul)
     y    = bi_addmm(o, a, W_down)                     [M, 4096]    residual add
     hf   = bi_rmsnorm(y, g_final)
     lg   = bi_matmul(hf, W_lm)                        [M, 151936]  bf16 logits
@@ -48,13 +47,13 @@ HIDDEN, KV, FFN, VOCAB = 4096, 1024, 12288, 151936
 EPS = 1e-6
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# (name, K, N) of the GEMM launches of one step, in order.
+# (name, K, N) of the GEMMs of one step (FLOP accounting; q, k and v run as one launch).
 GEMMS = [("q", HIDDEN, HIDDEN), ("k", HIDDEN, KV), ("v", HIDDEN, KV), ("o", HIDDEN, HIDDEN),
          ("gate_up", HIDDEN, 2 * FFN), ("down", FFN, HIDDEN), ("lm_head", HIDDEN, VOCAB)]
-OPS_UNFUSED = ["rms1", "q", "k", "v", "o", "rms2", "gate_up", "silu_mul", "down", "rms3", "lm_head",
+QKV = HIDDEN + 2 * KV
+OPS_UNFUSED = ["rms1", "qkv", "o", "rms2", "gate_up", "silu_mul", "down", "rms3", "lm_head",
                "log_softmax", "mean"]
-OPS_FUSED = ["rms1", "q", "k", "v", "o", "rms2", "gate_up_silu", "down", "rms3", "lm_head",
-             "log_softmax", "mean"]
+OPS_FUSED = ["rms1", "qkv", "o", "rms2", "gate_up_silu", "down", "rms3", "lm_head", "log_softmax", "mean"]
 
 
 def gemm_flops_per_row() -> int:
@@ -142,11 +141,15 @@ class Workload:
         self.host = make_weights()
         self.x_host = inputs.rows_normal(10, row0, rows, HIDDEN)
         self.dev = {k: v.to(device) for k, v in self.host.items()}
+        # q, k and v as one projection: W_qkv = [W_q; W_k; W_v], bias zero on the k, v columns
+        self.dev["W_qkv"] = torch.cat([self.dev["W_q"], self.dev["W_k"], self.dev["W_v"]]).contiguous()
+        self.dev["b_qkv"] = torch.cat([self.dev["b_q"], torch.zeros(2 * KV, dtype=torch.bfloat16,
+                                                                     device=device)]).contiguous()
         self.x = self.x_host.to(device)
         e = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device=device)
         M = rows
         self.buf = {
-            "h1": e(M, HIDDEN), "q": e(M, HIDDEN), "k": e(M, KV), "v": e(M, KV), "o": e(M, HIDDEN),
+            "h1": e(M, HIDDEN), "qkv": e(M, QKV), "o": e(M, HIDDEN),
             "h2": e(M, HIDDEN), "gu": e(M, 2 * FFN), "a": e(M, FFN), "y": e(M, HIDDEN),
             "hf": e(M, HIDDEN), "lg": e(M, VOCAB), "lp": e(M, VOCAB, dt=torch.float32),
             "ce": e(M, dt=torch.float32),
@@ -171,10 +174,8 @@ def run_step(wl: Workload, x, marks=None):
 
     mark(0)
     bi.bi_rmsnorm(x, W["g_attn"], EPS, out=B["h1"]); step_done()
-    bi.bi_addmm(W["b_q"], B["h1"], W["W_q"], "nk", out=B["q"]); step_done()
-    bi.bi_matmul(B["h1"], W["W_k"], "nk", out=B["k"]); step_done()
-    bi.bi_matmul(B["h1"], W["W_v"], "nk", out=B["v"]); step_done()
-    bi.bi_addmm(x, B["q"], W["W_o"], "nk", out=B["o"]); step_done()
+    bi.bi_addmm(W["b_qkv"], B["h1"], W["W_qkv"], "nk", out=B["qkv"]); step_done()
+    bi.bi_addmm(x, B["qkv"][:, :HIDDEN], W["W_o"], "nk", out=B["o"]); step_done()
     bi.bi_rmsnorm(B["o"], W["g_mlp"], EPS, out=B["h2"]); step_done()
     if wl.fused:
         bi.bi_matmul_silu_mul(B["h2"], W["W_gu"], "nk", out=B["a"]); step_done()
@@ -387,7 +388,7 @@ def run_bi(args):
     lm_ms = per_op["lm_head"]
     lm_flops = 2 * M * HIDDEN * VOCAB
     achieved = lm_flops / (lm_ms / 1e3) / 1e12
-    gemm_ms = sum(per_op[n] for n in ("q", "k", "v", "o", "gate_up", "gate_up_silu", "down", "lm_head")
+    gemm_ms = sum(per_op[n] for n in ("qkv", "o", "gate_up", "gate_up_silu", "down", "lm_head")
                   if n in per_op)
     row_bytes = row_op_bytes_per_row()
     row_gbs = {op: round(b * M / (per_op[op] / 1e3) / 1e9, 1) for op, b in row_bytes.items()
