@@ -729,28 +729,39 @@ class ToyDecoder:
                                    dtype=torch.float32)
         return lp.argmax(-1), lp
 
-    def generate(self, impl, prompts, new_tokens, watch=None, digest=None):
+    def generate(self, impl, prompts, new_tokens, watch=None, digest=None, context=0, context_seeds=None):
         """Greedy decoding of a batch of equal-length prompts [B, P]: returns [B, new_tokens].
+        With `context` > 0 every sequence starts from `context` cached positions of random keys
+        and values (N(0, 1), drawn on the device from the sequence's seed in `context_seeds`).
         With `watch` (a row index) and `digest` (a hashlib object), the bits of that row's
         log-prob vector at every step are fed to the digest."""
         import torch
         B, P = prompts.shape
+        T = context + P + new_tokens
+        kc = [torch.zeros(B, T, self.HKV, self.HEAD, dtype=torch.bfloat16, device=self.device)
+              for _ in range(self.LAYERS)]
+        vc = [torch.zeros_like(kc[0]) for _ in range(self.LAYERS)]
+        for b in range(B if context else 0):
+            g = torch.Generator(device=self.device)
+            g.manual_seed(int(context_seeds[b]))
+            for l in range(self.LAYERS):
+                for cache in (kc[l], vc[l]):
+                    cache[b, :context] = torch.randn(context, self.HKV, self.HEAD, generator=g,
+                                                     device=self.device).to(torch.bfloat16)
 
         def step(tok, pos):
             nxt, lp = self.step(impl, tok, kc, vc, pos)
             if digest is not None:
                 digest.update(lp[watch].contiguous().view(torch.int32).cpu().numpy().tobytes())
             return nxt
-        T = P + new_tokens
-        kc = [torch.zeros(B, T, self.HKV, self.HEAD, dtype=torch.bfloat16, device=self.device)
-              for _ in range(self.LAYERS)]
-        vc = [torch.zeros_like(kc[0]) for _ in range(self.LAYERS)]
+
         out = []
         tok = prompts[:, 0]
-        for pos in range(T - 1):
+        for i in range(P + new_tokens - 1):
+            pos = context + i
             nxt = step(tok, pos)
-            if pos + 1 < P:
-                tok = prompts[:, pos + 1]
+            if i + 1 < P:
+                tok = prompts[:, i + 1]
             else:
                 out.append(nxt)
                 tok = nxt
@@ -759,7 +770,7 @@ class ToyDecoder:
 
 
 def uniqueness(trials: int, new_tokens: int = 32, prompt_len: int = 16, max_batch: int = 64, seed: int = 950,
-               device="cuda"):
+               device="cuda", context: int = 0):
     """Decode one fixed prompt greedily inside `trials` random batch compositions (random batch
     size 1..max_batch, random position, random other prompts) with each implementation, and
     count the distinct completions of the fixed prompt and the distinct bit patterns of its
@@ -779,8 +790,11 @@ def uniqueness(trials: int, new_tokens: int = 32, prompt_len: int = 16, max_batc
             others = torch.randint(0, ToyDecoder.VOC, (b, prompt_len), generator=gt)
             at = int(torch.randint(0, b, (1,), generator=gt))
             others[at] = target
+            ctx_seeds = torch.randint(1, 2 ** 31 - 1, (b,), generator=gt)
+            ctx_seeds[at] = seed  # the fixed prompt always sees the same context
             h = hashlib.sha256()
-            comp = model.generate(impl, others.to(device), new_tokens, watch=at, digest=h)[at].tolist()
+            comp = model.generate(impl, others.to(device), new_tokens, watch=at, digest=h, context=context,
+                                  context_seeds=ctx_seeds)[at].tolist()
             key = tuple(comp)
             seen[key] = seen.get(key, 0) + 1
             bits.add(h.hexdigest())
@@ -792,8 +806,9 @@ def uniqueness(trials: int, new_tokens: int = 32, prompt_len: int = 16, max_batc
 def run_uniqueness(args):
     import torch
     t0 = time.perf_counter()
-    res = uniqueness(args.uniqueness)
+    res = uniqueness(args.uniqueness, context=args.context)
     print(json.dumps({"experiment": "greedy completions of one prompt over random batch compositions",
+                      "context_tokens": args.context,
                       "model": "random-weight 4-layer decoder, hidden 1024, 8 q / 2 kv heads of 128, "
                                "ffn 2816, vocab 32000",
                       "new_tokens": 32, "prompt_len": 16, "batch_sizes": "1..64",
@@ -819,6 +834,8 @@ def main():
     ap.add_argument("--sweep-out", default="", help="write the sweep as JSON to this path")
     ap.add_argument("--uniqueness", type=int, default=0,
                     help="run the batch-composition uniqueness experiment with this many trials")
+    ap.add_argument("--context", type=int, default=4096,
+                    help="cached context positions per sequence in the uniqueness experiment")
     ap.add_argument("--kernel-case", default="", help="launch one kernel on a fixed case: "
                     + ", ".join(sorted(KERNEL_CASES)))
     args = ap.parse_args()

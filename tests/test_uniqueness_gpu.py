@@ -11,7 +11,7 @@ pytestmark = pytest.mark.gpu
 
 
 def test_one_completion_across_batch_compositions():
-    res = bench.uniqueness(trials=24, new_tokens=16, max_batch=48)
+    res = bench.uniqueness(trials=24, new_tokens=16, max_batch=48, context=2048)
     print("unique completions:", res)
     assert res["bi"]["unique"] == 1, res
     assert res["bi"]["unique_logprob_bits"] == 1, res  # every step's log-probs, bit for bit
