@@ -89,7 +89,9 @@ def test_log_softmax_parity_fp32(M, V):
     assert_lsm_close(y, oracle.log_softmax(x.numpy()), f"log_softmax fp32 M={M} V={V}")
 
 
-@pytest.mark.parametrize("V", [151936, 1000, 1001])
+# 1001 takes the scalar path, the others the streamed path (ring of 6 stages: rows of 1, 6, 7,
+# 10 and 19 chunks).
+@pytest.mark.parametrize("V", [151936, 1000, 1001, 110000, 155648, 155656, 4096])
 def test_log_softmax_parity_bf16(V):
     M = 5
     x = inputs.rows_normal(121, 0, M, V, std=1.3)
