@@ -28,7 +28,7 @@ constexpr int kAttnKStride = kAttnD + 8;  // padded K row (bf16): conflict-free 
 struct AttnSmem {
     __nv_bfloat16 k[kAttnSplit][kAttnKStride];
     __nv_bfloat16 v[kAttnSplit][kAttnD];
-    float q[kAttnMaxGroup][kAttnD];
+    __nv_bfloat16 q[kAttnMaxGroup][kAttnD];
     float p[kAttnMaxGroup][kAttnSplit];
     float red[kAttnMaxGroup][4];
     float stat[kAttnMaxGroup][2];
@@ -39,6 +39,7 @@ __host__ __device__ inline int64_t attn_splits(int64_t L) { return (L + kAttnSpl
 // Launch 1: grid (ceil(Lmax / kAttnSplit), Hkv, B), kAttnThreads threads, sizeof(AttnSmem)
 // bytes of dynamic shared memory.  part_ms: [B, Hq, S] float2 (max, sum); part_acc:
 // [B, Hq, S, D] float, S = ceil(Lmax / kAttnSplit).
+template <int G>  // query heads per kv head (1, 2, 4 or 8)
 __global__ void __launch_bounds__(kAttnThreads)
     decode_attention_split_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                                   const __nv_bfloat16 *__restrict__ v, const int32_t *__restrict__ lens,
@@ -49,7 +50,6 @@ __global__ void __launch_bounds__(kAttnThreads)
     AttnSmem &sm = *reinterpret_cast<AttnSmem *>(attn_raw);
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int G = Hq / Hkv;
     const int64_t S = attn_splits(Lmax);
     int64_t L = lens[b];
     if (L < 1 || L > Lmax) {
@@ -60,51 +60,56 @@ __global__ void __launch_bounds__(kAttnThreads)
     if (t0 >= L) return;  // this split is past the sequence's end: it has no partial
     const int n_tok = (int)(L - t0 < kAttnSplit ? L - t0 : kAttnSplit);
 
-    // Stage q (as fp32) for the group's query heads, and the split's K and V rows.
-    for (int i = tid; i < G * kAttnD; i += kAttnThreads) {
-        const int j = i / kAttnD, d = i % kAttnD;
-        sm.q[j][d] = __bfloat162float(q[((int64_t)b * Hq + (int64_t)g * G + j) * kAttnD + d]);
+    // Stage q for the group's query heads and the split's K rows (copy group 1), then the V rows
+    // (copy group 2), all as 16-byte async copies; rows past the sequence are zero-filled.  The
+    // scores only wait for group 1, so V lands while they are computed.
+    for (int c = tid; c < G * (kAttnD / 8); c += kAttnThreads) {
+        const int j = c / (kAttnD / 8), col = (c % (kAttnD / 8)) * 8;
+        cp_async16(&sm.q[j][col], q + ((int64_t)b * Hq + (int64_t)g * G + j) * kAttnD + col, 16u);
     }
-    // All copies are issued before the one wait; rows past the sequence are zero-filled.
     for (int c = tid; c < kAttnSplit * (kAttnD / 8); c += kAttnThreads) {
         const int row = c / (kAttnD / 8), col = (c % (kAttnD / 8)) * 8;
         const bool in = row < n_tok;
         const int64_t off = in ? (((int64_t)b * Lmax + t0 + row) * Hkv + g) * kAttnD + col : 0;
         cp_async16(&sm.k[row][col], k + off, in ? 16u : 0u);
+    }
+    cp_async_commit();
+    for (int c = tid; c < kAttnSplit * (kAttnD / 8); c += kAttnThreads) {
+        const int row = c / (kAttnD / 8), col = (c % (kAttnD / 8)) * 8;
+        const bool in = row < n_tok;
+        const int64_t off = in ? (((int64_t)b * Lmax + t0 + row) * Hkv + g) * kAttnD + col : 0;
         cp_async16(&sm.v[row][col], v + off, in ? 16u : 0u);
     }
-    cp_async_wait_all();
+    cp_async_commit();
+    cp_async_wait_pending<1>();  // q and K have landed (V may still be in flight)
     __syncthreads();
 
     // Scores: thread t takes token t0 + t; s_j = scale * sum_d q_j[d] k_t[d], d ascending.
-    float s[kAttnMaxGroup];
+    float s[G];
 #pragma unroll
-    for (int j = 0; j < kAttnMaxGroup; ++j) s[j] = 0.0f;
+    for (int j = 0; j < G; ++j) s[j] = 0.0f;
 #pragma unroll 2
     for (int d = 0; d < kAttnD; d += 8) {
         const uint4 kw = *reinterpret_cast<const uint4 *>(&sm.k[tid][d]);
         const float kf[8] = {bf16lo(kw.x), bf16hi(kw.x), bf16lo(kw.y), bf16hi(kw.y),
                              bf16lo(kw.z), bf16hi(kw.z), bf16lo(kw.w), bf16hi(kw.w)};
 #pragma unroll
-        for (int j = 0; j < kAttnMaxGroup; ++j) {
-            if (j < G) {
-                // q rows are read as 16-byte broadcasts (every thread the same address)
-                const float4 qa = *reinterpret_cast<const float4 *>(&sm.q[j][d]);
-                const float4 qb = *reinterpret_cast<const float4 *>(&sm.q[j][d + 4]);
-                const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+        for (int j = 0; j < G; ++j) {
+            // q rows are read as 16-byte broadcasts (every thread the same address)
+            const uint4 qw = *reinterpret_cast<const uint4 *>(&sm.q[j][d]);
+            const float qv[8] = {bf16lo(qw.x), bf16hi(qw.x), bf16lo(qw.y), bf16hi(qw.y),
+                                 bf16lo(qw.z), bf16hi(qw.z), bf16lo(qw.w), bf16hi(qw.w)};
 #pragma unroll
-                for (int e = 0; e < 8; ++e) s[j] = fmaf(qv[e], kf[e], s[j]);
-            }
+            for (int e = 0; e < 8; ++e) s[j] = fmaf(qv[e], kf[e], s[j]);
         }
     }
     const bool live = tid < n_tok;
 #pragma unroll
-    for (int j = 0; j < kAttnMaxGroup; ++j) s[j] = live ? s[j] * scale : kNegInf;
+    for (int j = 0; j < G; ++j) s[j] = live ? s[j] * scale : kNegInf;
 
     // Per head: maximum over the split (fixed butterfly, then warp partials in order).
 #pragma unroll
-    for (int j = 0; j < kAttnMaxGroup; ++j) {
-        if (j >= G) break;
+    for (int j = 0; j < G; ++j) {
         float m = s[j];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -119,8 +124,7 @@ __global__ void __launch_bounds__(kAttnThreads)
     __syncthreads();
     // p = exp(s - m); per-head sums by the same fixed tree.
 #pragma unroll
-    for (int j = 0; j < kAttnMaxGroup; ++j) {
-        if (j >= G) break;
+    for (int j = 0; j < G; ++j) {
         const float pj = live ? __expf(s[j] - sm.stat[j][0]) : 0.0f;
         sm.p[j][tid] = pj;
         const float w_sum = warp_sum(pj);
@@ -134,26 +138,28 @@ __global__ void __launch_bounds__(kAttnThreads)
     }
     __syncthreads();
 
+    cp_async_wait_pending<0>();  // V has landed
+    __syncthreads();
+
     // Weighted value sums: thread d accumulates sum_t p_j[t] v_t[d], t ascending.
-    float acc[kAttnMaxGroup];
+    float acc[G];
 #pragma unroll
-    for (int j = 0; j < kAttnMaxGroup; ++j) acc[j] = 0.0f;
+    for (int j = 0; j < G; ++j) acc[j] = 0.0f;
     // Tokens four at a time (p rows read as 16-byte broadcasts); rows past n_tok hold p = 0
     // and zero-filled values, so the padded tail adds exact zeros.
     for (int t = 0; t < n_tok; t += 4) {
         const float v0 = __bfloat162float(sm.v[t][tid]), v1 = __bfloat162float(sm.v[t + 1][tid]),
                     v2 = __bfloat162float(sm.v[t + 2][tid]), v3 = __bfloat162float(sm.v[t + 3][tid]);
 #pragma unroll
-        for (int j = 0; j < kAttnMaxGroup; ++j) {
-            if (j < G) {
-                const float4 pj = *reinterpret_cast<const float4 *>(&sm.p[j][t]);
-                acc[j] = fmaf(pj.x, v0, acc[j]);
-                acc[j] = fmaf(pj.y, v1, acc[j]);
-                acc[j] = fmaf(pj.z, v2, acc[j]);
-                acc[j] = fmaf(pj.w, v3, acc[j]);
-            }
+        for (int j = 0; j < G; ++j) {
+            const float4 pj = *reinterpret_cast<const float4 *>(&sm.p[j][t]);
+            acc[j] = fmaf(pj.x, v0, acc[j]);
+            acc[j] = fmaf(pj.y, v1, acc[j]);
+            acc[j] = fmaf(pj.z, v2, acc[j]);
+            acc[j] = fmaf(pj.w, v3, acc[j]);
         }
     }
+#pragma unroll
     for (int j = 0; j < G; ++j) {
         const int64_t bh = (int64_t)b * Hq + (int64_t)g * G + j;
         part_acc[(bh * S + split) * kAttnD + tid] = acc[j];

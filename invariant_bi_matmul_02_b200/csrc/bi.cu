@@ -75,8 +75,14 @@ bi_status device_state(DeviceState **out)
                 return BI_ERR_CUDA;
             d.gemm_clusters = n;
         }
-        if (cudaFuncSetAttribute(bi::decode_attention_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(bi::AttnSmem)) != cudaSuccess)
+        if (cudaFuncSetAttribute(bi::decode_attention_split_kernel<1>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(bi::AttnSmem)) != cudaSuccess ||
+            cudaFuncSetAttribute(bi::decode_attention_split_kernel<2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(bi::AttnSmem)) != cudaSuccess ||
+            cudaFuncSetAttribute(bi::decode_attention_split_kernel<4>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(bi::AttnSmem)) != cudaSuccess ||
+            cudaFuncSetAttribute(bi::decode_attention_split_kernel<8>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(bi::AttnSmem)) != cudaSuccess)
             return BI_ERR_CUDA;
         if (cudaFuncSetAttribute(bi::log_softmax_stream_kernel<true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kLsmSmem) != cudaSuccess ||
@@ -447,7 +453,8 @@ bi_status bi_decode_attention(const void *q, const void *k_cache, const void *v_
 {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Lmax <= 0) return B == 0 ? BI_OK : BI_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return BI_ERR_INVALID_ARG;
-    if (D != bi::kAttnD || Hq / Hkv > bi::kAttnMaxGroup) return BI_ERR_UNSUPPORTED;
+    const int64_t group = Hq / Hkv;
+    if (D != bi::kAttnD || (group != 1 && group != 2 && group != 4 && group != 8)) return BI_ERR_UNSUPPORTED;
     if (B > 65535 || Hkv > 65535 || Hq > 65535 || bi::attn_splits(Lmax) > kI32Max) return BI_ERR_UNSUPPORTED;
     if (B == 0) return BI_OK;
     if (!q || !k_cache || !v_cache || !seq_lens || !out || !scratch) return BI_ERR_INVALID_ARG;
@@ -465,9 +472,18 @@ bi_status bi_decode_attention(const void *q, const void *k_cache, const void *v_
     const auto *qb = static_cast<const __nv_bfloat16 *>(q);
     const auto *kb = static_cast<const __nv_bfloat16 *>(k_cache);
     const auto *vb = static_cast<const __nv_bfloat16 *>(v_cache);
-    bi::decode_attention_split_kernel<<<dim3((unsigned)S, (unsigned)Hkv, (unsigned)B), bi::kAttnThreads,
-                                        sizeof(bi::AttnSmem), s>>>(qb, kb, vb, seq_lens, part_ms, part_acc,
-                                                                   (int)Hq, (int)Hkv, Lmax, scale, dev->status);
+    const dim3 grid((unsigned)S, (unsigned)Hkv, (unsigned)B);
+    switch (Hq / Hkv) {  // the group size is a property of the model, not of the batch
+    case 1: bi::decode_attention_split_kernel<1><<<grid, bi::kAttnThreads, sizeof(bi::AttnSmem), s>>>(
+                qb, kb, vb, seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
+    case 2: bi::decode_attention_split_kernel<2><<<grid, bi::kAttnThreads, sizeof(bi::AttnSmem), s>>>(
+                qb, kb, vb, seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
+    case 4: bi::decode_attention_split_kernel<4><<<grid, bi::kAttnThreads, sizeof(bi::AttnSmem), s>>>(
+                qb, kb, vb, seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
+    case 8: bi::decode_attention_split_kernel<8><<<grid, bi::kAttnThreads, sizeof(bi::AttnSmem), s>>>(
+                qb, kb, vb, seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
+    default: return BI_ERR_UNSUPPORTED;
+    }
     bi::decode_attention_combine_kernel<<<dim3((unsigned)Hq, (unsigned)B), bi::kAttnD, 0, s>>>(
         part_ms, part_acc, seq_lens, static_cast<__nv_bfloat16 *>(out), (int)Hq, Lmax);
     return launched();

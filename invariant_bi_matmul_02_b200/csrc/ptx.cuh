@@ -399,3 +399,17 @@ __device__ __forceinline__ void cp_async_wait_all()
 }
 
 }  // namespace bi
+
+namespace bi {
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// Wait until at most `n` of this thread's committed copy groups are still pending.
+template <int n>
+__device__ __forceinline__ void cp_async_wait_pending()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(n) : "memory");
+}
+
+}  // namespace bi
+
