@@ -597,6 +597,7 @@ KERNEL_CASES = {
     "mean": "bi_mean M=16384 H=4096 fp32",
     "log_softmax": "bi_log_softmax M=1024 V=151936 bf16 -> fp32",
     "silu_mul": "bi_silu_mul M=1024 F=12288",
+    "decode_attention": "bi_decode_attention B=64 L=4096, 32 q / 8 kv heads of 128",
 }
 
 
@@ -645,6 +646,18 @@ def run_kernel_case(args):
         h = torch.empty(1024, FFN, dtype=torch.bfloat16, device=dev)
         fn = lambda: bi.bi_silu_mul(gu, out=h)
         work, unit = 6 * FFN * 1024, "GB/s"
+    elif name == "decode_attention":
+        B, L, Hq, Hkv, D = 64, 4096, 32, 8, 128
+        g = torch.Generator(device=dev)
+        g.manual_seed(56)
+        q = torch.randn(B, Hq, D, generator=g, device=dev).to(torch.bfloat16)
+        k = torch.randn(B, L, Hkv, D, generator=g, device=dev).to(torch.bfloat16)
+        v = torch.randn(B, L, Hkv, D, generator=g, device=dev).to(torch.bfloat16)
+        sl = torch.full((B,), L, dtype=torch.int32, device=dev)
+        scr = torch.empty(bi.bi_decode_attention_scratch_bytes(B, Hq, D, L), dtype=torch.uint8, device=dev)
+        o = torch.empty_like(q)
+        fn = lambda: bi.bi_decode_attention(q, k, v, sl, scratch=scr, out=o)
+        work, unit = 2 * B * L * Hkv * D * 2, "GB/s"
     else:
         raise SystemExit(f"unknown kernel case {name}; choose from {sorted(KERNEL_CASES)}")
     for _ in range(args.warmup):
