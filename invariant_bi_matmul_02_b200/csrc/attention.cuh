@@ -23,24 +23,41 @@ constexpr int kAttnD = 128;
 constexpr int kAttnSplit = 128;       // tokens per split (one per thread in the score phase)
 constexpr int kAttnThreads = 128;
 constexpr int kAttnMaxGroup = 8;      // query heads per kv head
-constexpr int kAttnKStride = kAttnD + 8;  // padded K row (bf16): conflict-free 16-byte reads
+constexpr int kAttnStride = kAttnD + 8;  // padded row (bf16): conflict-free ldmatrix rows
+constexpr int kAttnWarps = kAttnThreads / 32;
 
 struct AttnSmem {
-    __nv_bfloat16 k[kAttnSplit][kAttnKStride];
-    __nv_bfloat16 v[kAttnSplit][kAttnD];
-    __nv_bfloat16 q[kAttnMaxGroup][kAttnD];
-    float p[kAttnMaxGroup][kAttnSplit];
-    float red[kAttnMaxGroup][4];
-    float stat[kAttnMaxGroup][2];
+    __nv_bfloat16 q[16][kAttnStride];           // the group's query heads, rows >= G zero
+    union {
+        __nv_bfloat16 k[kAttnSplit][kAttnStride];
+        float o[kAttnWarps][kAttnMaxGroup][kAttnD];  // per-warp partial outputs, after the scores
+    } ko;
+    __nv_bfloat16 v[kAttnSplit][kAttnStride];
+    float red[kAttnWarps][16];
+    float stat[16][2];
 };
 
 __host__ __device__ inline int64_t attn_splits(int64_t L) { return (L + kAttnSplit - 1) / kAttnSplit; }
 
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&p);
+}
+
 // Launch 1: grid (ceil(Lmax / kAttnSplit), Hkv, B), kAttnThreads threads, sizeof(AttnSmem)
 // bytes of dynamic shared memory.  part_ms: [B, Hq, S] float2 (max, sum); part_acc:
 // [B, Hq, S, D] float, S = ceil(Lmax / kAttnSplit).
+//
+// Tensor-core form (mma.sync m16n8k16, bf16 in, fp32 accumulate).  Warp w owns tokens
+// 32w .. 32w+31 of the split.  Scores: S = Q . K^T with Q the group's heads padded to 16 rows;
+// every score accumulates its eight 16-wide D steps in ascending order.  Then, per head, the
+// split's maximum and sum of exp(s - max) (fp32) come from fixed trees: a thread's own values
+// in order, the lane quad (xor 1, 2), the warps in order.  Weighted sums: O_w = P_w . V_w with
+// P split into two bf16 terms (about 16 significant bits), two 16-token steps in ascending
+// order; the four warps' O_w are added in warp order.
 template <int G>  // query heads per kv head (1, 2, 4 or 8)
-__global__ void __launch_bounds__(kAttnThreads)
+__global__ void __launch_bounds__(kAttnThreads, 3)
     decode_attention_split_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                                   const __nv_bfloat16 *__restrict__ v, const int32_t *__restrict__ lens,
                                   float2 *__restrict__ part_ms, float *__restrict__ part_acc, int Hq, int Hkv,
@@ -50,6 +67,7 @@ __global__ void __launch_bounds__(kAttnThreads)
     AttnSmem &sm = *reinterpret_cast<AttnSmem *>(attn_raw);
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
     const int64_t S = attn_splits(Lmax);
     int64_t L = lens[b];
     if (L < 1 || L > Lmax) {
@@ -60,18 +78,19 @@ __global__ void __launch_bounds__(kAttnThreads)
     if (t0 >= L) return;  // this split is past the sequence's end: it has no partial
     const int n_tok = (int)(L - t0 < kAttnSplit ? L - t0 : kAttnSplit);
 
-    // Stage q for the group's query heads and the split's K rows (copy group 1), then the V rows
-    // (copy group 2), all as 16-byte async copies; rows past the sequence are zero-filled.  The
-    // scores only wait for group 1, so V lands while they are computed.
-    for (int c = tid; c < G * (kAttnD / 8); c += kAttnThreads) {
+    // Stage Q (rows >= G zero) and K in copy group 1, V in copy group 2 (16-byte async
+    // copies; rows past the sequence zero-filled).  The scores wait for group 1 only.
+    for (int c = tid; c < 16 * (kAttnD / 8); c += kAttnThreads) {
         const int j = c / (kAttnD / 8), col = (c % (kAttnD / 8)) * 8;
-        cp_async16(&sm.q[j][col], q + ((int64_t)b * Hq + (int64_t)g * G + j) * kAttnD + col, 16u);
+        const bool in = j < G;
+        cp_async16(&sm.q[j][col], q + (in ? ((int64_t)b * Hq + (int64_t)g * G + j) * kAttnD + col : 0),
+                   in ? 16u : 0u);
     }
     for (int c = tid; c < kAttnSplit * (kAttnD / 8); c += kAttnThreads) {
         const int row = c / (kAttnD / 8), col = (c % (kAttnD / 8)) * 8;
         const bool in = row < n_tok;
         const int64_t off = in ? (((int64_t)b * Lmax + t0 + row) * Hkv + g) * kAttnD + col : 0;
-        cp_async16(&sm.k[row][col], k + off, in ? 16u : 0u);
+        cp_async16(&sm.ko.k[row][col], k + off, in ? 16u : 0u);
     }
     cp_async_commit();
     for (int c = tid; c < kAttnSplit * (kAttnD / 8); c += kAttnThreads) {
@@ -81,88 +100,139 @@ __global__ void __launch_bounds__(kAttnThreads)
         cp_async16(&sm.v[row][col], v + off, in ? 16u : 0u);
     }
     cp_async_commit();
-    cp_async_wait_pending<1>();  // q and K have landed (V may still be in flight)
+    cp_async_wait_pending<1>();
     __syncthreads();
 
-    // Scores: thread t takes token t0 + t; s_j = scale * sum_d q_j[d] k_t[d], d ascending.
-    float s[G];
+    // ---- scores: acc[nt] is the 16 x 8 tile (heads x tokens 32w + 8nt ..)
+    float acc[4][4];
 #pragma unroll
-    for (int j = 0; j < G; ++j) s[j] = 0.0f;
-#pragma unroll 2
-    for (int d = 0; d < kAttnD; d += 8) {
-        const uint4 kw = *reinterpret_cast<const uint4 *>(&sm.k[tid][d]);
-        const float kf[8] = {bf16lo(kw.x), bf16hi(kw.x), bf16lo(kw.y), bf16hi(kw.y),
-                             bf16lo(kw.z), bf16hi(kw.z), bf16lo(kw.w), bf16hi(kw.w)};
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-            // q rows are read as 16-byte broadcasts (every thread the same address)
-            const uint4 qw = *reinterpret_cast<const uint4 *>(&sm.q[j][d]);
-            const float qv[8] = {bf16lo(qw.x), bf16hi(qw.x), bf16lo(qw.y), bf16hi(qw.y),
-                                 bf16lo(qw.z), bf16hi(qw.z), bf16lo(qw.w), bf16hi(qw.w)};
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) s[j] = fmaf(qv[e], kf[e], s[j]);
+    for (int kk = 0; kk < kAttnD / 16; ++kk) {
+        uint32_t af[4];
+        ldsm_x4(af, &sm.q[(lane & 7) + 8 * ((lane >> 3) & 1)][16 * kk + 8 * (lane >> 4)]);
+#pragma unroll
+        for (int nt = 0; nt < 4; nt += 2) {
+            // matrices: (tile nt, d 0-7), (nt, d 8-15), (nt+1, d 0-7), (nt+1, d 8-15) of this step
+            uint32_t bf[4];
+            ldsm_x4(bf, &sm.ko.k[32 * warp + 8 * (nt + (lane >> 4)) + (lane & 7)][16 * kk + 8 * ((lane >> 3) & 1)]);
+            mma_16816_bf16(acc[nt], af, bf[0], bf[1]);
+            mma_16816_bf16(acc[nt + 1], af, bf[2], bf[3]);
         }
     }
-    const bool live = tid < n_tok;
+    // scale and mask: element (row gid / gid+8, token 32w + 8nt + 2tig + {0,1})
 #pragma unroll
-    for (int j = 0; j < G; ++j) s[j] = live ? s[j] * scale : kNegInf;
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int tok = 32 * warp + 8 * nt + 2 * tig + (e & 1);
+            acc[nt][e] = tok < n_tok ? acc[nt][e] * scale : kNegInf;
+        }
 
-    // Per head: maximum over the split (fixed butterfly, then warp partials in order).
+    // ---- per-head max: own values in order, quad butterfly, warps in order
+    float mx[2];
 #pragma unroll
-    for (int j = 0; j < G; ++j) {
-        float m = s[j];
+    for (int h = 0; h < 2; ++h) {
+        float m = acc[0][2 * h];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) sm.red[j][warp] = m;
+        for (int nt = 0; nt < 4; ++nt) m = fmaxf(fmaxf(m, acc[nt][2 * h]), acc[nt][2 * h + 1]);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        mx[h] = m;
+    }
+    if (tig == 0) {
+        sm.red[warp][gid] = mx[0];
+        sm.red[warp][gid + 8] = mx[1];
     }
     __syncthreads();
-    if (tid < G) {
-        float m = sm.red[tid][0];
-        for (int w = 1; w < kAttnThreads / 32; ++w) m = fmaxf(m, sm.red[tid][w]);
+    if (tid < 16) {
+        float m = sm.red[0][tid];
+        for (int w = 1; w < kAttnWarps; ++w) m = fmaxf(m, sm.red[w][tid]);
         sm.stat[tid][0] = m;
     }
     __syncthreads();
-    // p = exp(s - m); per-head sums by the same fixed tree.
+    // ---- p = exp(s - max); per-head sums by the same trees
+    float sum[2];
 #pragma unroll
-    for (int j = 0; j < G; ++j) {
-        const float pj = live ? __expf(s[j] - sm.stat[j][0]) : 0.0f;
-        sm.p[j][tid] = pj;
-        const float w_sum = warp_sum(pj);
-        if (lane == 0) sm.red[j][warp] = w_sum;
+    for (int h = 0; h < 2; ++h) {
+        const float m = sm.stat[gid + 8 * h][0];
+        float l = 0.0f;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float &x = acc[nt][2 * h + e];
+                x = x == kNegInf ? 0.0f : __expf(x - m);
+                l = __fadd_rn(l, x);
+            }
+        l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 1));
+        l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 2));
+        sum[h] = l;
     }
-    __syncthreads();
-    if (tid < G) {
-        float l = sm.red[tid][0];
-        for (int w = 1; w < kAttnThreads / 32; ++w) l = __fadd_rn(l, sm.red[tid][w]);
-        sm.stat[tid][1] = l;
+    __syncthreads();  // every warp has read sm.stat / sm.red
+    if (tig == 0) {
+        sm.red[warp][gid] = sum[0];
+        sm.red[warp][gid + 8] = sum[1];
     }
-    __syncthreads();
-
     cp_async_wait_pending<0>();  // V has landed
     __syncthreads();
+    if (tid < 16) {
+        float l = sm.red[0][tid];
+        for (int w = 1; w < kAttnWarps; ++w) l = __fadd_rn(l, sm.red[w][tid]);
+        sm.stat[tid][1] = l;
+    }
 
-    // Weighted value sums: thread d accumulates sum_t p_j[t] v_t[d], t ascending.
-    float acc[G];
+    // ---- O_w = P_w . V_w: A from the score tiles (two 8-token tiles per 16-token step)
+    float o[kAttnD / 8][4];
 #pragma unroll
-    for (int j = 0; j < G; ++j) acc[j] = 0.0f;
-    // Tokens four at a time (p rows read as 16-byte broadcasts); rows past n_tok hold p = 0
-    // and zero-filled values, so the padded tail adds exact zeros.
-    for (int t = 0; t < n_tok; t += 4) {
-        const float v0 = __bfloat162float(sm.v[t][tid]), v1 = __bfloat162float(sm.v[t + 1][tid]),
-                    v2 = __bfloat162float(sm.v[t + 2][tid]), v3 = __bfloat162float(sm.v[t + 3][tid]);
+    for (int dt = 0; dt < kAttnD / 8; ++dt)
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-            const float4 pj = *reinterpret_cast<const float4 *>(&sm.p[j][t]);
-            acc[j] = fmaf(pj.x, v0, acc[j]);
-            acc[j] = fmaf(pj.y, v1, acc[j]);
-            acc[j] = fmaf(pj.z, v2, acc[j]);
-            acc[j] = fmaf(pj.w, v3, acc[j]);
+        for (int e = 0; e < 4; ++e) o[dt][e] = 0.0f;
+    // P enters the tensor cores as two bf16 terms, hi = bf16(p) and lo = bf16(p - hi), so the
+    // weights keep about 16 significant bits; per 16-token step the hi product is added first.
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const float *p0 = acc[2 * j], *p1 = acc[2 * j + 1];
+        const float pv[8] = {p0[0], p0[1], p0[2], p0[3], p1[0], p1[1], p1[2], p1[3]};
+        float hi[8], lo[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            hi[e] = __bfloat162float(__float2bfloat16_rn(pv[e]));
+            lo[e] = pv[e] - hi[e];
+        }
+        const uint32_t pa_hi[4] = {pack_bf16(hi[0], hi[1]), pack_bf16(hi[2], hi[3]), pack_bf16(hi[4], hi[5]),
+                                   pack_bf16(hi[6], hi[7])};
+        const uint32_t pa_lo[4] = {pack_bf16(lo[0], lo[1]), pack_bf16(lo[2], lo[3]), pack_bf16(lo[4], lo[5]),
+                                   pack_bf16(lo[6], lo[7])};
+        const int tok0 = 32 * warp + 16 * j;
+#pragma unroll
+        for (int dt = 0; dt < kAttnD / 8; dt += 2) {
+            // matrices (transposed): (tokens 0-7, d tile dt), (tokens 8-15, dt), (0-7, dt+1), (8-15, dt+1)
+            uint32_t vf[4];
+            ldsm_x4_trans(vf, &sm.v[tok0 + (lane & 7) + 8 * ((lane >> 3) & 1)][8 * (dt + (lane >> 4))]);
+            mma_16816_bf16(o[dt], pa_hi, vf[0], vf[1]);
+            mma_16816_bf16(o[dt], pa_lo, vf[0], vf[1]);
+            mma_16816_bf16(o[dt + 1], pa_hi, vf[2], vf[3]);
+            mma_16816_bf16(o[dt + 1], pa_lo, vf[2], vf[3]);
         }
     }
+    __syncthreads();  // K is no longer read: its space holds the per-warp outputs
+#pragma unroll
+    for (int dt = 0; dt < kAttnD / 8; ++dt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int row = gid + 8 * (e >> 1), col = 8 * dt + 2 * tig + (e & 1);
+            if (row < G) sm.ko.o[warp][row][col] = o[dt][e];
+        }
+    __syncthreads();
 #pragma unroll
     for (int j = 0; j < G; ++j) {
+        float r = sm.ko.o[0][j][tid];
+        for (int w = 1; w < kAttnWarps; ++w) r = __fadd_rn(r, sm.ko.o[w][j][tid]);
         const int64_t bh = (int64_t)b * Hq + (int64_t)g * G + j;
-        part_acc[(bh * S + split) * kAttnD + tid] = acc[j];
+        part_acc[(bh * S + split) * kAttnD + tid] = r;
         if (tid == 0) part_ms[bh * S + split] = make_float2(sm.stat[j][0], sm.stat[j][1]);
     }
 }

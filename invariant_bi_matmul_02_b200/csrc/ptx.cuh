@@ -413,3 +413,36 @@ __device__ __forceinline__ void cp_async_wait_pending()
 
 }  // namespace bi
 
+
+namespace bi {
+
+// ---------------------------------------------------------------- warp-level MMA (decode attention)
+
+// Four 8x8 b16 matrices from shared memory; lane i supplies the address of row i % 8 of
+// matrix i / 8.  Register j receives row lane / 4, elements 2 (lane % 4) and +1 of matrix j.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *row_addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_addr(row_addr)));
+}
+
+// As ldsm_x4 with each 8x8 matrix transposed on the way.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void *row_addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_addr(row_addr)));
+}
+
+// D = A (16x16 bf16, row) . B (16x8 bf16, col) + C, fp32 accumulate.
+__device__ __forceinline__ void mma_16816_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+}  // namespace bi
