@@ -3,9 +3,12 @@
 Tolerances (written here once, used by every parity test):
 * bf16 outputs:        |gpu - ref| <= 2^-7 |ref| + 1e-3
 * fp32 log_softmax:    |gpu - ref| <= 1e-4
-* fp32 mean:           |gpu - ref| <= (ceil(log2 H) + 2) 2^-24 sum|x| / H + 2^-24 |ref|
-  (the error bound of a tree-shaped fp32 sum of depth ceil(log2 H) + 2, then one
-  correctly rounded division)
+* fp32 mean:           |gpu - ref| <= 1.01 d 2^-24 sum|x| / H + 2^-24 |ref|
+  where d = mean_chain_depth(H) is the longest chain of fp32 additions an element passes
+  through in bi_mean's fixed order (per-thread running sums, then the block tree): the
+  first-order error bound of
+  recursive summation in a fixed order (Higham, Accuracy and Stability of Numerical
+  Algorithms, section 4.2), then one correctly rounded division
 """
 import math
 
@@ -43,10 +46,24 @@ def assert_lsm_close(gpu: torch.Tensor, ref: np.ndarray, what: str = ""):
     assert worst <= LSM_ABS, f"{what}: max |err| {worst} > {LSM_ABS}"
 
 
+def mean_chain_depth(H: int) -> int:
+    """Longest chain of fp32 additions in bi_mean's order for rows of H elements: one block of
+    T threads per row (T = 32 ceil(((H / 4 + 3) / 4) / 32), clamped to [32, 1024]).
+    H % 4 == 0: thread t keeps four running sums, one per lane of its float4 groups t, t + T,
+    ...; each adds g = ceil(H / 4 / T) values, then the four meet in a 2-level tree.  Otherwise
+    thread t adds its ceil(H / T) elements into one sum.  The block tree then adds 10 levels
+    (warp butterfly, then a butterfly over the warp sums)."""
+    v = (H // 4 + 3) // 4
+    T = min(1024, max(32, -(-v // 32) * 32))
+    if H % 4 == 0:
+        return -(-(H // 4) // T) + 2 + 10
+    return -(-H // T) + 10
+
+
 def assert_mean_close(gpu: torch.Tensor, ref: np.ndarray, x: np.ndarray, what: str = ""):
     H = x.shape[1]
     g = to_np64(gpu)
-    depth = math.ceil(math.log2(max(H, 2))) + 2
+    depth = 1.01 * mean_chain_depth(H)
     bound = depth * U32 * np.abs(x.astype(np.float64)).sum(axis=1) / H + U32 * np.abs(ref)
     err = np.abs(g - ref)
     assert np.all(err <= bound), f"{what}: worst excess {float((err - bound).max())}"
