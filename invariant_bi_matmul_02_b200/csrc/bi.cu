@@ -87,7 +87,17 @@ bi_status device_state(DeviceState **out)
         if (cudaFuncSetAttribute(bi::log_softmax_stream_kernel<true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kLsmSmem) != cudaSuccess ||
             cudaFuncSetAttribute(bi::log_softmax_stream_kernel<false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kLsmSmem) != cudaSuccess)
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kLsmSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(bi::log_softmax_cluster_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kClSliceBytesMax) != cudaSuccess ||
+            cudaFuncSetAttribute(bi::log_softmax_cluster_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kClSliceBytesMax) != cudaSuccess)
+            return BI_ERR_CUDA;
+        if (bi::kRowCluster > 8 &&  // clusters above the portable size must be allowed per kernel
+            (cudaFuncSetAttribute(bi::log_softmax_cluster_kernel<true>,
+                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
+             cudaFuncSetAttribute(bi::log_softmax_cluster_kernel<false>,
+                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess))
             return BI_ERR_CUDA;
         d.ready = true;
     }
@@ -129,17 +139,42 @@ bi_status encode_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_
 
 bi_status launched() { return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA; }
 
+// Launch `kernel` with one cluster of bi::kRowCluster CTAs per row, rows on grid.y in slices of
+// at most 65535; the kernel takes the slice's first row as its `row0` argument.
+template <typename... KArgs, typename... Args>
+bi_status launch_row_clusters(void (*kernel)(KArgs...), int64_t M, size_t smem, cudaStream_t s, Args... args)
+{
+    for (int64_t row0 = 0; row0 < M; row0 += 65535) {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(bi::kRowCluster, (unsigned)(M - row0 < 65535 ? M - row0 : 65535), 1);
+        cfg.blockDim = dim3(bi::kClThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr{};
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = bi::kRowCluster;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kernel, args..., row0) != cudaSuccess) return BI_ERR_CUDA;
+    }
+    return BI_OK;
+}
+
 // N is the number of output columns.  With fuse_silu, B holds 2N rows ([gate; up]) and
 // the output is silu(A . gate^T) * (A . up^T).
 bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, const void *A, int64_t lda,
                       const void *B, int64_t ldb, int b_layout, void *C, int64_t ldc, int c_dtype,
-                      int64_t M, int64_t N, int64_t K, void *stream, int fuse_silu = 0)
+                      int64_t M, int64_t N, int64_t K, void *stream, int fuse_silu = 0,
+                      float *lse_partial = nullptr)
 {
     if (M < 0 || N < 0 || K < 0) return BI_ERR_INVALID_ARG;
     if (b_layout != BI_B_KN && b_layout != BI_B_NK) return BI_ERR_INVALID_ARG;
     if (c_dtype != BI_BF16 && c_dtype != BI_F32) return BI_ERR_INVALID_ARG;
     if (M > kI32Max || (fuse_silu ? 2 * N : N) > kI32Max || K > kI32Max) return BI_ERR_UNSUPPORTED;
     if (M == 0 || N == 0) return BI_OK;
+    if (lse_partial && (fuse_silu || reinterpret_cast<uintptr_t>(lse_partial) % 8 != 0)) return BI_ERR_ALIGNMENT;
     const int64_t b_rows = fuse_silu ? 2 * N : N;  // extent of B along the output dimension
     if (!C || ldc < N) return BI_ERR_INVALID_ARG;
     if (addend_mode != bi::kAddNone) {
@@ -175,6 +210,8 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
     p.addend = static_cast<const __nv_bfloat16 *>(input);
     p.status = dev->status;
     p.wait_limit_ns = kWaitLimitNs;
+    p.lse_partial = reinterpret_cast<float2 *>(lse_partial);
+    p.lse_per_row = p.n_blocks;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
     if (K == 0 && !fuse_silu) {
@@ -182,6 +219,11 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
         int64_t blocks = (total + 255) / 256;
         if (blocks > (int64_t)dev->sms * 16) blocks = (int64_t)dev->sms * 16;
         bi::gemm_k0_fill_kernel<<<(unsigned)blocks, 256, 0, s>>>(p);
+        if (lse_partial) {
+            int64_t pb = (M * p.lse_per_row + 127) / 128;
+            if (pb > (int64_t)dev->sms * 16) pb = (int64_t)dev->sms * 16;
+            bi::gemm_k0_partials_kernel<<<(unsigned)pb, 128, 0, s>>>(p);
+        }
         return launched();
     }
 
@@ -257,6 +299,55 @@ bi_status bi_matmul_silu_mul(const void *A, int64_t lda, const void *B, int64_t 
                        1);
 }
 
+int64_t bi_lse_partials_per_row(int64_t N)
+{
+    return N <= 0 ? 0 : (N + bi::kPairBN - 1) / bi::kPairBN;
+}
+
+bi_status bi_matmul_lse(const void *A, int64_t lda, const void *B, int64_t ldb, bi_b_layout b_layout, void *C,
+                        int64_t ldc, bi_dtype c_dtype, float *partials, int64_t M, int64_t N, int64_t K,
+                        void *stream)
+{
+    if (M > 0 && N > 0 && !partials) return BI_ERR_INVALID_ARG;
+    return gemm_common(nullptr, 0, bi::kAddNone, A, lda, B, ldb, b_layout, C, ldc, c_dtype, M, N, K, stream, 0,
+                       partials);
+}
+
+bi_status bi_log_softmax_partials(const void *x, int64_t ldx, bi_dtype x_dtype, const float *partials,
+                                  float *row_stats, float *y, int64_t M, int64_t V, void *stream)
+{
+    if (M < 0 || V < 0) return BI_ERR_INVALID_ARG;
+    if (x_dtype != BI_BF16 && x_dtype != BI_F32) return BI_ERR_INVALID_ARG;
+    if (M > kI32Max || V > kI32Max) return BI_ERR_UNSUPPORTED;
+    if (M == 0) return BI_OK;
+    if (V == 0 || !x || !y || !partials || !row_stats || ldx < V) return BI_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(partials) % 8 != 0 || reinterpret_cast<uintptr_t>(row_stats) % 8 != 0)
+        return BI_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool bf16 = x_dtype == BI_BF16;
+    const int64_t P = bi_lse_partials_per_row(V);
+    const float2 *part = reinterpret_cast<const float2 *>(partials);
+    float2 *rs = reinterpret_cast<float2 *>(row_stats);
+    bi::lse_row_stats_kernel<<<(unsigned)((M + bi::kRowStatWarps - 1) / bi::kRowStatWarps),
+                               bi::kRowStatWarps * 32, 0, s>>>(part, P, rs, M);
+    const bool vec = V % 8 == 0 && ldx % (bf16 ? 8 : 4) == 0 && aligned16(x) && aligned16(y);
+    const unsigned chunks = (unsigned)bi::apply_chunks(V);
+    for (int64_t row0 = 0; row0 < M; row0 += 65535) {  // rows on grid.y
+        const dim3 grid(chunks, (unsigned)(M - row0 < 65535 ? M - row0 : 65535));
+        if (vec && bf16)
+            bi::log_softmax_apply_vec_kernel<true><<<grid, bi::kApplyThreads, 0, s>>>(
+                static_cast<const uint8_t *>(x), ldx, rs, y, V, row0);
+        else if (vec)
+            bi::log_softmax_apply_vec_kernel<false><<<grid, bi::kApplyThreads, 0, s>>>(
+                static_cast<const uint8_t *>(x), ldx, rs, y, V, row0);
+        else if (bf16)
+            bi::log_softmax_apply_scalar_kernel<true><<<grid, bi::kApplyThreads, 0, s>>>(x, ldx, rs, y, V, row0);
+        else
+            bi::log_softmax_apply_scalar_kernel<false><<<grid, bi::kApplyThreads, 0, s>>>(x, ldx, rs, y, V, row0);
+    }
+    return launched();
+}
+
 bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H, float eps,
                      void *stream)
 {
@@ -324,6 +415,15 @@ bi_status bi_log_softmax(const void *x, bi_dtype x_dtype, float *y, int64_t M, i
         bi_status st = device_state(&dev);
         if (st != BI_OK) return st;
         const uint8_t *xb = static_cast<const uint8_t *>(x);
+        const int elem = bf16 ? 2 : 4;
+        const int64_t slice_bytes = bi::cluster_slice(V) * elem;
+        if (V * elem >= bi::kClusterRowBytes && slice_bytes <= bi::kClSliceBytesMax) {  // a cluster per row
+            st = bf16 ? launch_row_clusters(bi::log_softmax_cluster_kernel<true>, M, (size_t)slice_bytes, s, xb, y, V,
+                                            dev->status, kWaitLimitNs)
+                      : launch_row_clusters(bi::log_softmax_cluster_kernel<false>, M, (size_t)slice_bytes, s, xb, y,
+                                            V, dev->status, kWaitLimitNs);
+            return st != BI_OK ? st : launched();
+        }
         if (bf16)
             bi::log_softmax_stream_kernel<true><<<(unsigned)M, bi::kLsmThreads, bi::kLsmSmem, s>>>(
                 xb, y, V, dev->status, kWaitLimitNs);

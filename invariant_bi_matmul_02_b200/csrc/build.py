@@ -12,7 +12,7 @@ PKG = os.path.dirname(CSRC)
 ROOT = os.path.dirname(PKG)
 INCLUDE = os.path.join(ROOT, "include")
 SOURCES = [os.path.join(CSRC, "bi.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, n) for n in ("gemm.cuh", "gemm_pair.cuh", "rowops.cuh", "ptx.cuh", "attention.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, n) for n in ("gemm.cuh", "gemm_pair.cuh", "rowops.cuh", "maxsum.cuh", "ptx.cuh", "attention.cuh")] + [
     os.path.join(INCLUDE, "bi.h")]
 LIB = os.path.join(PKG, "libbi.so")
 

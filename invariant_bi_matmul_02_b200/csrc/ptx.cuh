@@ -231,6 +231,14 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t local, uint32_t rank)
     return r;
 }
 
+// Load from a shared::cluster address (this CTA's or a peer's shared memory).
+__device__ __forceinline__ float2 ld_dsmem_f32x2(uint32_t cluster_addr)
+{
+    float2 v;
+    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(cluster_addr) : "memory");
+    return v;
+}
+
 // All threads of every CTA of the cluster.
 __device__ __forceinline__ void cluster_sync_all()
 {

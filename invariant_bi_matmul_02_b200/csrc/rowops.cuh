@@ -12,11 +12,10 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include "maxsum.cuh"
 #include "ptx.cuh"
 
 namespace bi {
-
-#define kNegInf (-__builtin_huge_valf())
 
 // --------------------------------------------------------------- fixed-order trees
 
@@ -41,30 +40,6 @@ __device__ __forceinline__ float block_sum(float v, float *red)
     return t;
 }
 
-// (max, sum of exp(x - max)) pairs.  The merge is symmetric in its two arguments
-// (no contracted multiply-adds), so both lanes of a butterfly pair hold equal bits.
-struct MaxSum {
-    float m, s;
-};
-
-__device__ __forceinline__ MaxSum merge(MaxSum a, MaxSum b)
-{
-    const float m = fmaxf(a.m, b.m);
-    if (m == kNegInf) return {m, 0.0f};
-    const float s = __fadd_rn(__fmul_rn(a.s, __expf(a.m - m)), __fmul_rn(b.s, __expf(b.m - m)));
-    return {m, s};
-}
-
-__device__ __forceinline__ MaxSum warp_merge(MaxSum v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        MaxSum w{__shfl_xor_sync(0xffffffffu, v.m, o), __shfl_xor_sync(0xffffffffu, v.s, o)};
-        v = merge(v, w);
-    }
-    return v;
-}
-
 __device__ __forceinline__ MaxSum block_merge(MaxSum v, float *red_m, float *red_s)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -79,15 +54,6 @@ __device__ __forceinline__ MaxSum block_merge(MaxSum v, float *red_m, float *red
     t = warp_merge(t);
     __syncthreads();
     return t;
-}
-
-// Running (max, sum) update with a group of values already reduced to their max `gm`.
-__device__ __forceinline__ void rescale_to(MaxSum &acc, float gm)
-{
-    if (gm > acc.m) {
-        acc.s = acc.m == kNegInf ? 0.0f : acc.s * __expf(acc.m - gm);
-        acc.m = gm;
-    }
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -232,19 +198,6 @@ __global__ void __launch_bounds__(1024) mean_scalar_kernel(const float *__restri
 }
 
 // --------------------------------------------------------------- log_softmax
-
-template <int P>
-__device__ __forceinline__ void lsm_accumulate(MaxSum &acc, const float (&v)[P])
-{
-    float gm = v[0];
-#pragma unroll
-    for (int k = 1; k < P; ++k) gm = fmaxf(gm, v[k]);
-    rescale_to(acc, gm);
-    if (acc.m != kNegInf) {
-#pragma unroll
-        for (int k = 0; k < P; ++k) acc.s += __expf(v[k] - acc.m);
-    }
-}
 
 // Scalar path for any V: element j belongs to thread j % T.
 template <bool BF16>
@@ -414,6 +367,136 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
 
 constexpr int kLsmSmem = kLsmStages * kLsmChunk;
 
+// --------------------------------------------------------------- long rows: one cluster per row
+
+// log_softmax rows of at least kClusterRowBytes bytes (vector path) whose slices fit in shared
+// memory are reduced by a cluster of kRowCluster CTAs.  CTA r owns the slice [r S, min(V, (r + 1) S)) of the row, with
+// S = cluster_slice(V) a multiple of 8 elements fixed by V alone.  Each CTA reduces its slice
+// in a fixed order; the CTAs' results meet through distributed shared memory and are folded in
+// rank order 0, 1, ..., kRowCluster - 1.  A short batch spreads over kRowCluster times as many
+// SMs as with one block per row, and each CTA keeps its slice in shared memory between the two
+// passes: the row is read from global memory once.
+#ifndef BI_ROW_CLUSTER
+#define BI_ROW_CLUSTER 4           // the one cluster shape every call uses; other values exist for experiments only
+#endif
+#ifndef BI_ROW_CLUSTER_THREADS
+#define BI_ROW_CLUSTER_THREADS 512
+#endif
+#ifndef BI_CLUSTER_ROW_BYTES
+#define BI_CLUSTER_ROW_BYTES (64 * 1024)
+#endif
+constexpr int kRowCluster = BI_ROW_CLUSTER;
+constexpr int kClThreads = BI_ROW_CLUSTER_THREADS;
+constexpr int64_t kClusterRowBytes = BI_CLUSTER_ROW_BYTES;
+constexpr int kClSliceBytesMax = 96 * 1024;  // log_softmax: largest slice held in shared memory
+constexpr int kClPieces = 4;                 // bulk copies per slice, each on its own barrier
+
+__host__ __device__ inline int64_t cluster_slice(int64_t V)
+{
+    return (V + 8 * kRowCluster - 1) / (8 * kRowCluster) * 8;
+}
+
+// log_softmax of one row per cluster; V % 8 == 0 (bf16) or V % 4 == 0 (fp32), x and y 16-byte
+// aligned, cluster_slice(V) * element size <= kClSliceBytesMax.  Grid (kRowCluster, rows).
+// Inside a slice, thread t folds the 4-element groups t, t + T, ... of each bulk piece in turn.
+template <bool BF16>
+__global__ void __launch_bounds__(kClThreads) log_softmax_cluster_kernel(
+    const uint8_t *__restrict__ x, float *__restrict__ y, int64_t V, int32_t *status, uint64_t wait_limit_ns,
+    int64_t row0)
+{
+    constexpr int kElem = BF16 ? 2 : 4;
+    extern __shared__ __align__(128) uint8_t cl_smem[];
+    __shared__ uint64_t full[kClPieces];
+    __shared__ float red_m[32], red_s[32];
+    __shared__ float2 cta_part;
+    __shared__ int abort_flag_s;
+    volatile int *abort_flag = &abort_flag_s;
+
+    const int tid = threadIdx.x;
+    const uint32_t rank = cluster_ctarank();
+    const int64_t row = row0 + blockIdx.y;
+    const int64_t S = cluster_slice(V);
+    const int64_t e_begin = (int64_t)rank * S;
+    const int64_t e_end = e_begin + S < V ? e_begin + S : V;
+    const int64_t n = e_end > e_begin ? e_end - e_begin : 0;  // elements of this CTA's slice
+    const uint32_t bytes = (uint32_t)(n * kElem);             // a multiple of 16
+    const uint32_t piece = ((bytes + kClPieces - 1) / kClPieces + 15u) / 16u * 16u;
+    const uint8_t *src = x + (row * V + e_begin) * kElem;
+
+    if (tid == 0) {
+        for (int p = 0; p < kClPieces; ++p) mbar_init(&full[p], 1);
+        abort_flag_s = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const uint64_t pol = l2_policy_evict_first();  // each byte of x is read once
+        for (int p = 0; p < kClPieces; ++p) {
+            const uint32_t off = (uint32_t)p * piece;
+            const uint32_t b = off < bytes ? (bytes - off < piece ? bytes - off : piece) : 0u;
+            if (b) {
+                mbar_arrive_expect_tx(&full[p], b);
+                bulk_load_hint(cl_smem + off, src + off, b, &full[p], pol);
+            } else {
+                mbar_arrive(&full[p]);  // an empty piece completes at once
+            }
+        }
+    }
+
+    auto load4 = [&](int64_t g, float (&v)[4]) {
+        if (BF16) {
+            const uint2 u = *reinterpret_cast<const uint2 *>(cl_smem + 8 * g);
+            v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+        } else {
+            const float4 f = *reinterpret_cast<const float4 *>(cl_smem + 16 * g);
+            v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+        }
+    };
+
+    MaxSum acc{kNegInf, 0.0f};
+    bool ok = true;
+    for (int p = 0; p < kClPieces; ++p) {
+        const bool got = wait_bounded(&full[p], 0, abort_flag, status, wait_limit_ns);
+        ok = __syncthreads_and(got ? 1 : 0) != 0;
+        if (!ok) break;
+        const uint32_t off = (uint32_t)p * piece;
+        const int64_t g0 = off / (4 * kElem);                                   // first group
+        const int64_t g1 = (off + piece < bytes ? off + piece : bytes) / (4 * kElem);
+        for (int64_t g = g0 + tid; g < g1; g += kClThreads) {
+            float v[4];
+            load4(g, v);
+            lsm_accumulate(acc, v);
+        }
+    }
+    const MaxSum cta = ok ? block_merge(acc, red_m, red_s) : MaxSum{kNegInf, 0.0f};
+    if (tid == 0) cta_part = make_float2(cta.m, cta.s);
+    cluster_sync_all();  // every CTA's (max, sum) is visible to the cluster
+    MaxSum row_ms{kNegInf, 0.0f};
+    for (uint32_t r = 0; r < (uint32_t)kRowCluster; ++r) {
+        const float2 pr = ld_dsmem_f32x2(map_to_rank(smem_addr(&cta_part), r));
+        row_ms = merge(row_ms, MaxSum{pr.x, pr.y});
+    }
+    if (ok) {
+        const float m = row_ms.m, ls = __logf(row_ms.s);
+        float *yr = y + row * V + e_begin;
+        for (int64_t g = tid; 4 * g < n; g += kClThreads) {
+            float v[4];
+            load4(g, v);
+            __stcs(reinterpret_cast<float4 *>(yr + 4 * g),
+                   make_float4((v[0] - m) - ls, (v[1] - m) - ls, (v[2] - m) - ls, (v[3] - m) - ls));
+        }
+    } else if (tid == 0) {
+        // A wait ran out: let the copies already issued land before shared memory goes away.
+        for (int p = 0; p < kClPieces; ++p) {
+            const uint32_t a = smem_addr(&full[p]);
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(a, 0) && global_timer_ns() - t0 < wait_limit_ns) {
+            }
+        }
+    }
+    cluster_sync_all();  // no CTA leaves while a peer may still read its cta_part
+}
+
 // --------------------------------------------------------------- log_softmax, split rows
 
 // Fixed-chunk multi-block variant for short batches.  The row is cut into chunks of
@@ -499,6 +582,92 @@ __global__ void __launch_bounds__(kSplitThreads) log_softmax_split_write_kernel(
         float4 *dst = reinterpret_cast<float4 *>(yr + e);
         __stcs(dst, make_float4((v[0] - m) - ls, (v[1] - m) - ls, (v[2] - m) - ls, (v[3] - m) - ls));
         __stcs(dst + 1, make_float4((v[4] - m) - ls, (v[5] - m) - ls, (v[6] - m) - ls, (v[7] - m) - ls));
+    }
+}
+
+// --------------------------------------------------------------- log_softmax from tile partials
+
+// Second half of the LM-head log_softmax whose first half runs in the GEMM epilogue: the GEMM
+// leaves, per row, one (max, sum of exp) pair for each of its P output tiles.
+//   Launch 1 (one warp per row): lane l folds pairs l, l+32, ... in ascending order, then a
+//            fixed xor butterfly gives the row's (m, log s).
+//   Launch 2 (block (c, i)): y = (x - m) - log(s) for chunk c of row i, kApplyChunk elements;
+//            every load of the chunk is issued before the row's (m, log s) is read.
+// x rows are ldx elements apart; y is [M, V] contiguous.
+constexpr int kRowStatWarps = 8;
+constexpr int kApplyThreads = 256;
+constexpr int kApplyGroups = 4;                                   // 8-element groups per thread
+constexpr int kApplyChunk = kApplyThreads * kApplyGroups * 8;    // 8192 elements per block
+
+__host__ __device__ inline int64_t apply_chunks(int64_t V) { return (V + kApplyChunk - 1) / kApplyChunk; }
+
+__global__ void __launch_bounds__(kRowStatWarps * 32) lse_row_stats_kernel(
+    const float2 *__restrict__ partial, int64_t P, float2 *__restrict__ row_stats, int64_t M)
+{
+    const int64_t row = (int64_t)blockIdx.x * kRowStatWarps + (threadIdx.x >> 5);
+    if (row >= M) return;
+    const int lane = threadIdx.x & 31;
+    const float2 *pr = partial + row * P;
+    MaxSum acc{kNegInf, 0.0f};
+    int64_t k = lane;
+    for (; k + 96 < P; k += 128) {  // four pairs in flight per lane, folded in ascending order
+        const float2 p0 = __ldg(pr + k), p1 = __ldg(pr + k + 32), p2 = __ldg(pr + k + 64), p3 = __ldg(pr + k + 96);
+        acc = merge(acc, MaxSum{p0.x, p0.y});
+        acc = merge(acc, MaxSum{p1.x, p1.y});
+        acc = merge(acc, MaxSum{p2.x, p2.y});
+        acc = merge(acc, MaxSum{p3.x, p3.y});
+    }
+    for (; k < P; k += 32) {
+        const float2 pk = __ldg(pr + k);
+        acc = merge(acc, MaxSum{pk.x, pk.y});
+    }
+    acc = warp_merge(acc);
+    if (lane == 0) row_stats[row] = make_float2(acc.m, __logf(acc.s));
+}
+
+// V % 8 == 0, x 16-byte aligned with ldx % 8 == 0 (bf16) or ldx % 4 == 0 (fp32).
+template <bool BF16>
+__global__ void __launch_bounds__(kApplyThreads) log_softmax_apply_vec_kernel(
+    const uint8_t *__restrict__ x, int64_t ldx, const float2 *__restrict__ row_stats,
+    float *__restrict__ y, int64_t V, int64_t row0)
+{
+    constexpr int kElem = BF16 ? 2 : 4;
+    const int64_t row = row0 + blockIdx.y;
+    const int64_t e0 = blockIdx.x * (int64_t)kApplyChunk;
+    const uint8_t *xr = x + row * ldx * kElem;
+    float v[kApplyGroups][8];
+#pragma unroll
+    for (int g = 0; g < kApplyGroups; ++g) {
+        const int64_t e = e0 + 8 * (int64_t)(g * kApplyThreads + threadIdx.x);
+        if (e < V) split_load8<BF16>(xr, e, v[g]);
+    }
+    const float2 st = __ldg(row_stats + row);
+    const float m = st.x, ls = st.y;
+    float *yr = y + row * V;
+#pragma unroll
+    for (int g = 0; g < kApplyGroups; ++g) {
+        const int64_t e = e0 + 8 * (int64_t)(g * kApplyThreads + threadIdx.x);
+        if (e >= V) break;
+        float4 *dst = reinterpret_cast<float4 *>(yr + e);
+        __stcs(dst, make_float4((v[g][0] - m) - ls, (v[g][1] - m) - ls, (v[g][2] - m) - ls, (v[g][3] - m) - ls));
+        __stcs(dst + 1, make_float4((v[g][4] - m) - ls, (v[g][5] - m) - ls, (v[g][6] - m) - ls, (v[g][7] - m) - ls));
+    }
+}
+
+// Any V and ldx: element e0 + g * T + t belongs to thread t.
+template <bool BF16>
+__global__ void __launch_bounds__(kApplyThreads) log_softmax_apply_scalar_kernel(
+    const void *__restrict__ xv, int64_t ldx, const float2 *__restrict__ row_stats,
+    float *__restrict__ y, int64_t V, int64_t row0)
+{
+    const int64_t row = row0 + blockIdx.y;
+    const int64_t e0 = blockIdx.x * (int64_t)kApplyChunk;
+    const float2 st = __ldg(row_stats + row);
+    const float m = st.x, ls = st.y;
+    for (int64_t e = e0 + threadIdx.x; e < V && e < e0 + kApplyChunk; e += kApplyThreads) {
+        const float xe = BF16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(xv)[row * ldx + e])
+                              : static_cast<const float *>(xv)[row * ldx + e];
+        y[row * V + e] = (xe - m) - ls;
     }
 }
 

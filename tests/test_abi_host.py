@@ -82,6 +82,18 @@ def test_host_validation_without_a_gpu(lib):
     assert lib.bi_log_softmax(fake, 9, fake, 2, 8, NULL) == I
     assert lib.bi_log_softmax(fake + 4, 1, fake, 2, 8, NULL) == A
     assert lib.bi_silu_mul(NULL, NULL, 2, 8, NULL) == I
+    # LM-head log_softmax halves: null or misaligned pairs, short row stride
+    assert lib.bi_matmul_lse(fake, 8, fake, 8, 1, fake, 8, 0, NULL, 2, 8, 8, NULL) == I
+    assert lib.bi_matmul_lse(fake, 8, fake, 8, 1, fake, 8, 0, fake + 4, 2, 8, 8, NULL) == A
+    assert lib.bi_matmul_lse(NULL, 8, NULL, 8, 1, NULL, 8, 0, NULL, 0, 8, 8, NULL) == binding.BI_OK
+    assert lib.bi_log_softmax_partials(fake, 7, 0, fake, fake, fake, 2, 8, NULL) == I
+    assert lib.bi_log_softmax_partials(fake, 8, 0, NULL, fake, fake, 2, 8, NULL) == I
+    assert lib.bi_log_softmax_partials(fake, 8, 0, fake, NULL, fake, 2, 8, NULL) == I
+    assert lib.bi_log_softmax_partials(fake, 8, 0, fake + 4, fake, fake, 2, 8, NULL) == A
+    assert lib.bi_log_softmax_partials(fake, 8, 0, fake, fake + 4, fake, 2, 8, NULL) == A
+    assert lib.bi_log_softmax_partials(fake, 8, 3, fake, fake, fake, 2, 8, NULL) == I
+    assert lib.bi_log_softmax_partials(NULL, 8, 0, NULL, NULL, NULL, 0, 8, NULL) == binding.BI_OK
+    assert [lib.bi_lse_partials_per_row(n) for n in (0, 1, 256, 257, 151936)] == [0, 1, 1, 2, 594]
     assert lib.bi_selftest_wait_timeout(10, NULL) == I
     v = ctypes.c_int32(0)
     assert lib.bi_get_device_status(NULL, None) == I

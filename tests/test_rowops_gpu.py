@@ -62,7 +62,26 @@ def test_mean_parity_small(M, H):
     assert_mean_close(y, oracle.mean(xn), xn, f"mean M={M} H={H}")
 
 
-@pytest.mark.parametrize("H", [256, 4096])
+@pytest.mark.parametrize("H", [16384, 151936, 16388, 16387])
+def test_mean_parity_long_rows(H):
+    """Long rows (the step's mean runs over 151936 log-probs), on the vector path and, for a
+    row length that breaks the 16-byte rule (16387), the scalar path."""
+    x = inputs.rows_normal_outliers(113 + H, 0, 5, H, torch.float32)
+    y = bi.bi_mean(x.to(DEV))
+    xn = x.numpy()
+    assert_mean_close(y, oracle.mean(xn), xn, f"mean long rows H={H}")
+
+
+def test_mean_long_rows_batch_invariance():
+    H = 151936
+    pool = inputs.rows_normal_outliers(115, 0, 512, H, torch.float32).to(DEV)
+    _check_invariance(lambda x: bi.bi_mean(x), pool, [1, 2, 3, 8, 64, 77, 148, 256, 512], 116)
+    first = bi.bi_mean(pool)
+    for _ in range(100):
+        assert same_bits(bi.bi_mean(pool), first)
+
+
+@pytest.mark.parametrize("H", [256, 4096, 131072])
 def test_mean_integer_exact(H):
     x = inputs.rows_int(111, 0, 9, H, dtype=torch.float32)
     y = bi.bi_mean(x.to(DEV)).cpu().double().numpy()
@@ -81,7 +100,7 @@ def test_mean_workload_sampled_rows():
 
 # ----------------------------------------------------------------------------- log_softmax
 
-@pytest.mark.parametrize("V", [1000, 8, 999, 4096])
+@pytest.mark.parametrize("V", [1000, 8, 999, 4096, 16384, 98304, 98312, 151936])
 @pytest.mark.parametrize("M", [1, 3, 17])
 def test_log_softmax_parity_fp32(M, V):
     x = inputs.rows_normal(120 + V, 0, M, V, dtype=torch.float32)
@@ -89,9 +108,11 @@ def test_log_softmax_parity_fp32(M, V):
     assert_lsm_close(y, oracle.log_softmax(x.numpy()), f"log_softmax fp32 M={M} V={V}")
 
 
-# 1001 takes the scalar path, the others the streamed path (ring of 6 stages: rows of 1, 6, 7,
-# 10 and 19 chunks).
-@pytest.mark.parametrize("V", [151936, 1000, 1001, 110000, 155648, 155656, 4096])
+# 1001 takes the scalar path; rows of >= 64 KB up to 4 x 96 KB (32768 <= V <= 196608 for bf16)
+# one cluster of 4 CTAs per row; the others the streamed path (a ring of 6 stages: rows of 1, 2,
+# 25 and 48 chunks).
+@pytest.mark.parametrize("V", [151936, 1000, 1001, 110000, 155648, 155656, 4096, 32760, 32768, 196608,
+                               196616, 393216])
 def test_log_softmax_parity_bf16(V):
     M = 5
     x = inputs.rows_normal(121, 0, M, V, std=1.3)
@@ -164,6 +185,14 @@ def test_log_softmax_batch_invariance():
     V = 151936
     pool = inputs.rows_normal(145, 0, 256, V, std=1.3).to(DEV)
     _check_invariance(lambda x: bi.bi_log_softmax(x), pool, [1, 2, 3, 8, 64, 77, 128, 256], 146)
+
+
+def test_log_softmax_streamed_rows_batch_invariance():
+    V = 393216  # beyond the cluster path's slice limit: the streamed one-block-per-row kernel
+    pool = inputs.rows_normal(149, 0, 64, V, std=1.3).to(DEV)
+    _check_invariance(lambda x: bi.bi_log_softmax(x), pool, [1, 2, 3, 17, 64], 150)
+    xf = pool[:8].float()
+    _check_invariance(lambda x: bi.bi_log_softmax(x), xf, [1, 3, 8], 151)
 
 
 def test_row_ops_repeatable_100_runs():
