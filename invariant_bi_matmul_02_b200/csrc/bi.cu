@@ -391,7 +391,10 @@ bi_status bi_mean(const float *x, float *y, int64_t M, int64_t H, void *stream)
     const int T = bi::mean_threads(H);
     if (H % 4 == 0) {
         if (!aligned16(x)) return BI_ERR_ALIGNMENT;
-        bi::mean_vec_kernel<<<(unsigned)M, T, 0, s>>>(reinterpret_cast<const float4 *>(x), y, H);
+        if (H / 4 >= 8 * (int64_t)T)
+            bi::mean_vec_kernel<true><<<(unsigned)M, T, 0, s>>>(reinterpret_cast<const float4 *>(x), y, H);
+        else
+            bi::mean_vec_kernel<false><<<(unsigned)M, T, 0, s>>>(reinterpret_cast<const float4 *>(x), y, H);
     } else {
         bi::mean_scalar_kernel<<<(unsigned)M, T, 0, s>>>(x, y, H);
     }

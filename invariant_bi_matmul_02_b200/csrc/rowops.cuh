@@ -160,6 +160,10 @@ __global__ void __launch_bounds__(1024) rmsnorm_scalar_kernel(const __nv_bfloat1
 
 // Vector path: H % 4 == 0.  Chunk c (4 floats) belongs to thread c % T; each thread
 // keeps four running sums (one per float4 lane) and folds them as (s0+s1)+(s2+s3).
+// LONG: eight float4 loads in flight per thread (rows of >= 8 T groups, which run one 1024-thread
+// block per SM); otherwise four.  The adds keep the ascending group order in both, so the sums
+// are the same bits either way.
+template <bool LONG>
 __global__ void __launch_bounds__(1024) mean_vec_kernel(const float4 *__restrict__ x,
                                                        float *__restrict__ y, int64_t H)
 {
@@ -169,6 +173,17 @@ __global__ void __launch_bounds__(1024) mean_vec_kernel(const float4 *__restrict
     float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
     int64_t c = threadIdx.x;
     const int T = blockDim.x;
+    if (LONG) {
+        for (; c + 7 * (int64_t)T < nch; c += 8 * (int64_t)T) {
+            float4 g[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) g[k] = __ldg(xr + c + k * (int64_t)T);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                s0 += g[k].x; s1 += g[k].y; s2 += g[k].z; s3 += g[k].w;
+            }
+        }
+    }
     for (; c + 3 * (int64_t)T < nch; c += 4 * (int64_t)T) {
         float4 a = __ldg(xr + c), b = __ldg(xr + c + T), d = __ldg(xr + c + 2 * T),
                e = __ldg(xr + c + 3 * T);
