@@ -361,23 +361,54 @@ def run_bi(args):
             per_op[op] += marks[s][i].elapsed_time(marks[s][i + 1])
     per_op = {k: v / args.steps for k, v in per_op.items()}
 
-    # end to end through the public API: pinned host input in, per-row result out, every step
+    # End to end through the public API: every step copies its input rows from pinned host
+    # memory and the host reads the step's per-row result back.  The copy for step s+1 runs on
+    # a copy stream while step s computes (two device input buffers), and the host reads step
+    # s's result while step s+1 is queued, so the GPU is never left waiting on the host.
     x_pinned = wl.x_host.pin_memory()
-    ce_pinned = torch.empty(M, dtype=torch.float32).pin_memory()
-    x_dev = torch.empty_like(wl.x)
+    ce_pinned = [torch.empty(M, dtype=torch.float32).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(wl.x) for _ in range(2)]
+    copy_stream = torch.cuda.Stream()
     e2e_steps = max(1, min(args.steps, 100))
-    for _ in range(2):
-        x_dev.copy_(x_pinned, non_blocking=True)
-        ce_pinned.copy_(run_step(wl, x_dev), non_blocking=True)
-        stream.synchronize()
+    host_sum = [0.0]
+
+    def e2e_run(n, start_ev=None):
+        copied = [torch.cuda.Event() for _ in range(2)]
+        consumed = [torch.cuda.Event() for _ in range(2)]
+        read = [torch.cuda.Event() for _ in range(2)]
+        if start_ev is not None:
+            copy_stream.wait_event(start_ev)
+        with torch.cuda.stream(copy_stream):
+            x_dev[0].copy_(x_pinned, non_blocking=True)
+            copied[0].record(copy_stream)
+        for s in range(n):
+            i = s % 2
+            if s + 1 < n:
+                j = (s + 1) % 2
+                with torch.cuda.stream(copy_stream):
+                    if s >= 1:
+                        copy_stream.wait_event(consumed[j])  # step s-1 is done with buffer j
+                    x_dev[j].copy_(x_pinned, non_blocking=True)
+                    copied[j].record(copy_stream)
+            stream.wait_event(copied[i])
+            ce = run_step(wl, x_dev[i])
+            consumed[i].record(stream)
+            if s >= 2:
+                read[i].synchronize()  # ce_pinned[i] (step s-2) has been read; reuse it
+            ce_pinned[i].copy_(ce, non_blocking=True)
+            read[i].record(stream)
+            if s >= 1:
+                read[(s - 1) % 2].synchronize()  # the host reads step s-1's result
+                host_sum[0] += float(ce_pinned[(s - 1) % 2][0])
+        read[(n - 1) % 2].synchronize()
+        host_sum[0] += float(ce_pinned[(n - 1) % 2][0])
+
+    e2e_run(2)
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        x_dev.copy_(x_pinned, non_blocking=True)
-        ce_pinned.copy_(run_step(wl, x_dev), non_blocking=True)
-        stream.synchronize()  # the host reads the step's result
+    e2e_run(e2e_steps, e0)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
