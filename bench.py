@@ -13,7 +13,7 @@ One *step* is one pass of every kernel of the path over a batch of M token rows
     y    = bi_addmm(o, a, W_down)                     [M, 4096]    residual add
     hf   = bi_rmsnorm(y, g_final)
     lg   = bi_matmul(hf, W_lm)                        [M, 151936]  bf16 logits
-    lp   = bi_log_softmax(lg)                         [M, 151936]  fp32, one cluster of 8 CTAs per row
+    lp   = bi_log_softmax(lg)                         [M, 151936]  fp32, one block per row
                                                                    (--lsm partials: bi_matmul_lse also
                                                                    leaves one (max, sum exp) pair per
                                                                    row and 256-column tile, and
@@ -638,7 +638,9 @@ def run_sweep(args):
                                 "torch_us": t_mt * 1e3, "torch_gbs": bym / t_mt / 1e6})
             print(f"{'mean_vocab':12s} {M:6d} {t_m*1e3:9.1f} {bym/t_m/1e6:8.0f} "
                   f"{100*bym/t_m/1e6/peaks['hbm_gbs']:5.1f}% {t_mt*1e3:9.1f} {bym/t_mt/1e6:10.0f}", flush=True)
-            for op, t in (("log_softmax", t_bi), ("log_softmax_split", t_sp), ("log_softmax_partials", t_pa)):
+            t_cl = _timed(lambda: bi.bi_log_softmax_cluster(x, out=y), flush, reps)
+            for op, t in (("log_softmax", t_bi), ("log_softmax_cluster", t_cl), ("log_softmax_split", t_sp),
+                          ("log_softmax_partials", t_pa)):
                 out["rows"].append({"op": op, "M": M, "bi_us": t * 1e3, "bi_gbs": by / t / 1e6,
                                     "bi_frac_hbm": by / t / 1e6 / peaks["hbm_gbs"],
                                     "torch_us": t_t * 1e3, "torch_gbs": by / t_t / 1e6})
@@ -663,6 +665,7 @@ KERNEL_CASES = {
     "mean": "bi_mean M=16384 H=4096 fp32",
     "mean_vocab": "bi_mean M=1024 H=151936 fp32 (the step's mean over log-probs)",
     "log_softmax": "bi_log_softmax M=1024 V=151936 bf16 -> fp32",
+    "log_softmax_cluster": "bi_log_softmax_cluster M=1024 V=151936 bf16 -> fp32 (4 CTAs per row)",
     "log_softmax_partials": "bi_log_softmax_partials M=1024 V=151936 bf16 -> fp32 (pairs precomputed)",
     "silu_mul": "bi_silu_mul M=1024 F=12288",
     "decode_attention": "bi_decode_attention B=64 L=4096, 32 q / 8 kv heads of 128",
@@ -717,6 +720,11 @@ def run_kernel_case(args):
         x = inputs.rows_normal(54, 0, 1024, VOCAB, std=1.3).to(dev)
         y = torch.empty(1024, VOCAB, dtype=torch.float32, device=dev)
         fn = lambda: bi.bi_log_softmax(x, out=y)
+        work, unit = 6 * VOCAB * 1024, "GB/s"
+    elif name == "log_softmax_cluster":
+        x = inputs.rows_normal(54, 0, 1024, VOCAB, std=1.3).to(dev)
+        y = torch.empty(1024, VOCAB, dtype=torch.float32, device=dev)
+        fn = lambda: bi.bi_log_softmax_cluster(x, out=y)
         work, unit = 6 * VOCAB * 1024, "GB/s"
     elif name == "log_softmax_partials":
         a = inputs.rows_normal(50, 0, 1024, HIDDEN).to(dev)

@@ -198,12 +198,31 @@ bi_status bi_mean(const float *x, float *y, int64_t M, int64_t H, void *stream);
  *
  *   x  device, [M, V] contiguous, x_dtype BI_F32 or BI_BF16 (bf16 is widened exactly);
  *   y  device, fp32, [M, V].
- *   Per-thread running (max, sum) pairs merged through a fixed tree; the row is read
- *   twice (once for the statistics, once to write y).
+ *   One thread block per row.  Per-thread running (max, sum) pairs merged through a fixed
+ *   tree; the row is read twice (once for the statistics, once to write y; the last chunks of
+ *   the first pass are still in shared memory for the second).
  *   x and y 16-byte aligned when V is a multiple of 8 (bf16) / 4 (f32), the vector path.
  */
 bi_status bi_log_softmax(const void *x, bi_dtype x_dtype, float *y, int64_t M, int64_t V,
                          void *stream);
+
+/*
+ * bi_log_softmax_cluster -- the same y as bi_log_softmax, for long rows, computed by a cluster of
+ * 4 CTAs per row (an opt-in variant: bi_log_softmax keeps one CTA per row).  Passage: as
+ * bi_log_softmax.  The row is cut into 4 slices of S = 8 * ceil(V / 32) elements, a cut fixed by V
+ * alone; each CTA bulk-copies its slice into shared memory, reduces it to a (max, sum of exp)
+ * pair, and every CTA folds the 4 pairs in rank order (distributed shared memory) before
+ * writing its slice of y from shared memory, so the row is read from memory once.  The result
+ * is batch-invariant; it is a different fixed order from bi_log_softmax's, so the two agree to
+ * the tolerance, not bit for bit.
+ *
+ *   x, x_dtype, y, M, V as bi_log_softmax; x and y 16-byte aligned.
+ *   Rows it takes: V % 8 == 0 (bf16) or V % 4 == 0 (fp32), V * element size >= 64 KiB and
+ *   S * element size <= 96 KiB, i.e. 32768 <= V <= 196608 for bf16 and 16384 <= V <= 98304 for
+ *   fp32.  Any other V returns BI_ERR_UNSUPPORTED without launching.
+ */
+bi_status bi_log_softmax_cluster(const void *x, bi_dtype x_dtype, float *y, int64_t M, int64_t V,
+                                 void *stream);
 
 /*
  * bi_log_softmax_split -- the same y as bi_log_softmax, computed by many blocks per row, for

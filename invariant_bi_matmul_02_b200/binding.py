@@ -37,6 +37,7 @@ SIGNATURES = {
     "bi_rmsnorm": (ctypes.c_int, [_p, _p, _p, _i64, _i64, ctypes.c_float, _p]),
     "bi_mean": (ctypes.c_int, [_p, _p, _i64, _i64, _p]),
     "bi_log_softmax": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p]),
+    "bi_log_softmax_cluster": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p]),
     "bi_log_softmax_split": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p, ctypes.c_size_t, _p]),
     "bi_log_softmax_split_scratch_bytes": (ctypes.c_size_t, [_i64, _i64]),
     "bi_log_softmax_split_noalloc": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p]),
@@ -303,6 +304,21 @@ def bi_log_softmax(x: torch.Tensor, out: torch.Tensor | None = None, stream=None
     _contig(out, "y")
     _check("bi_log_softmax", load().bi_log_softmax(x.data_ptr(), _DT[x.dtype], out.data_ptr(), M, V,
                                                    _stream(stream)))
+    return out
+
+
+def bi_log_softmax_cluster(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """log_softmax over the last dimension by a cluster of 4 CTAs per row (long rows only:
+    32768 <= V <= 196608 for bf16, 16384 <= V <= 98304 for fp32)."""
+    _need_cuda(x, "x", (torch.float32, torch.bfloat16))
+    _contig(x, "x")
+    M, V = x.shape
+    if out is None:
+        out = torch.empty((M, V), dtype=torch.float32, device=x.device)
+    _need_cuda(out, "y", (torch.float32,))
+    _contig(out, "y")
+    _check("bi_log_softmax_cluster", load().bi_log_softmax_cluster(x.data_ptr(), _DT[x.dtype], out.data_ptr(), M,
+                                                                   V, _stream(stream)))
     return out
 
 

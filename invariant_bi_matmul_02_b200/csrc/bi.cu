@@ -418,15 +418,6 @@ bi_status bi_log_softmax(const void *x, bi_dtype x_dtype, float *y, int64_t M, i
         bi_status st = device_state(&dev);
         if (st != BI_OK) return st;
         const uint8_t *xb = static_cast<const uint8_t *>(x);
-        const int elem = bf16 ? 2 : 4;
-        const int64_t slice_bytes = bi::cluster_slice(V) * elem;
-        if (V * elem >= bi::kClusterRowBytes && slice_bytes <= bi::kClSliceBytesMax) {  // a cluster per row
-            st = bf16 ? launch_row_clusters(bi::log_softmax_cluster_kernel<true>, M, (size_t)slice_bytes, s, xb, y, V,
-                                            dev->status, kWaitLimitNs)
-                      : launch_row_clusters(bi::log_softmax_cluster_kernel<false>, M, (size_t)slice_bytes, s, xb, y,
-                                            V, dev->status, kWaitLimitNs);
-            return st != BI_OK ? st : launched();
-        }
         if (bf16)
             bi::log_softmax_stream_kernel<true><<<(unsigned)M, bi::kLsmThreads, bi::kLsmSmem, s>>>(
                 xb, y, V, dev->status, kWaitLimitNs);
@@ -440,6 +431,31 @@ bi_status bi_log_softmax(const void *x, bi_dtype x_dtype, float *y, int64_t M, i
             bi::log_softmax_scalar_kernel<false><<<(unsigned)M, T, 0, s>>>(x, y, V);
     }
     return launched();
+}
+
+bi_status bi_log_softmax_cluster(const void *x, bi_dtype x_dtype, float *y, int64_t M, int64_t V, void *stream)
+{
+    if (M < 0 || V < 0) return BI_ERR_INVALID_ARG;
+    if (x_dtype != BI_BF16 && x_dtype != BI_F32) return BI_ERR_INVALID_ARG;
+    if (M > kI32Max || V > kI32Max) return BI_ERR_UNSUPPORTED;
+    if (M == 0) return BI_OK;
+    if (V == 0 || !x || !y) return BI_ERR_INVALID_ARG;
+    const bool bf16 = x_dtype == BI_BF16;
+    const int elem = bf16 ? 2 : 4;
+    const int64_t slice_bytes = bi::cluster_slice(V) * elem;
+    if (V % (bf16 ? 8 : 4) != 0 || V * elem < bi::kClusterRowBytes || slice_bytes > bi::kClSliceBytesMax)
+        return BI_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(y)) return BI_ERR_ALIGNMENT;
+    DeviceState *dev = nullptr;
+    bi_status st = device_state(&dev);
+    if (st != BI_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint8_t *xb = static_cast<const uint8_t *>(x);
+    st = bf16 ? launch_row_clusters(bi::log_softmax_cluster_kernel<true>, M, (size_t)slice_bytes, s, xb, y, V,
+                                    dev->status, kWaitLimitNs)
+              : launch_row_clusters(bi::log_softmax_cluster_kernel<false>, M, (size_t)slice_bytes, s, xb, y, V,
+                                    dev->status, kWaitLimitNs);
+    return st != BI_OK ? st : launched();
 }
 
 size_t bi_log_softmax_split_scratch_bytes(int64_t M, int64_t V)

@@ -384,8 +384,9 @@ constexpr int kLsmSmem = kLsmStages * kLsmChunk;
 
 // --------------------------------------------------------------- long rows: one cluster per row
 
-// log_softmax rows of at least kClusterRowBytes bytes (vector path) whose slices fit in shared
-// memory are reduced by a cluster of kRowCluster CTAs.  CTA r owns the slice [r S, min(V, (r + 1) S)) of the row, with
+// The cluster variant of log_softmax (bi_log_softmax_cluster, an opt-in entry point beside the
+// one-block-per-row bi_log_softmax): rows of at least kClusterRowBytes bytes whose slices fit in
+// shared memory are reduced by a cluster of kRowCluster CTAs.  CTA r owns the slice [r S, min(V, (r + 1) S)) of the row, with
 // S = cluster_slice(V) a multiple of 8 elements fixed by V alone.  Each CTA reduces its slice
 // in a fixed order; the CTAs' results meet through distributed shared memory and are folded in
 // rank order 0, 1, ..., kRowCluster - 1.  A short batch spreads over kRowCluster times as many

@@ -108,9 +108,8 @@ def test_log_softmax_parity_fp32(M, V):
     assert_lsm_close(y, oracle.log_softmax(x.numpy()), f"log_softmax fp32 M={M} V={V}")
 
 
-# 1001 takes the scalar path; rows of >= 64 KB up to 4 x 96 KB (32768 <= V <= 196608 for bf16)
-# one cluster of 4 CTAs per row; the others the streamed path (a ring of 6 stages: rows of 1, 2,
-# 25 and 48 chunks).
+# 1001 takes the scalar path, the others the streamed path (a ring of 6 stages of 16 KB: rows of
+# 1, 4, 14, 19, 24, 25 and 48 chunks).
 @pytest.mark.parametrize("V", [151936, 1000, 1001, 110000, 155648, 155656, 4096, 32760, 32768, 196608,
                                196616, 393216])
 def test_log_softmax_parity_bf16(V):
@@ -188,7 +187,7 @@ def test_log_softmax_batch_invariance():
 
 
 def test_log_softmax_streamed_rows_batch_invariance():
-    V = 393216  # beyond the cluster path's slice limit: the streamed one-block-per-row kernel
+    V = 393216  # 48 ring chunks per row
     pool = inputs.rows_normal(149, 0, 64, V, std=1.3).to(DEV)
     _check_invariance(lambda x: bi.bi_log_softmax(x), pool, [1, 2, 3, 17, 64], 150)
     xf = pool[:8].float()
