@@ -937,7 +937,7 @@ def main():
                          "the GEMM epilogue and one pass (bi_matmul_lse + bi_log_softmax_partials)")
     ap.add_argument("--mlp", choices=["fused", "unfused"], default="fused",
                     help="gate/up + SiLU*up as one fused GEMM (default) or GEMM then bi_silu_mul")
-    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--cpu-budget", type=float, default=25.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="per-kernel M sweeps (table, not JSON line)")
     ap.add_argument("--sweep-shapes", default="", help="comma list of sweep groups (q/o,k/v,...,rows)")
