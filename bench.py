@@ -243,10 +243,15 @@ def cpu_baseline(host: dict, x_host, budget_s: float = 15.0) -> dict:
     t0 = time.perf_counter()
     oracle_step_rows(host, x_host[:rows], cores)
     dt = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle_step_rows(host, x_host[:1], 1)  # the same oracle on one core
+    dt1 = time.perf_counter() - t0
     return {"value": rows * gemm_flops_per_row() / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
             "kind": "oracle",
             "sample": f"{rows} of {x_host.shape[0]} rows through the whole step in fp64 "
-                      f"({dt:.1f} s, after a 1-row calibration of {t1:.2f} s)"}
+                      f"({dt:.1f} s, after a 1-row calibration of {t1:.2f} s)",
+            "value_1core": gemm_flops_per_row() / dt1 / 1e12,
+            "sample_1core": f"1 row through the whole step in fp64 on one thread ({dt1:.2f} s)"}
 
 
 # ----------------------------------------------------------------------------- clocks
