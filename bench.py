@@ -552,9 +552,20 @@ def _timed(fn, flush, reps):
     return statistics.median(times)
 
 
+def _rows_differing(t, ref1):
+    """Rows of t whose bits differ from the same rows computed alone (ref1)."""
+    import torch
+    n = ref1.shape[0]
+    view = torch.int16 if t.element_size() == 2 else torch.int32
+    return int((t[:n].contiguous().view(view) != ref1.contiguous().view(view)).any(dim=1).sum())
+
+
 def run_sweep(args):
     """Per-kernel M sweeps: bi kernels vs torch defaults, L2 flushed before every rep.
-    Also counts, for torch's defaults, rows whose bits differ from their M = 1 result."""
+    For the first 64 rows of every M, both bi's and torch's outputs are compared bit for bit
+    with the same rows computed alone (M = 1): bi must differ in none (invariance), torch's
+    count is the negative control.  With --sweep-out the JSON is rewritten after every point,
+    and --resume skips the points already in it."""
     import torch
     import torch.nn.functional as F
     from invariant_bi_matmul_02_b200 import binding as bi
@@ -566,95 +577,142 @@ def run_sweep(args):
     flush = lambda: scratch.fill_(1.0)
     reps = max(5, min(args.steps, 30))
     out = {"peaks": peaks, "peak_source": src, "gemm": [], "rows": []}
+    if args.resume and args.sweep_out and os.path.exists(args.sweep_out):
+        with open(args.sweep_out) as f:
+            prev = json.load(f)
+        out["gemm"], out["rows"] = prev.get("gemm", []), prev.get("rows", [])
+    have = {("gemm", r["shape"], r["M"]) for r in out["gemm"]} | {("rows", r["op"], r["M"]) for r in out["rows"]}
+
+    def save():
+        if args.sweep_out:
+            tmp = args.sweep_out + ".tmp"
+            with open(tmp, "w") as f:
+                json.dump(out, f, indent=1)
+            os.replace(tmp, args.sweep_out)
+
+    def row_rec(op, M, t_bi, by, t_t, bi_diff, t_diff, n):
+        rec = {"op": op, "M": M, "bi_us": t_bi * 1e3, "bi_gbs": by / t_bi / 1e6,
+               "bi_frac_hbm": by / t_bi / 1e6 / peaks["hbm_gbs"], "torch_us": t_t * 1e3,
+               "torch_gbs": by / t_t / 1e6, "bi_rows_differing_from_m1": bi_diff,
+               "torch_rows_differing_from_m1": t_diff, "rows_compared": n}
+        out["rows"].append(rec)
+        save()
+        print(f"{op:20s} {M:6d} {t_bi*1e3:9.1f} {by/t_bi/1e6:8.0f} {100*by/t_bi/1e6/peaks['hbm_gbs']:5.1f}% "
+              f"{t_t*1e3:9.1f} {by/t_t/1e6:10.0f} {bi_diff:>5d}/{n} {t_diff:>5d}/{n}", flush=True)
+
     print(f"peaks ({src}): {peaks}")
     print(f"{'shape':9s} {'M':>5s} {'bi us':>9s} {'bi TF/s':>8s} {'%pk':>6s} {'GB/s':>7s} "
-          f"{'torch us':>9s} {'torch TF/s':>10s} {'torch rows != M=1':>18s}")
+          f"{'torch us':>9s} {'torch TF/s':>10s} {'bi != M=1':>10s} {'torch != M=1':>12s}")
     for name, K, N in SWEEP_SHAPES:
         if args.sweep_shapes and name not in args.sweep_shapes.split(","):
             continue
+        if all(("gemm", name, M) in have for M in SWEEP_M):
+            continue
         w = inputs.weight_normal(40, (N, K)).to(dev)
         pool = inputs.rows_normal(41, 0, max(SWEEP_M), K).to(dev)
-        ref_torch = F.linear(pool[:64], w)  # torch's own rows computed at M = 64 ...
-        ref1 = torch.cat([F.linear(pool[i:i + 1], w) for i in range(64)])  # ... and at M = 1
+        ref1 = torch.cat([F.linear(pool[i:i + 1], w) for i in range(64)])  # torch's rows at M = 1
+        ref1_bi = torch.cat([bi.bi_matmul(pool[i:i + 1], w, "nk") for i in range(64)])
         for M in SWEEP_M:
+            if ("gemm", name, M) in have:
+                continue
             a = pool[:M]
             c = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
             t_bi = _timed(lambda: bi.bi_matmul(a, w, "nk", out=c), flush, reps)
+            n = min(M, 64)
+            bi_diff = _rows_differing(c, ref1_bi[:n])
             t_t = _timed(lambda: torch.mm(a, w.t(), out=c), flush, reps)
+            diff = _rows_differing(F.linear(a, w), ref1[:n])
             fl = 2 * M * N * K
             by = gemm_bytes(M, K, N)
-            rows_cmp = min(M, 64)
-            tc = F.linear(a, w)[:rows_cmp]
-            diff = int((tc.view(torch.int16) != ref1[:rows_cmp].view(torch.int16)).any(dim=1).sum())
             rec = {"shape": name, "K": K, "N": N, "M": M, "bi_us": t_bi * 1e3,
                    "bi_tflops": fl / t_bi / 1e9, "bi_frac_tensor": fl / t_bi / 1e9 / peaks["bf16_tflops"],
                    "bi_gbs": by / t_bi / 1e6, "bi_frac_hbm": by / t_bi / 1e6 / peaks["hbm_gbs"],
                    "torch_us": t_t * 1e3, "torch_tflops": fl / t_t / 1e9,
-                   "torch_rows_differing_from_m1": diff, "rows_compared": rows_cmp}
+                   "bi_rows_differing_from_m1": bi_diff,
+                   "torch_rows_differing_from_m1": diff, "rows_compared": n}
             out["gemm"].append(rec)
+            save()
             print(f"{name:9s} {M:5d} {t_bi*1e3:9.1f} {rec['bi_tflops']:8.1f} "
                   f"{100*rec['bi_frac_tensor']:5.1f}% {rec['bi_gbs']:7.0f} {t_t*1e3:9.1f} "
-                  f"{rec['torch_tflops']:10.1f} {diff:>10d}/{rows_cmp}", flush=True)
-        del w, pool, ref_torch, ref1
+                  f"{rec['torch_tflops']:10.1f} {bi_diff:>7d}/{n} {diff:>9d}/{n}", flush=True)
+        del w, pool, ref1, ref1_bi
         torch.cuda.empty_cache()
     if not args.sweep_shapes or "rows" in args.sweep_shapes.split(","):
-        print(f"{'op':12s} {'M':>6s} {'bi us':>9s} {'GB/s':>8s} {'%HBM':>6s} {'torch us':>9s} {'torch GB/s':>10s}")
+        print(f"{'op':20s} {'M':>6s} {'bi us':>9s} {'GB/s':>8s} {'%HBM':>6s} {'torch us':>9s} {'torch GB/s':>10s} "
+              f"{'bi!=M=1':>7s} {'torch!=M=1':>10s}")
         g = inputs.gain(42, HIDDEN).to(dev)
+        x64 = inputs.rows_normal_outliers(43, 0, 64, HIDDEN, torch.bfloat16).to(dev)  # rows are seed-keyed
+        ones = {
+            "rmsnorm": (torch.cat([bi.bi_rmsnorm(x64[i:i + 1], g, EPS) for i in range(64)]),
+                        torch.cat([F.rms_norm(x64[i:i + 1], (HIDDEN,), g, EPS) for i in range(64)])),
+            "mean": (torch.cat([bi.bi_mean(x64[i:i + 1].float()) for i in range(64)])[:, None],
+                     torch.cat([x64[i:i + 1].float().mean(-1) for i in range(64)])[:, None]),
+        }
         for M in [1, 8, 64, 148, 256, 1024, 4096, 8192, 16384, 3, 77, 1000]:
+            if ("rows", "rmsnorm", M) in have and ("rows", "mean", M) in have:
+                continue
             x = inputs.rows_normal_outliers(43, 0, M, HIDDEN, torch.bfloat16).to(dev)
             xf = x.float()
             y = torch.empty_like(x)
             ym = torch.empty(M, dtype=torch.float32, device=dev)
+            n = min(M, 64)
             for op, fn, tfn, by in (
                 ("rmsnorm", lambda: bi.bi_rmsnorm(x, g, EPS, out=y),
                  lambda: F.rms_norm(x, (HIDDEN,), g, EPS), 4 * HIDDEN * M),
                 ("mean", lambda: bi.bi_mean(xf, out=ym), lambda: xf.mean(-1), (4 * HIDDEN + 4) * M)):
                 t_bi = _timed(fn, flush, reps)
+                bi_out = (y if op == "rmsnorm" else ym[:, None])
+                bi_diff = _rows_differing(bi_out, ones[op][0][:n])
                 t_t = _timed(tfn, flush, reps)
-                out["rows"].append({"op": op, "M": M, "bi_us": t_bi * 1e3, "bi_gbs": by / t_bi / 1e6,
-                                    "bi_frac_hbm": by / t_bi / 1e6 / peaks["hbm_gbs"],
-                                    "torch_us": t_t * 1e3, "torch_gbs": by / t_t / 1e6})
-                print(f"{op:12s} {M:6d} {t_bi*1e3:9.1f} {by/t_bi/1e6:8.0f} "
-                      f"{100*by/t_bi/1e6/peaks['hbm_gbs']:5.1f}% {t_t*1e3:9.1f} {by/t_t/1e6:10.0f}",
-                      flush=True)
+                t_out = tfn()
+                t_diff = _rows_differing(t_out if op == "rmsnorm" else t_out[:, None], ones[op][1][:n])
+                row_rec(op, M, t_bi, by, t_t, bi_diff, t_diff, n)
+        xv64 = inputs.rows_normal(44, 0, 64, VOCAB, std=1.3).to(dev)
+        one_v = {"log_softmax": torch.cat([bi.bi_log_softmax(xv64[i:i + 1]) for i in range(64)]),
+                 "log_softmax_cluster": torch.cat([bi.bi_log_softmax_cluster(xv64[i:i + 1]) for i in range(64)]),
+                 "log_softmax_split": torch.cat([bi.bi_log_softmax_split(xv64[i:i + 1]) for i in range(64)]),
+                 "torch": torch.cat([torch.log_softmax(xv64[i:i + 1], -1, dtype=torch.float32) for i in range(64)])}
+        lp64 = one_v["log_softmax"]  # the step's mean runs over log-probs
+        one_m = (torch.cat([bi.bi_mean(lp64[i:i + 1]) for i in range(64)])[:, None],
+                 torch.cat([lp64[i:i + 1].mean(-1) for i in range(64)])[:, None])
         for M in [1, 8, 64, 256, 1024]:
+            ops_v = ("log_softmax", "log_softmax_cluster", "log_softmax_split", "log_softmax_partials", "mean_vocab")
+            if all(("rows", op, M) in have for op in ops_v):
+                continue
             x = inputs.rows_normal(44, 0, M, VOCAB, std=1.3).to(dev)
             y = torch.empty(M, VOCAB, dtype=torch.float32, device=dev)
             by = 6 * VOCAB * M
-            t_bi = _timed(lambda: bi.bi_log_softmax(x, out=y), flush, reps)
+            n = min(M, 64)
             t_t = _timed(lambda: torch.log_softmax(x, -1, dtype=torch.float32), flush, reps)
+            t_diff = _rows_differing(torch.log_softmax(x, -1, dtype=torch.float32), one_v["torch"][:n])
+            t_bi = _timed(lambda: bi.bi_log_softmax(x, out=y), flush, reps)
+            row_rec("log_softmax", M, t_bi, by, t_t, _rows_differing(y, one_v["log_softmax"][:n]), t_diff, n)
+            lp = y.clone()
+            t_cl = _timed(lambda: bi.bi_log_softmax_cluster(x, out=y), flush, reps)
+            row_rec("log_softmax_cluster", M, t_cl, by, t_t,
+                    _rows_differing(y, one_v["log_softmax_cluster"][:n]), t_diff, n)
             scr = torch.empty(bi.bi_log_softmax_split_scratch_bytes(M, VOCAB), dtype=torch.uint8, device=dev)
             t_sp = _timed(lambda: bi.bi_log_softmax_split(x, scr, out=y), flush, reps)
-            # second half of the LM-head path: the pairs come from a GEMM epilogue; here they are
-            # taken from a GEMM whose logits then stand in for x (same pass, same bytes)
+            row_rec("log_softmax_split", M, t_sp, by, t_t, _rows_differing(y, one_v["log_softmax_split"][:n]),
+                    t_diff, n)
+            # second half of the LM-head path: the pairs come from a GEMM epilogue, so its x is that
+            # GEMM's logits (same pass, same bytes); its invariance is tested in tests/test_lse_gpu.py
             aw = inputs.rows_normal(45, 0, M, HIDDEN).to(dev)
             ww = inputs.weight_normal(46, (VOCAB, HIDDEN)).to(dev)
             xl, part = bi.bi_matmul_lse(aw, ww, "nk")
             del ww
             rs = torch.empty(M, 2, dtype=torch.float32, device=dev)
             t_pa = _timed(lambda: bi.bi_log_softmax_partials(xl, part, out=y, row_stats=rs), flush, reps)
-            xm = torch.empty(M, VOCAB, dtype=torch.float32, device=dev).normal_()
+            row_rec("log_softmax_partials", M, t_pa, by, t_t, 0, t_diff, 0)
+            del xl, part
             ym = torch.empty(M, dtype=torch.float32, device=dev)
-            t_m = _timed(lambda: bi.bi_mean(xm, out=ym), flush, reps)
-            t_mt = _timed(lambda: xm.mean(-1), flush, reps)
-            bym = (4 * VOCAB + 4) * M
-            out["rows"].append({"op": "mean_vocab", "M": M, "bi_us": t_m * 1e3, "bi_gbs": bym / t_m / 1e6,
-                                "bi_frac_hbm": bym / t_m / 1e6 / peaks["hbm_gbs"],
-                                "torch_us": t_mt * 1e3, "torch_gbs": bym / t_mt / 1e6})
-            print(f"{'mean_vocab':12s} {M:6d} {t_m*1e3:9.1f} {bym/t_m/1e6:8.0f} "
-                  f"{100*bym/t_m/1e6/peaks['hbm_gbs']:5.1f}% {t_mt*1e3:9.1f} {bym/t_mt/1e6:10.0f}", flush=True)
-            t_cl = _timed(lambda: bi.bi_log_softmax_cluster(x, out=y), flush, reps)
-            for op, t in (("log_softmax", t_bi), ("log_softmax_cluster", t_cl), ("log_softmax_split", t_sp),
-                          ("log_softmax_partials", t_pa)):
-                out["rows"].append({"op": op, "M": M, "bi_us": t * 1e3, "bi_gbs": by / t / 1e6,
-                                    "bi_frac_hbm": by / t / 1e6 / peaks["hbm_gbs"],
-                                    "torch_us": t_t * 1e3, "torch_gbs": by / t_t / 1e6})
-                print(f"{op:12s} {M:6d} {t*1e3:9.1f} {by/t/1e6:8.0f} "
-                      f"{100*by/t/1e6/peaks['hbm_gbs']:5.1f}% {t_t*1e3:9.1f} {by/t_t/1e6:10.0f}",
-                      flush=True)
-    if args.sweep_out:
-        with open(args.sweep_out, "w") as f:
-            json.dump(out, f, indent=1)
+            t_m = _timed(lambda: bi.bi_mean(lp, out=ym), flush, reps)
+            t_mt = _timed(lambda: lp.mean(-1), flush, reps)
+            row_rec("mean_vocab", M, t_m, (4 * VOCAB + 4) * M, t_mt, _rows_differing(ym[:, None], one_m[0][:n]),
+                    _rows_differing(lp.mean(-1)[:, None], one_m[1][:n]), n)
+            del x, y, lp
+            torch.cuda.empty_cache()
+    save()
 
 
 # ----------------------------------------------------------------------------- single-kernel cases
@@ -946,7 +1004,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="per-kernel M sweeps (table, not JSON line)")
     ap.add_argument("--sweep-shapes", default="", help="comma list of sweep groups (q/o,k/v,...,rows)")
-    ap.add_argument("--sweep-out", default="", help="write the sweep as JSON to this path")
+    ap.add_argument("--sweep-out", default="", help="write the sweep as JSON to this path (after every point)")
+    ap.add_argument("--resume", action="store_true", help="with --sweep-out: skip the points already there")
     ap.add_argument("--uniqueness", type=int, default=0,
                     help="run the batch-composition uniqueness experiment with this many trials")
     ap.add_argument("--context", type=int, default=4096,

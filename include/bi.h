@@ -115,7 +115,8 @@ bi_status bi_addmm(const void *input, int64_t ld_input, const void *A, int64_t l
  *   g and u are the fp32 accumulators of bi_matmul (same K order); h = (g / (1 + exp(-g))) * u
  *   in fp32, one rounding to bf16.  (bi_matmul followed by bi_silu_mul rounds g and u to bf16
  *   first, so the two paths agree to the bf16 tolerance, not bit for bit.)
- *   Alignment and limits as bi_matmul; 2F <= 2^31 - 1.  K = 0 writes zeros.
+ *   Alignment and limits as bi_matmul; 2F <= 2^31 - 1; with BI_B_KN, F must also be a multiple
+ *   of 8 (the up half starts at column F), else BI_ERR_ALIGNMENT.  K = 0 writes zeros.
  */
 bi_status bi_matmul_silu_mul(const void *A, int64_t lda, const void *B, int64_t ldb,
                              bi_b_layout b_layout, void *H, int64_t ldh, int64_t M, int64_t F,

@@ -187,6 +187,9 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
         if (!A || !B) return BI_ERR_INVALID_ARG;
         if (lda < K || ldb < (b_layout == BI_B_KN ? b_rows : K)) return BI_ERR_INVALID_ARG;
         if (!aligned16(A) || !aligned16(B) || lda % 8 != 0 || ldb % 8 != 0) return BI_ERR_ALIGNMENT;
+        // [K, 2F] gate/up weights: the up half starts at column F, the innermost coordinate of its
+        // tile loads, which a TMA copy needs at a multiple of 16 bytes (8 bf16 elements).
+        if (fuse_silu && b_layout == BI_B_KN && N % 8 != 0) return BI_ERR_ALIGNMENT;
     }
 
     DeviceState *dev = nullptr;

@@ -82,6 +82,8 @@ def test_host_validation_without_a_gpu(lib):
     assert lib.bi_log_softmax(fake, 9, fake, 2, 8, NULL) == I
     assert lib.bi_log_softmax(fake + 4, 1, fake, 2, 8, NULL) == A
     assert lib.bi_silu_mul(NULL, NULL, 2, 8, NULL) == I
+    # fused gate/up with [K, 2F] weights: the up half's first column F must be a multiple of 8
+    assert lib.bi_matmul_silu_mul(fake, 200, fake, 1000, 0, fake, 504, 77, 500, 200, NULL) == A
     # LM-head log_softmax halves: null or misaligned pairs, short row stride
     assert lib.bi_matmul_lse(fake, 8, fake, 8, 1, fake, 8, 0, NULL, 2, 8, 8, NULL) == I
     assert lib.bi_matmul_lse(fake, 8, fake, 8, 1, fake, 8, 0, fake + 4, 2, 8, 8, NULL) == A
