@@ -246,10 +246,12 @@ __global__ void __launch_bounds__(1024, 1) log_softmax_scalar_kernel(const void 
 // again.  Pass-1 copies ask L2 to keep their lines (they are read again in pass 2),
 // pass-2 copies and the y stores ask it to drop theirs.
 //
-// Element order (fixed by V alone): the row is cut into chunks of kLsmChunk bytes; a chunk
-// into groups of 4 elements; thread t owns groups t, t + T, t + 2T, ... of every chunk and
-// folds them in that order, chunk after chunk.  Consecutive threads read consecutive
-// shared-memory words and write consecutive 16-byte pieces of y.
+// Element order (fixed by V alone): the row is cut into chunks of kLsmChunk bytes; in pass 1
+// a chunk into groups of 8 elements, thread t owning groups t and t + T (bf16; group t for
+// fp32): per chunk a thread takes the maximum of its elements, rescales its running pair once
+// and adds their exp(x - max) in order, chunk after chunk.  Pass 2 writes 4-element groups,
+// thread t owning t, t + T, ...  Consecutive threads read consecutive 16-byte shared-memory
+// pieces and write consecutive 16-byte pieces of y.
 //
 // Copy schedule: copy j (j = 0, 1, ...) goes to stage j % S and completes phase j / S of
 // that stage's barrier.  Copies 0 .. n-1 are the n chunks of pass 1; copies n .. n+R-1
@@ -267,7 +269,6 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
 {
     constexpr int kElem = BF16 ? 2 : 4;
     constexpr int kPerChunk = kLsmChunk / kElem;      // elements per chunk
-    constexpr int kGroups = kPerChunk / 4;            // groups of 4 elements per chunk
     extern __shared__ __align__(128) uint8_t lsm_smem[];
     uint8_t(*ring)[kLsmChunk] = reinterpret_cast<uint8_t(*)[kLsmChunk]>(lsm_smem);
     __shared__ uint64_t full[kLsmStages];
@@ -309,16 +310,54 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
                                      abort_flag, status, wait_limit_ns);
         return __syncthreads_and(ok ? 1 : 0) != 0;
     };
-    // Fold or write the chunk held by copy j.
+    // Fold the chunk held by copy j: thread t takes the 8-element groups t, t + T, ... of the
+    // chunk (one 16-byte shared-memory read per group for bf16, two for fp32; elements past V
+    // count as -inf), reduces them to their maximum, rescales its running pair once, then adds
+    // exp(x - max) for its elements in order.
     MaxSum acc{kNegInf, 0.0f};
     float m = 0.0f, ls = 0.0f;
-    auto visit = [&](int j, bool write) {
-        const int c = j < n ? j : j - n;
-        const int64_t e0 = (int64_t)c * kPerChunk;
+    constexpr int kFoldPer = kPerChunk / kLsmThreads;  // elements per thread and chunk: 16 bf16, 8 fp32
+    // Elements of the row in the chunk of copy j (kPerChunk except in the row's last chunk).
+    auto chunk_valid = [&](int j) -> int {
+        const int64_t e0 = (int64_t)(j < n ? j : j - n) * kPerChunk;
+        return V - e0 < kPerChunk ? (int)(V - e0) : kPerChunk;
+    };
+    auto fold = [&](int j) {
+        const int valid = chunk_valid(j);
         const uint8_t *buf = ring[j % kLsmStages];
-        for (int g = tid; g < kGroups; g += kLsmThreads) {
-            const int64_t e = e0 + 4 * (int64_t)g;
-            if (e >= V) break;
+        float v[kFoldPer];
+#pragma unroll
+        for (int i = 0; i < kFoldPer / 8; ++i) {
+            const int g = tid + i * kLsmThreads;
+            float *w = v + 8 * i;
+            if (BF16) {
+                const uint4 u = 8 * g < valid ? *reinterpret_cast<const uint4 *>(buf + 16 * g) : make_uint4(0, 0, 0, 0);
+                w[0] = bf16lo(u.x); w[1] = bf16hi(u.x); w[2] = bf16lo(u.y); w[3] = bf16hi(u.y);
+                w[4] = bf16lo(u.z); w[5] = bf16hi(u.z); w[6] = bf16lo(u.w); w[7] = bf16hi(u.w);
+            } else {
+                const float4 a = 8 * g < valid ? *reinterpret_cast<const float4 *>(buf + 32 * g)
+                                               : make_float4(0, 0, 0, 0);
+                const float4 b = 8 * g + 4 < valid ? *reinterpret_cast<const float4 *>(buf + 32 * g + 16)
+                                                   : make_float4(0, 0, 0, 0);
+                w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+            }
+        }
+        if (valid < kPerChunk) {  // the row's last chunk: elements past V count as -inf
+#pragma unroll
+            for (int i = 0; i < kFoldPer / 8; ++i)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (8 * (tid + i * kLsmThreads) + k >= valid) v[8 * i + k] = kNegInf;
+        }
+        lsm_accumulate(acc, v);
+    };
+    // Write y for the chunk held by copy j: thread t takes the 4-element groups t, t + T, ...
+    // (one coalesced 16-byte store each).
+    auto write_y = [&](int j) {
+        const int valid = chunk_valid(j);
+        const uint8_t *buf = ring[j % kLsmStages];
+        float4 *yc = reinterpret_cast<float4 *>(yr + (int64_t)(j < n ? j : j - n) * kPerChunk);
+        for (int g = tid; 4 * g < valid; g += kLsmThreads) {
             float v[4];
             if (BF16) {
                 const uint2 u = *reinterpret_cast<const uint2 *>(buf + 8 * g);
@@ -327,12 +366,7 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
                 const float4 f = *reinterpret_cast<const float4 *>(buf + 16 * g);
                 v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
             }
-            if (!write) {
-                lsm_accumulate(acc, v);
-            } else {
-                __stcs(reinterpret_cast<float4 *>(yr + e),
-                       make_float4((v[0] - m) - ls, (v[1] - m) - ls, (v[2] - m) - ls, (v[3] - m) - ls));
-            }
+            __stcs(yc + g, make_float4((v[0] - m) - ls, (v[1] - m) - ls, (v[2] - m) - ls, (v[3] - m) - ls));
         }
     };
     // After the last use of copy j's stage, start copy j + S if it exists.
@@ -348,7 +382,7 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
     // Pass 1: copies 0 .. n-1.  Stages of the last S chunks are kept for pass 2.
     for (int j = 0; j < n && ok; ++j) {
         if (!(ok = landed(j))) break;
-        visit(j, false);
+        fold(j);
         if (j + kLsmStages < n) refill(j);
         else __syncthreads();
     }
@@ -358,12 +392,12 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
         ls = __logf(row.s);
         // Pass 2, resident chunks R .. n-1 (copies R .. n-1), then copies n .. n+R-1.
         for (int j = R; j < n; ++j) {
-            visit(j, true);
+            write_y(j);
             refill(j);
         }
         for (int j = n; j < copies && ok; ++j) {
             if (!(ok = landed(j))) break;
-            visit(j, true);
+            write_y(j);
             refill(j);
         }
     }
