@@ -246,10 +246,11 @@ __global__ void __launch_bounds__(1024, 1) log_softmax_scalar_kernel(const void 
 // again.  Pass-1 copies ask L2 to keep their lines (they are read again in pass 2),
 // pass-2 copies and the y stores ask it to drop theirs.
 //
-// Element order (fixed by V alone): the row is cut into chunks of kLsmChunk bytes; in pass 1
-// a chunk into groups of 8 elements, thread t owning groups t and t + T (bf16; group t for
-// fp32): per chunk a thread takes the maximum of its elements, rescales its running pair once
-// and adds their exp(x - max) in order, chunk after chunk.  Pass 2 writes 4-element groups,
+// Element order (fixed by V alone): the row is cut into chunks of kLsmChunk bytes and, in
+// pass 1, each chunk into sub-blocks of kLsmFoldBytes; a sub-block into groups of 8 elements,
+// thread t owning groups t and t + T (bf16; group t for fp32): per sub-block a thread takes the
+// maximum of its elements, rescales its running pair once and adds their exp(x - max) in
+// order, sub-block after sub-block.  Pass 2 writes 4-element groups,
 // thread t owning t, t + T, ...  Consecutive threads read consecutive 16-byte shared-memory
 // pieces and write consecutive 16-byte pieces of y.
 //
@@ -259,8 +260,9 @@ __global__ void __launch_bounds__(1024, 1) log_softmax_scalar_kernel(const void 
 // their stages when pass 1 ends and are used by pass 2 without a copy.  A copy is issued
 // once the previous occupant of its stage has been consumed for the last time.
 constexpr int kLsmThreads = 512;
-constexpr int kLsmChunk = 16384;
-constexpr int kLsmStages = 6;
+constexpr int kLsmChunk = 32768;      // bytes per bulk copy
+constexpr int kLsmStages = 3;
+constexpr int kLsmFoldBytes = 16384;  // pass 1 folds a chunk in sub-blocks of this many bytes
 
 template <bool BF16>
 __global__ void __launch_bounds__(kLsmThreads, 2)
@@ -316,40 +318,48 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
     // exp(x - max) for its elements in order.
     MaxSum acc{kNegInf, 0.0f};
     float m = 0.0f, ls = 0.0f;
-    constexpr int kFoldPer = kPerChunk / kLsmThreads;  // elements per thread and chunk: 16 bf16, 8 fp32
+    // Pass 1 folds a chunk in sub-blocks of kLsmFoldBytes, each as described above.
+    constexpr int kSubPer = kLsmFoldBytes / kElem;        // elements per sub-block
+    constexpr int kFoldPer = kSubPer / kLsmThreads;        // per thread and sub-block: 16 bf16, 8 fp32
     // Elements of the row in the chunk of copy j (kPerChunk except in the row's last chunk).
     auto chunk_valid = [&](int j) -> int {
         const int64_t e0 = (int64_t)(j < n ? j : j - n) * kPerChunk;
         return V - e0 < kPerChunk ? (int)(V - e0) : kPerChunk;
     };
     auto fold = [&](int j) {
-        const int valid = chunk_valid(j);
-        const uint8_t *buf = ring[j % kLsmStages];
-        float v[kFoldPer];
+        const int chunk_elems = chunk_valid(j);
+#pragma unroll 1
+        for (int sb = 0; sb < kLsmChunk / kLsmFoldBytes; ++sb) {
+            const int valid = chunk_elems - sb * kSubPer;  // elements of the row in this sub-block
+            if (valid <= 0) break;
+            const uint8_t *buf = ring[j % kLsmStages] + sb * kLsmFoldBytes;
+            float v[kFoldPer];
 #pragma unroll
-        for (int i = 0; i < kFoldPer / 8; ++i) {
-            const int g = tid + i * kLsmThreads;
-            float *w = v + 8 * i;
-            if (BF16) {
-                const uint4 u = 8 * g < valid ? *reinterpret_cast<const uint4 *>(buf + 16 * g) : make_uint4(0, 0, 0, 0);
-                w[0] = bf16lo(u.x); w[1] = bf16hi(u.x); w[2] = bf16lo(u.y); w[3] = bf16hi(u.y);
-                w[4] = bf16lo(u.z); w[5] = bf16hi(u.z); w[6] = bf16lo(u.w); w[7] = bf16hi(u.w);
-            } else {
-                const float4 a = 8 * g < valid ? *reinterpret_cast<const float4 *>(buf + 32 * g)
-                                               : make_float4(0, 0, 0, 0);
-                const float4 b = 8 * g + 4 < valid ? *reinterpret_cast<const float4 *>(buf + 32 * g + 16)
+            for (int i = 0; i < kFoldPer / 8; ++i) {
+                const int g = tid + i * kLsmThreads;
+                float *w = v + 8 * i;
+                if (BF16) {
+                    const uint4 u =
+                        8 * g < valid ? *reinterpret_cast<const uint4 *>(buf + 16 * g) : make_uint4(0, 0, 0, 0);
+                    w[0] = bf16lo(u.x); w[1] = bf16hi(u.x); w[2] = bf16lo(u.y); w[3] = bf16hi(u.y);
+                    w[4] = bf16lo(u.z); w[5] = bf16hi(u.z); w[6] = bf16lo(u.w); w[7] = bf16hi(u.w);
+                } else {
+                    const float4 a = 8 * g < valid ? *reinterpret_cast<const float4 *>(buf + 32 * g)
                                                    : make_float4(0, 0, 0, 0);
-                w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+                    const float4 b = 8 * g + 4 < valid ? *reinterpret_cast<const float4 *>(buf + 32 * g + 16)
+                                                       : make_float4(0, 0, 0, 0);
+                    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+                }
             }
-        }
-        if (valid < kPerChunk) {  // the row's last chunk: elements past V count as -inf
+            if (valid < kSubPer) {  // the row's last sub-block: elements past V count as -inf
 #pragma unroll
-            for (int i = 0; i < kFoldPer / 8; ++i)
+                for (int i = 0; i < kFoldPer / 8; ++i)
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    if (8 * (tid + i * kLsmThreads) + k >= valid) v[8 * i + k] = kNegInf;
+                    for (int k = 0; k < 8; ++k)
+                        if (8 * (tid + i * kLsmThreads) + k >= valid) v[8 * i + k] = kNegInf;
+            }
+            lsm_accumulate(acc, v);
         }
-        lsm_accumulate(acc, v);
     };
     // Write y for the chunk held by copy j: thread t takes the 4-element groups t, t + T, ...
     // (one coalesced 16-byte store each).
