@@ -139,6 +139,24 @@ bi_status encode_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_
 
 bi_status launched() { return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA; }
 
+// Launch `kernel` with programmatic stream serialization: it may start while the previous kernel
+// in the stream finishes, and waits (griddep_wait) for it before touching global memory.
+template <typename... KArgs, typename... Args>
+bi_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr{};
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
+
 // Launch `kernel` with one cluster of bi::kRowCluster CTAs per row, rows on grid.y in slices of
 // at most 65535; the kernel takes the slice's first row as its `row0` argument.
 template <typename... KArgs, typename... Args>
@@ -245,8 +263,9 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
 
     const int64_t pairs = dev->gemm_clusters;
     const int grid = 2 * (int)(tiles < pairs ? tiles : pairs);
-    bi::gemm_bf16_pair_kernel<<<grid, bi::kGemmThreads, bi::kPairSmem, s>>>(tm_a, tm_b, p);
-    return launched();
+    st = launch_pdl(bi::gemm_bf16_pair_kernel, dim3(grid), dim3(bi::kGemmThreads), (size_t)bi::kPairSmem, s, tm_a,
+                    tm_b, p);
+    return st != BI_OK ? st : launched();
 }
 
 __global__ void selftest_wait_kernel(int32_t *status, uint64_t limit_ns)
@@ -360,6 +379,7 @@ bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H
     if (H == 0 || !x || !w || !y) return BI_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int T = bi::rmsnorm_threads(H);
+    bi_status st = BI_OK;
     if (H % 8 == 0) {
         if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return BI_ERR_ALIGNMENT;
         const int64_t cpt = (H / 8 + T - 1) / T;
@@ -367,15 +387,16 @@ bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H
         const uint4 *wv = static_cast<const uint4 *>(w);
         uint4 *yv = static_cast<uint4 *>(y);
         switch (cpt) {
-        case 1: bi::rmsnorm_vec_kernel<1><<<(unsigned)M, T, 0, s>>>(xv, wv, yv, H, eps); break;
-        case 2: bi::rmsnorm_vec_kernel<2><<<(unsigned)M, T, 0, s>>>(xv, wv, yv, H, eps); break;
-        case 3: bi::rmsnorm_vec_kernel<3><<<(unsigned)M, T, 0, s>>>(xv, wv, yv, H, eps); break;
-        case 4: bi::rmsnorm_vec_kernel<4><<<(unsigned)M, T, 0, s>>>(xv, wv, yv, H, eps); break;
+        case 1: st = launch_pdl(bi::rmsnorm_vec_kernel<1>, dim3((unsigned)M), dim3(T), 0, s, xv, wv, yv, H, eps); break;
+        case 2: st = launch_pdl(bi::rmsnorm_vec_kernel<2>, dim3((unsigned)M), dim3(T), 0, s, xv, wv, yv, H, eps); break;
+        case 3: st = launch_pdl(bi::rmsnorm_vec_kernel<3>, dim3((unsigned)M), dim3(T), 0, s, xv, wv, yv, H, eps); break;
+        case 4: st = launch_pdl(bi::rmsnorm_vec_kernel<4>, dim3((unsigned)M), dim3(T), 0, s, xv, wv, yv, H, eps); break;
         default:
             bi::rmsnorm_scalar_kernel<<<(unsigned)M, T, 0, s>>>(
                 static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w),
                 static_cast<__nv_bfloat16 *>(y), H, eps);
         }
+        if (st != BI_OK) return st;
     } else {
         bi::rmsnorm_scalar_kernel<<<(unsigned)M, T, 0, s>>>(
             static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w),
@@ -392,12 +413,16 @@ bi_status bi_mean(const float *x, float *y, int64_t M, int64_t H, void *stream)
     if (H == 0 || !x || !y) return BI_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int T = bi::mean_threads(H);
+    bi_status st = BI_OK;
     if (H % 4 == 0) {
         if (!aligned16(x)) return BI_ERR_ALIGNMENT;
         if (H / 4 >= 8 * (int64_t)T)
-            bi::mean_vec_kernel<true><<<(unsigned)M, T, 0, s>>>(reinterpret_cast<const float4 *>(x), y, H);
+            st = launch_pdl(bi::mean_vec_kernel<true>, dim3((unsigned)M), dim3(T), 0, s,
+                            reinterpret_cast<const float4 *>(x), y, H);
         else
-            bi::mean_vec_kernel<false><<<(unsigned)M, T, 0, s>>>(reinterpret_cast<const float4 *>(x), y, H);
+            st = launch_pdl(bi::mean_vec_kernel<false>, dim3((unsigned)M), dim3(T), 0, s,
+                            reinterpret_cast<const float4 *>(x), y, H);
+        if (st != BI_OK) return st;
     } else {
         bi::mean_scalar_kernel<<<(unsigned)M, T, 0, s>>>(x, y, H);
     }
@@ -421,12 +446,11 @@ bi_status bi_log_softmax(const void *x, bi_dtype x_dtype, float *y, int64_t M, i
         bi_status st = device_state(&dev);
         if (st != BI_OK) return st;
         const uint8_t *xb = static_cast<const uint8_t *>(x);
-        if (bf16)
-            bi::log_softmax_stream_kernel<true><<<(unsigned)M, bi::kLsmThreads, bi::kLsmSmem, s>>>(
-                xb, y, V, dev->status, kWaitLimitNs);
-        else
-            bi::log_softmax_stream_kernel<false><<<(unsigned)M, bi::kLsmThreads, bi::kLsmSmem, s>>>(
-                xb, y, V, dev->status, kWaitLimitNs);
+        st = bf16 ? launch_pdl(bi::log_softmax_stream_kernel<true>, dim3((unsigned)M), dim3(bi::kLsmThreads),
+                               (size_t)bi::kLsmSmem, s, xb, y, V, dev->status, kWaitLimitNs)
+                  : launch_pdl(bi::log_softmax_stream_kernel<false>, dim3((unsigned)M), dim3(bi::kLsmThreads),
+                               (size_t)bi::kLsmSmem, s, xb, y, V, dev->status, kWaitLimitNs);
+        if (st != BI_OK) return st;
     } else {
         if (bf16)
             bi::log_softmax_scalar_kernel<true><<<(unsigned)M, T, 0, s>>>(x, y, V);

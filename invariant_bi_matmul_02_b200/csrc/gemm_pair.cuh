@@ -98,6 +98,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_holder;
+    // Everything above touched only this cluster's shared and tensor memory; global memory is
+    // read and written only after the previous kernel in the stream has completed.
+    griddep_wait();
+    griddep_launch_dependents();
 
     // Fused SiLU * up: a pair tile yields kHalfBN columns of h; CTA 0 stages gate rows
     // n0 .. n0+127 and CTA 1 the up rows F + n0 .. so each CTA's accumulator holds gate in

@@ -239,6 +239,14 @@ __device__ __forceinline__ float2 ld_dsmem_f32x2(uint32_t cluster_addr)
     return v;
 }
 
+// Programmatic dependent launch.  griddep_wait: block until the grids this one depends on
+// (the previous kernel in the stream, when this grid was launched with programmatic stream
+// serialization) have completed and their memory is visible; without such a launch it returns
+// at once.  griddep_launch_dependents: allow the next grid in the stream to start launching
+// (its threads still wait in their own griddep_wait for this grid to complete).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // All threads of every CTA of the cluster.
 __device__ __forceinline__ void cluster_sync_all()
 {

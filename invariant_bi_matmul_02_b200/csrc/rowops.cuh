@@ -94,6 +94,8 @@ __global__ void __launch_bounds__(1024) rmsnorm_vec_kernel(const uint4 *__restri
                                                           float eps)
 {
     __shared__ float red[32];
+    griddep_wait();  // the previous kernel's output (x) is complete
+    griddep_launch_dependents();
     const int64_t nch = H / 8;
     const int T = blockDim.x;
     const uint4 *xr = x + (int64_t)blockIdx.x * nch;
@@ -168,6 +170,8 @@ __global__ void __launch_bounds__(1024) mean_vec_kernel(const float4 *__restrict
                                                        float *__restrict__ y, int64_t H)
 {
     __shared__ float red[32];
+    griddep_wait();  // the previous kernel's output (x) is complete
+    griddep_launch_dependents();
     const int64_t nch = H / 4;
     const float4 *xr = x + (int64_t)blockIdx.x * nch;
     float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
@@ -291,6 +295,8 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
         abort_flag_s = 0;
         fence_mbar_init();
     }
+    griddep_wait();  // the previous kernel's output (x) is complete
+    griddep_launch_dependents();
     __syncthreads();
 
     int issued = 0;  // meaningful in thread 0 only
