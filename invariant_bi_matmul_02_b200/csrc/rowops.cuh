@@ -164,7 +164,8 @@ __global__ void __launch_bounds__(1024) rmsnorm_scalar_kernel(const __nv_bfloat1
 // keeps four running sums (one per float4 lane) and folds them as (s0+s1)+(s2+s3).
 // LONG: eight float4 loads in flight per thread (rows of >= 8 T groups, which run one 1024-thread
 // block per SM); otherwise four.  The adds keep the ascending group order in both, so the sums
-// are the same bits either way.
+// are the same bits either way.  x is read once, with an evict-first hint, so the reads do not
+// push out of L2 the lines of x (e.g. the last rows a log_softmax just wrote) not yet read.
 template <bool LONG>
 __global__ void __launch_bounds__(1024) mean_vec_kernel(const float4 *__restrict__ x,
                                                        float *__restrict__ y, int64_t H)
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(1024) mean_vec_kernel(const float4 *__restrict
         for (; c + 7 * (int64_t)T < nch; c += 8 * (int64_t)T) {
             float4 g[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) g[k] = __ldg(xr + c + k * (int64_t)T);
+            for (int k = 0; k < 8; ++k) g[k] = __ldcs(xr + c + k * (int64_t)T);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 s0 += g[k].x; s1 += g[k].y; s2 += g[k].z; s3 += g[k].w;
@@ -189,15 +190,15 @@ __global__ void __launch_bounds__(1024) mean_vec_kernel(const float4 *__restrict
         }
     }
     for (; c + 3 * (int64_t)T < nch; c += 4 * (int64_t)T) {
-        float4 a = __ldg(xr + c), b = __ldg(xr + c + T), d = __ldg(xr + c + 2 * T),
-               e = __ldg(xr + c + 3 * T);
+        float4 a = __ldcs(xr + c), b = __ldcs(xr + c + T), d = __ldcs(xr + c + 2 * T),
+               e = __ldcs(xr + c + 3 * T);
         s0 += a.x; s1 += a.y; s2 += a.z; s3 += a.w;
         s0 += b.x; s1 += b.y; s2 += b.z; s3 += b.w;
         s0 += d.x; s1 += d.y; s2 += d.z; s3 += d.w;
         s0 += e.x; s1 += e.y; s2 += e.z; s3 += e.w;
     }
     for (; c < nch; c += T) {
-        float4 a = __ldg(xr + c);
+        float4 a = __ldcs(xr + c);
         s0 += a.x; s1 += a.y; s2 += a.z; s3 += a.w;
     }
     float s = __fadd_rn(__fadd_rn(s0, s1), __fadd_rn(s2, s3));
@@ -248,7 +249,8 @@ __global__ void __launch_bounds__(1024, 1) log_softmax_scalar_kernel(const void 
 // builds the row's (max, sum of exp); pass 2 writes y = (x - max) - log(sum), starting
 // with the last chunks of the row, which are still in the ring, and streaming the rest
 // again.  Pass-1 copies ask L2 to keep their lines (they are read again in pass 2),
-// pass-2 copies and the y stores ask it to drop theirs.
+// pass-2 copies ask it to drop theirs.  y is stored with the default policy, so the last rows
+// written are still in L2 for a kernel that reads y next (the mean over log-probs in a step).
 //
 // Element order (fixed by V alone): the row is cut into chunks of kLsmChunk bytes and, in
 // pass 1, each chunk into sub-blocks of kLsmFoldBytes; a sub-block into groups of 8 elements,
@@ -382,7 +384,7 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
                 const float4 f = *reinterpret_cast<const float4 *>(buf + 16 * g);
                 v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
             }
-            __stcs(yc + g, make_float4((v[0] - m) - ls, (v[1] - m) - ls, (v[2] - m) - ls, (v[3] - m) - ls));
+            yc[g] = make_float4((v[0] - m) - ls, (v[1] - m) - ls, (v[2] - m) - ls, (v[3] - m) - ls);
         }
     };
     // After the last use of copy j's stage, start copy j + S if it exists.
