@@ -1,0 +1,72 @@
+"""Host-side logic of bench.py (no GPU): FLOP and byte accounting, the traffic record's
+validity check, the CLI's warm-up rule and the parsing of sampled clocks."""
+import json
+
+import pytest
+
+import bench
+
+
+def test_gemm_flops_per_row_counts_every_projection():
+    H, KV, F, V = 4096, 1024, 12288, 151936
+    expect = 2 * (H * H + H * KV + H * KV + H * H + H * 2 * F + F * H + H * V)
+    assert bench.gemm_flops_per_row() == expect
+    assert abs(expect / 1e9 - 1.6305) < 1e-4
+
+
+def test_row_op_bytes_are_algorithmic():
+    b = bench.row_op_bytes_per_row()
+    assert b["log_softmax"] == 6 * 151936  # bf16 read once, fp32 written once
+    assert b["mean"] == 4 * 151936 + 4
+    assert b["rms1"] == 4 * 4096
+
+
+def test_traffic_record_is_used_only_for_its_source_case_and_rows(tmp_path, monkeypatch):
+    rec = {"gemm_source_sha": bench.gemm_source_sha(), "rows": 1024, "kernel_case": "gemm_lm_head",
+           "dram_bytes_per_launch": 123456789}
+    path = tmp_path / "traffic.json"
+    path.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(path))
+    assert bench.measured_traffic(1024, "gemm_lm_head") == 123456789
+    assert bench.measured_traffic(2048, "gemm_lm_head") is None
+    assert bench.measured_traffic(1024, "gemm_lm_head_lse") is None
+    rec["gemm_source_sha"] = "0" * 16  # captured on another kernel source
+    path.write_text(json.dumps(rec))
+    assert bench.measured_traffic(1024, "gemm_lm_head") is None
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
+    assert bench.measured_traffic(1024, "gemm_lm_head") is None
+
+
+def test_committed_traffic_record_matches_the_current_source():
+    assert bench.measured_traffic(1024, "gemm_lm_head") is not None
+
+
+def test_cli_refuses_fewer_than_three_warmup_steps(monkeypatch):
+    monkeypatch.setattr("sys.argv", ["bench.py", "--warmup", "2"])
+    with pytest.raises(SystemExit):
+        bench.main()
+
+
+class _FakeSmi:
+    def __init__(self, text):
+        self.text = text
+
+    def terminate(self):
+        pass
+
+    def communicate(self, timeout=None):
+        return self.text, ""
+
+
+def test_clock_sampler_reports_median_and_active_reasons():
+    lines = ["0, 1800, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active",
+             "0, 1700, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+             "0, 1900, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+             "garbled line"]
+    s = bench.ClockSampler(0)
+    s.proc = _FakeSmi("\n".join(lines))
+    out = s.stop()
+    assert out["sm_mhz"] == 1800 and out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["sw_power_cap"] and out["samples"] == 3
+    s.proc = _FakeSmi("0, 900, 1965, 500.0, 0x8, Active, Not Active, Not Active, Not Active")
+    assert s.stop()["reasons"] == ["hw_slowdown"]
