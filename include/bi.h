@@ -32,7 +32,11 @@
  *     buffer.  The library allocates no device memory in any call.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
  *     asynchronous on that stream.  Argument errors are returned before anything
- *     is launched; a launch failure returns BI_ERR_CUDA.
+ *     is launched; a launch failure returns BI_ERR_CUDA.  The GEMM, RMSNorm, mean and
+ *     one-block log_softmax kernels are launched with programmatic stream serialization:
+ *     they may start their on-chip set-up while the previous kernel on the stream drains,
+ *     and read or write global memory only after that kernel has completed, so stream
+ *     order holds as for any launch.
  *   - M = 0 (no rows) is a no-op that returns BI_OK.
  *   - Outputs must not overlap inputs.
  *   - bf16 is IEEE-style bfloat16 (1-8-7); every bf16 output is rounded once,
