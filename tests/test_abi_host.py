@@ -118,3 +118,25 @@ def test_missing_library_fails_loudly(tmp_path):
             binding.load(str(tmp_path / "libbi.so"))
     finally:
         binding._lib = saved
+
+
+def test_product_path_and_oracle_share_nothing():
+    """The CUDA path (package, kernels, header) never names the oracle, and the oracle never
+    names the package or its kernels: the two meet only in the tests, the smoke check and the
+    benchmark's CPU baseline."""
+    import glob
+    import os
+    import re
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    product = (glob.glob(os.path.join(root, "invariant_bi_matmul_02_b200", "*.py"))
+               + glob.glob(os.path.join(root, "invariant_bi_matmul_02_b200", "csrc", "*"))
+               + glob.glob(os.path.join(root, "include", "*.h")))
+    for path in product:
+        if os.path.isdir(path) or path.endswith((".so", ".pyc")):
+            continue
+        text = open(path, errors="replace").read()
+        code = "\n".join(l for l in text.splitlines() if "import" in l or "#include" in l)
+        assert not re.search(r"\boracle\b", code), f"{path} imports the oracle"
+    for path in glob.glob(os.path.join(root, "oracle", "*.[pc]*")):
+        text = open(path, errors="replace").read()
+        assert "invariant_bi_matmul_02_b200" not in text and "csrc" not in text, f"{path} uses the CUDA path"
