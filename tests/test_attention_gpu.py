@@ -24,7 +24,7 @@ def make(seed, B, Hq, Hkv, Lmax):
     return q, k, v
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 8), (16, 2), (8, 1)])
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 8), (16, 8), (16, 2), (8, 1)])  # group sizes 4, 1, 2, 8, 8
 @pytest.mark.parametrize("lens", [[1, 128, 300], [127, 129, 256, 257], [5]])
 def test_attention_parity(Hq, Hkv, lens):
     B, Lmax = len(lens), max(lens) + 3
