@@ -729,6 +729,32 @@ def run_sweep(args):
                     _rows_differing(lp.mean(-1)[:, None], one_m[1][:n]), n)
             del x, y, lp
             torch.cuda.empty_cache()
+    if args.sweep_shapes and "attention" in args.sweep_shapes.split(","):
+        # decode attention, Qwen3-8B heads: bi_decode_attention against torch's SDPA (GQA), L2
+        # flushed before every call; caches [B, L, 8, 128] (SDPA gets them as [B, 8, L, 128])
+        Hq, Hkv, D = 32, 8, 128
+        out.setdefault("attention", [])
+        print(f"{'B':>4s} {'L':>6s} {'bi us':>9s} {'GB/s':>7s} {'%HBM':>6s} {'sdpa us':>9s}")
+        for B, L in [(1, 1024), (8, 1024), (32, 2048), (64, 4096), (128, 2048)]:
+            g = torch.Generator(device=dev)
+            g.manual_seed(58)
+            q = torch.randn(B, Hq, D, generator=g, device=dev).to(torch.bfloat16)
+            k = torch.randn(B, L, Hkv, D, generator=g, device=dev).to(torch.bfloat16)
+            v = torch.randn(B, L, Hkv, D, generator=g, device=dev).to(torch.bfloat16)
+            sl = torch.full((B,), L, dtype=torch.int32, device=dev)
+            scr = torch.empty(bi.bi_decode_attention_scratch_bytes(B, Hq, D, L), dtype=torch.uint8, device=dev)
+            o = torch.empty_like(q)
+            t_bi = _timed(lambda: bi.bi_decode_attention(q, k, v, sl, scratch=scr, out=o), flush, reps)
+            qt, kt, vt = q.view(B, Hq, 1, D), k.permute(0, 2, 1, 3).contiguous(), v.permute(0, 2, 1, 3).contiguous()
+            t_t = _timed(lambda: F.scaled_dot_product_attention(qt, kt, vt, enable_gqa=True), flush, reps)
+            by = 2 * B * L * Hkv * D * 2
+            out["attention"].append({"B": B, "L": L, "bi_us": t_bi * 1e3, "bi_gbs": by / t_bi / 1e6,
+                                     "bi_frac_hbm": by / t_bi / 1e6 / peaks["hbm_gbs"], "sdpa_us": t_t * 1e3})
+            save()
+            print(f"{B:4d} {L:6d} {t_bi*1e3:9.1f} {by/t_bi/1e6:7.0f} {100*by/t_bi/1e6/peaks['hbm_gbs']:5.1f}% "
+                  f"{t_t*1e3:9.1f}", flush=True)
+            del q, k, v, kt, vt, scr, o
+            torch.cuda.empty_cache()
     save()
 
 
@@ -1020,7 +1046,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=25.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="per-kernel M sweeps (table, not JSON line)")
-    ap.add_argument("--sweep-shapes", default="", help="comma list of sweep groups (q/o,k/v,...,rows)")
+    ap.add_argument("--sweep-shapes", default="",
+                    help="comma list of sweep groups (q/o,k/v,gate/up,down,lm_head,rows; attention only when named)")
     ap.add_argument("--sweep-out", default="", help="write the sweep as JSON to this path (after every point)")
     ap.add_argument("--resume", action="store_true", help="with --sweep-out: skip the points already there")
     ap.add_argument("--uniqueness", type=int, default=0,

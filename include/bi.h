@@ -32,8 +32,9 @@
  *     buffer.  The library allocates no device memory in any call.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
  *     asynchronous on that stream.  Argument errors are returned before anything
- *     is launched; a launch failure returns BI_ERR_CUDA.  The GEMM, RMSNorm, mean and
- *     one-block log_softmax kernels are launched with programmatic stream serialization:
+ *     is launched; a launch failure returns BI_ERR_CUDA.  The GEMM, RMSNorm, mean,
+ *     one-block log_softmax and decode-attention kernels are launched with programmatic
+ *     stream serialization:
  *     they may start their on-chip set-up while the previous kernel on the stream drains,
  *     and read or write global memory only after that kernel has completed, so stream
  *     order holds as for any launch.

@@ -65,6 +65,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3)
 {
     extern __shared__ __align__(16) uint8_t attn_raw[];
     AttnSmem &sm = *reinterpret_cast<AttnSmem *>(attn_raw);
+    griddep_wait();  // the previous kernel's output (q, the caches, the lengths) is complete
+    griddep_launch_dependents();
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
@@ -243,6 +245,8 @@ __global__ void __launch_bounds__(kAttnD)
                                     const int32_t *__restrict__ lens, __nv_bfloat16 *__restrict__ out,
                                     int Hq, int64_t Lmax)
 {
+    griddep_wait();  // every split's partials are complete
+    griddep_launch_dependents();
     const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
     const int64_t S = attn_splits(Lmax);
     int64_t L = lens[b];

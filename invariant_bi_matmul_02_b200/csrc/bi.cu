@@ -619,19 +619,23 @@ bi_status bi_decode_attention(const void *q, const void *k_cache, const void *v_
     const auto *kb = static_cast<const __nv_bfloat16 *>(k_cache);
     const auto *vb = static_cast<const __nv_bfloat16 *>(v_cache);
     const dim3 grid((unsigned)S, (unsigned)Hkv, (unsigned)B);
+    const size_t smem = sizeof(bi::AttnSmem);
     switch (Hq / Hkv) {  // the group size is a property of the model, not of the batch
-    case 1: bi::decode_attention_split_kernel<1><<<grid, bi::kAttnThreads, sizeof(bi::AttnSmem), s>>>(
-                qb, kb, vb, seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
-    case 2: bi::decode_attention_split_kernel<2><<<grid, bi::kAttnThreads, sizeof(bi::AttnSmem), s>>>(
-                qb, kb, vb, seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
-    case 4: bi::decode_attention_split_kernel<4><<<grid, bi::kAttnThreads, sizeof(bi::AttnSmem), s>>>(
-                qb, kb, vb, seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
-    case 8: bi::decode_attention_split_kernel<8><<<grid, bi::kAttnThreads, sizeof(bi::AttnSmem), s>>>(
-                qb, kb, vb, seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
+    case 1: st = launch_pdl(bi::decode_attention_split_kernel<1>, grid, dim3(bi::kAttnThreads), smem, s, qb, kb, vb,
+                            seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
+    case 2: st = launch_pdl(bi::decode_attention_split_kernel<2>, grid, dim3(bi::kAttnThreads), smem, s, qb, kb, vb,
+                            seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
+    case 4: st = launch_pdl(bi::decode_attention_split_kernel<4>, grid, dim3(bi::kAttnThreads), smem, s, qb, kb, vb,
+                            seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
+    case 8: st = launch_pdl(bi::decode_attention_split_kernel<8>, grid, dim3(bi::kAttnThreads), smem, s, qb, kb, vb,
+                            seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
     default: return BI_ERR_UNSUPPORTED;
     }
-    bi::decode_attention_combine_kernel<<<dim3((unsigned)Hq, (unsigned)B), bi::kAttnD, 0, s>>>(
-        part_ms, part_acc, seq_lens, static_cast<__nv_bfloat16 *>(out), (int)Hq, Lmax);
+    if (st != BI_OK) return st;
+    st = launch_pdl(bi::decode_attention_combine_kernel, dim3((unsigned)Hq, (unsigned)B), dim3(bi::kAttnD), 0, s,
+                    static_cast<const float2 *>(part_ms), static_cast<const float *>(part_acc), seq_lens,
+                    static_cast<__nv_bfloat16 *>(out), (int)Hq, Lmax);
+    if (st != BI_OK) return st;
     return launched();
 }
 
