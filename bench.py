@@ -14,11 +14,6 @@ One *step* is one pass of every kernel of the path over a batch of M token rows
     hf   = bi_rmsnorm(y, g_final)
     lg   = bi_matmul(hf, W_lm)                        [M, 151936]  bf16 logits
     lp   = bi_log_softmax(lg)                         [M, 151936]  fp32, one block per row
-                                                                   (--lsm partials: bi_matmul_lse also
-                                                                   leaves one (max, sum exp) pair per
-                                                                   row and 256-column tile, and
-                                                                   bi_log_softmax_partials makes one
-                                                                   pass over lg)
     ce   = bi_mean(lp)                                [M]          mean log-prob (= -H(uniform, p))
 
 (attention itself is not one of the batch-invariant reduction kernels; q stands
@@ -138,12 +133,11 @@ def make_weights() -> dict:
 class Workload:
     """Weights (shared by all ranks) and this rank's rows, resident on the device."""
 
-    def __init__(self, rows: int, row0: int, device, fused_mlp: bool = True, lsm: str = "rows"):
+    def __init__(self, rows: int, row0: int, device, fused_mlp: bool = True):
         import torch
         from invariant_bi_matmul_02_b200 import inputs
         self.M = rows
         self.fused = fused_mlp
-        self.lsm = lsm
         self.ops = OPS_FUSED if fused_mlp else OPS_UNFUSED
         self.host = make_weights()
         self.x_host = inputs.rows_normal(10, row0, rows, HIDDEN)
@@ -159,8 +153,7 @@ class Workload:
             "h1": e(M, HIDDEN), "qkv": e(M, QKV), "o": e(M, HIDDEN),
             "h2": e(M, HIDDEN), "gu": e(M, 2 * FFN), "a": e(M, FFN), "y": e(M, HIDDEN),
             "hf": e(M, HIDDEN), "lg": e(M, VOCAB), "lp": e(M, VOCAB, dt=torch.float32),
-            "ce": e(M, dt=torch.float32), "lsp": e(M, -(-VOCAB // 256), 2, dt=torch.float32),
-            "lss": e(M, 2, dt=torch.float32),
+            "ce": e(M, dt=torch.float32),
         }
 
 
@@ -201,14 +194,8 @@ def run_step(wl: Workload, x, marks=None, only=None):
         begin("silu_mul"); bi.bi_silu_mul(B["gu"], out=B["a"]); end("silu_mul")
     begin("down"); bi.bi_addmm(B["o"], B["a"], W["W_down"], "nk", out=B["y"]); end("down")
     begin("rms3"); bi.bi_rmsnorm(B["y"], W["g_final"], EPS, out=B["hf"]); end("rms3")
-    if wl.lsm == "partials":
-        begin("lm_head"); bi.bi_matmul_lse(B["hf"], W["W_lm"], "nk", out=B["lg"], partials=B["lsp"]); end("lm_head")
-        begin("log_softmax")
-        bi.bi_log_softmax_partials(B["lg"], B["lsp"], out=B["lp"], row_stats=B["lss"])
-        end("log_softmax")
-    else:
-        begin("lm_head"); bi.bi_matmul(B["hf"], W["W_lm"], "nk", out=B["lg"]); end("lm_head")
-        begin("log_softmax"); bi.bi_log_softmax(B["lg"], out=B["lp"]); end("log_softmax")
+    begin("lm_head"); bi.bi_matmul(B["hf"], W["W_lm"], "nk", out=B["lg"]); end("lm_head")
+    begin("log_softmax"); bi.bi_log_softmax(B["lg"], out=B["lp"]); end("log_softmax")
     begin("mean"); bi.bi_mean(B["lp"], out=B["ce"]); end("mean")
     return B["ce"]
 
@@ -340,7 +327,7 @@ def run_bi(args):
 
     from invariant_bi_matmul_02_b200.shard import weak_rows
     M = args.rows
-    wl = Workload(M, weak_rows(M, rank)[0], device, fused_mlp=args.mlp == "fused", lsm=args.lsm)
+    wl = Workload(M, weak_rows(M, rank)[0], device, fused_mlp=args.mlp == "fused")
     OPS = wl.ops
     stream = torch.cuda.current_stream()
 
@@ -480,16 +467,13 @@ def run_bi(args):
                        "accumulate": "fp32", "parallelism": f"replicas x{world} (rows sharded)",
                        "mlp": "gate/up GEMM with SiLU*up in its epilogue" if wl.fused
                               else "gate/up GEMM, then bi_silu_mul",
-                       "log_softmax": "per-tile (max, sum exp) in the LM-head GEMM epilogue, then one pass"
-                                      if wl.lsm == "partials" else "bi_log_softmax after the LM head",
+                       "log_softmax": "bi_log_softmax after the LM head",
                        "l2": "working set ~3 GB > 126 MB L2; no flush",
                        "gemm_tile": bi.bi_gemm_config()},
-            "roofline": {"kernel": ("bi_matmul_lse" if wl.lsm == "partials" else "bi_matmul")
-                                   + " LM head launch [%d x 4096] x [4096 x 151936]" % M,
+            "roofline": {"kernel": "bi_matmul LM head launch [%d x 4096] x [4096 x 151936]" % M,
                          "bound": "tensor", "achieved": round(achieved, 1), "peak": peak_tf,
                          "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
-                         "traffic": measured_traffic(M, "gemm_lm_head_lse" if wl.lsm == "partials"
-                                                     else "gemm_lm_head"),
+                         "traffic": measured_traffic(M, "gemm_lm_head"),
                          "algorithmic_bytes": gemm_bytes(M, HIDDEN, VOCAB),
                          "peak_source": f"{peak_src} {'bf16_tflops_sustained' if long_run else 'bf16_tflops'}"},
             "gemm_all_launches_tflops": round(flops_step / (gemm_ms / 1e3) / 1e12, 1),
@@ -501,7 +485,7 @@ def run_bi(args):
             "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(wl.x.numel() * 2), "d2h_bytes_per_step": int(M * 4),
                     "steps": e2e_steps},
-            "gpu_launches": (len(OPS) + (1 if wl.lsm == "partials" else 0)) * args.steps,
+            "gpu_launches": len(OPS) * args.steps,
             "clocks": clocks,
             "device_status": status,
         }
@@ -693,7 +677,7 @@ def run_sweep(args):
         one_m = (torch.cat([bi.bi_mean(lp64[i:i + 1]) for i in range(64)])[:, None],
                  torch.cat([lp64[i:i + 1].mean(-1) for i in range(64)])[:, None])
         for M in [1, 8, 64, 256, 1024]:
-            ops_v = ("log_softmax", "log_softmax_cluster", "log_softmax_split", "log_softmax_partials", "mean_vocab")
+            ops_v = ("log_softmax", "log_softmax_cluster", "log_softmax_split", "mean_vocab")
             if all(("rows", op, M) in have for op in ops_v):
                 continue
             x = inputs.rows_normal(44, 0, M, VOCAB, std=1.3).to(dev)
@@ -712,16 +696,6 @@ def run_sweep(args):
             t_sp = _timed(lambda: bi.bi_log_softmax_split(x, scr, out=y), flush, reps)
             row_rec("log_softmax_split", M, t_sp, by, t_t, _rows_differing(y, one_v["log_softmax_split"][:n]),
                     t_diff, n)
-            # second half of the LM-head path: the pairs come from a GEMM epilogue, so its x is that
-            # GEMM's logits (same pass, same bytes); its invariance is tested in tests/test_lse_gpu.py
-            aw = inputs.rows_normal(45, 0, M, HIDDEN).to(dev)
-            ww = inputs.weight_normal(46, (VOCAB, HIDDEN)).to(dev)
-            xl, part = bi.bi_matmul_lse(aw, ww, "nk")
-            del ww
-            rs = torch.empty(M, 2, dtype=torch.float32, device=dev)
-            t_pa = _timed(lambda: bi.bi_log_softmax_partials(xl, part, out=y, row_stats=rs), flush, reps)
-            row_rec("log_softmax_partials", M, t_pa, by, t_t, 0, t_diff, 0)
-            del xl, part
             ym = torch.empty(M, dtype=torch.float32, device=dev)
             t_m = _timed(lambda: bi.bi_mean(lp, out=ym), flush, reps)
             t_mt = _timed(lambda: lp.mean(-1), flush, reps)
@@ -764,7 +738,6 @@ KERNEL_CASES = {
     # name: (description, bytes in + out) -- inputs larger than L2, a few hundred MB on the device
     "gemm_gate_up": "bi_matmul M=1024 K=4096 N=24576 (B [N, K])",
     "gemm_lm_head": "bi_matmul M=1024 K=4096 N=151936 (B [N, K])",
-    "gemm_lm_head_lse": "bi_matmul_lse M=1024 K=4096 N=151936 (B [N, K]), per-tile (max, sum exp) pairs",
     "gemm_qo_m256": "bi_matmul M=256 K=4096 N=4096 (B [N, K])",
     "gemm_gate_up_silu": "bi_matmul_silu_mul M=1024 K=4096 F=12288 (B [2F, K])",
     "rmsnorm": "bi_rmsnorm M=16384 H=4096 bf16",
@@ -772,7 +745,6 @@ KERNEL_CASES = {
     "mean_vocab": "bi_mean M=1024 H=151936 fp32 (the step's mean over log-probs)",
     "log_softmax": "bi_log_softmax M=1024 V=151936 bf16 -> fp32",
     "log_softmax_cluster": "bi_log_softmax_cluster M=1024 V=151936 bf16 -> fp32 (4 CTAs per row)",
-    "log_softmax_partials": "bi_log_softmax_partials M=1024 V=151936 bf16 -> fp32 (pairs precomputed)",
     "silu_mul": "bi_silu_mul M=1024 F=12288",
     "decode_attention": "bi_decode_attention B=64 L=4096, 32 q / 8 kv heads of 128",
 }
@@ -794,15 +766,11 @@ def run_kernel_case(args):
         work, unit = 2 * 1024 * 2 * FFN * HIDDEN, "TFLOP/s"
     elif name.startswith("gemm"):
         M, K, N = {"gemm_gate_up": (1024, HIDDEN, 2 * FFN), "gemm_lm_head": (1024, HIDDEN, VOCAB),
-                   "gemm_lm_head_lse": (1024, HIDDEN, VOCAB), "gemm_qo_m256": (256, HIDDEN, HIDDEN)}[name]
+                   "gemm_qo_m256": (256, HIDDEN, HIDDEN)}[name]
         a = inputs.rows_normal(50, 0, M, K).to(dev)
         w = inputs.weight_normal(51, (N, K)).to(dev)
         c = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        if name == "gemm_lm_head_lse":
-            part = torch.empty(M, bi.bi_lse_partials_per_row(N), 2, dtype=torch.float32, device=dev)
-            fn = lambda: bi.bi_matmul_lse(a, w, "nk", out=c, partials=part)
-        else:
-            fn = lambda: bi.bi_matmul(a, w, "nk", out=c)
+        fn = lambda: bi.bi_matmul(a, w, "nk", out=c)
         work, unit = 2 * M * N * K, "TFLOP/s"
     elif name in ("rmsnorm", "mean"):
         x = inputs.rows_normal_outliers(52, 0, 16384, HIDDEN, torch.bfloat16).to(dev)
@@ -831,15 +799,6 @@ def run_kernel_case(args):
         x = inputs.rows_normal(54, 0, 1024, VOCAB, std=1.3).to(dev)
         y = torch.empty(1024, VOCAB, dtype=torch.float32, device=dev)
         fn = lambda: bi.bi_log_softmax_cluster(x, out=y)
-        work, unit = 6 * VOCAB * 1024, "GB/s"
-    elif name == "log_softmax_partials":
-        a = inputs.rows_normal(50, 0, 1024, HIDDEN).to(dev)
-        w = inputs.weight_normal(51, (VOCAB, HIDDEN)).to(dev)
-        x, part = bi.bi_matmul_lse(a, w, "nk")
-        del w
-        y = torch.empty(1024, VOCAB, dtype=torch.float32, device=dev)
-        rs = torch.empty(1024, 2, dtype=torch.float32, device=dev)
-        fn = lambda: bi.bi_log_softmax_partials(x, part, out=y, row_stats=rs)
         work, unit = 6 * VOCAB * 1024, "GB/s"
     elif name == "silu_mul":
         gu = inputs.rows_normal(55, 0, 1024, 2 * FFN, std=2.0).to(dev)
@@ -1038,9 +997,6 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--rows", type=int, default=1024, help="token rows per GPU per step")
     ap.add_argument("--impl", choices=["bi", "reference"], default="bi")
-    ap.add_argument("--lsm", choices=["rows", "partials"], default="rows",
-                    help="LM-head log_softmax: bi_log_softmax after a plain GEMM (default), or pairs from "
-                         "the GEMM epilogue and one pass (bi_matmul_lse + bi_log_softmax_partials)")
     ap.add_argument("--mlp", choices=["fused", "unfused"], default="fused",
                     help="gate/up + SiLU*up as one fused GEMM (default) or GEMM then bi_silu_mul")
     ap.add_argument("--cpu-budget", type=float, default=25.0)

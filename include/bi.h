@@ -30,9 +30,13 @@
  *   - Tensors are row-major.  Pointers marked "device" point to global memory
  *     of the current CUDA device; the caller allocates, owns and frees every
  *     buffer.  The library allocates no device memory in any call.
- *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *   - `stream` is a cudaStream_t passed as `void *` (so that this header needs no CUDA
+ *     header; NULL = the legacy default stream).  Calls are
  *     asynchronous on that stream.  Argument errors are returned before anything
- *     is launched; a launch failure returns BI_ERR_CUDA.  The GEMM, RMSNorm, mean,
+ *     is launched; a launch failure returns BI_ERR_CUDA.  The status is the result of this
+ *     call's own launches: an error left by another library's earlier launch on the thread
+ *     is neither reported nor cleared (apart from a context-wide fault, which fails every
+ *     launch).  The GEMM, RMSNorm, mean,
  *     one-block log_softmax and decode-attention kernels are launched with programmatic
  *     stream serialization:
  *     they may start their on-chip set-up while the previous kernel on the stream drains,
@@ -42,6 +46,11 @@
  *   - Outputs must not overlap inputs.
  *   - bf16 is IEEE-style bfloat16 (1-8-7); every bf16 output is rounded once,
  *     to nearest-even, from an fp32 value.
+ *   - The library keeps per-device state for the life of the process (the SM count, the
+ *     status word's address, kernel attributes, the no-allocation array's address) and a
+ *     cache of encoded TMA tensor maps keyed by (base address, extents, row stride, box).
+ *     Calls across a cudaDeviceReset of a device the library has already used are not
+ *     supported: the cached device addresses belong to the context that reset destroyed.
  *   - Every device-side wait is bounded; a wait that runs out records
  *     BI_ERR_TIMEOUT in a per-device status word, the kernel releases what it
  *     holds and returns.  Read it with bi_get_device_status.
@@ -126,51 +135,6 @@ bi_status bi_addmm(const void *input, int64_t ld_input, const void *A, int64_t l
 bi_status bi_matmul_silu_mul(const void *A, int64_t lda, const void *B, int64_t ldb,
                              bi_b_layout b_layout, void *H, int64_t ldh, int64_t M, int64_t F,
                              int64_t K, void *stream);
-
-/*
- * bi_matmul_lse -- bi_matmul that also reduces each row of every output tile to a
- * (max, sum of exp) pair: the first half of a log_softmax over the LM-head logits, done in the
- * GEMM epilogue while the tile is still on chip.  Passage: as bi_matmul for C, as
- * bi_log_softmax for the pairs (ross.abutalabs.com "thinking-machines-lab/batch_invariant_ops",
- * "When to avoid": mm and log_softmax are both covered); fusing the two is this library's
- * design, not the pages'.
- *
- *   A, B, b_layout, C, ldc, c_dtype, M, N, K as bi_matmul (same tile configuration, same bits
- *   in C).
- *   partials  device, fp32, [M, P, 2] contiguous, P = bi_lse_partials_per_row(N), 8-byte
- *             aligned; owned by the caller, overwritten.  partials[i, t] = (m, s) with m the
- *             max of row i of C over columns [256 t, 256 t + 256) (those < N) and s the sum of
- *             exp(c - m) over them, folded in ascending column order, 32 columns at a time.  The
- *             values folded are those stored in C (bf16-rounded when c_dtype is BI_BF16).
- *   A null `partials` with M, N > 0 returns BI_ERR_INVALID_ARG.
- */
-bi_status bi_matmul_lse(const void *A, int64_t lda, const void *B, int64_t ldb, bi_b_layout b_layout,
-                        void *C, int64_t ldc, bi_dtype c_dtype, float *partials, int64_t M, int64_t N,
-                        int64_t K, void *stream);
-
-/* Pairs per row that bi_matmul_lse writes for N output columns: ceil(N / 256) (0 if N <= 0). */
-int64_t bi_lse_partials_per_row(int64_t N);
-
-/*
- * bi_log_softmax_partials -- the second half: y = (x - m) - log(s) per row, where (m, s) is
- * row i's pairs from bi_matmul_lse merged in one fixed order (pair k goes to lane k mod 32, each
- * lane folds its pairs in ascending k, then a fixed xor butterfly across the 32 lanes).
- * Passage: as bi_log_softmax.  Two launches: the merge (one warp per row), then one pass over
- * x.  Batch-invariant; a different fixed order from bi_log_softmax's, so the two agree to the
- * tolerance, not bit for bit.
- *
- *   x          device, [M, V] with row stride ldx >= V elements, x_dtype BI_BF16 or BI_F32: the
- *              C of the bi_matmul_lse call that wrote `partials` (N = V).
- *   partials   device, as written by that call ([M, bi_lse_partials_per_row(V), 2] fp32); read
- *              only.
- *   row_stats  device, fp32, [M, 2], 8-byte aligned, owned by the caller and overwritten with each
- *              row's (m, log s).
- *   y          device, fp32, [M, V] contiguous.
- *   Vector path when V % 8 == 0, x and y 16-byte aligned and ldx a multiple of 8 (bf16) / 4
- *   (fp32); any other layout takes a scalar path with the same arithmetic.
- */
-bi_status bi_log_softmax_partials(const void *x, int64_t ldx, bi_dtype x_dtype, const float *partials,
-                                  float *row_stats, float *y, int64_t M, int64_t V, void *stream);
 
 /*
  * bi_rmsnorm -- y = x * r * w,  r = 1 / sqrt( sum_j x_j^2 / H + eps ), per row.

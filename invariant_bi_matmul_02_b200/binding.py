@@ -30,10 +30,6 @@ SIGNATURES = {
                                 _i64, _i64, _i64, _p]),
     "bi_matmul_silu_mul": (ctypes.c_int, [_p, _i64, _p, _i64, ctypes.c_int, _p, _i64, _i64, _i64, _i64,
                                           _p]),
-    "bi_matmul_lse": (ctypes.c_int, [_p, _i64, _p, _i64, ctypes.c_int, _p, _i64, ctypes.c_int, _p,
-                                     _i64, _i64, _i64, _p]),
-    "bi_lse_partials_per_row": (_i64, [_i64]),
-    "bi_log_softmax_partials": (ctypes.c_int, [_p, _i64, ctypes.c_int, _p, _p, _p, _i64, _i64, _p]),
     "bi_rmsnorm": (ctypes.c_int, [_p, _p, _p, _i64, _i64, ctypes.c_float, _p]),
     "bi_mean": (ctypes.c_int, [_p, _p, _i64, _i64, _p]),
     "bi_log_softmax": (ctypes.c_int, [_p, ctypes.c_int, _p, _i64, _i64, _p]),
@@ -87,10 +83,24 @@ def _check(name: str, status: int):
         raise BiError(name, status)
 
 
+def _current_device() -> int:
+    return torch.cuda.current_device()
+
+
+def _same_device(index: int, name: str):
+    """The library launches on the current device and looks up its per-device state there, so
+    every tensor and the stream of a call must live on that device."""
+    cur = _current_device()
+    if index != cur:
+        raise ValueError(f"{name} is on cuda:{index} but the current device is cuda:{cur}; "
+                         "call under `with torch.cuda.device(...)`")
+
+
 def _stream(stream):
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, torch.cuda.Stream):
+        _same_device(stream.device.index, "stream")
         return stream.cuda_stream
     return int(stream)
 
@@ -100,6 +110,7 @@ def _need_cuda(t: torch.Tensor, name: str, dtypes):
         raise ValueError(f"{name} must be a CUDA tensor")
     if t.dtype not in dtypes:
         raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    _same_device(t.get_device(), name)
 
 
 def _ld(t: torch.Tensor, name: str) -> int:
@@ -202,65 +213,6 @@ def bi_matmul_silu_mul(a: torch.Tensor, b: torch.Tensor, b_layout: str = "nk",
     return out
 
 
-def bi_lse_partials_per_row(N: int) -> int:
-    return int(load().bi_lse_partials_per_row(int(N)))
-
-
-def bi_matmul_lse(a: torch.Tensor, b: torch.Tensor, b_layout: str = "nk", out: torch.Tensor | None = None,
-                  partials: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
-                  stream=None) -> tuple[torch.Tensor, torch.Tensor]:
-    """C = A . B as bi_matmul, plus one (max, sum of exp) pair per row and 256-column tile of C:
-    partials [M, bi_lse_partials_per_row(N), 2] fp32.  Returns (C, partials)."""
-    _need_cuda(a, "A", (torch.bfloat16,))
-    _need_cuda(b, "B", (torch.bfloat16,))
-    M, N, K = _gemm_shapes(a, b, b_layout)
-    if out is None:
-        out = torch.empty((M, N), dtype=out_dtype, device=a.device)
-    _need_cuda(out, "C", (torch.bfloat16, torch.float32))
-    if tuple(out.shape) != (M, N):
-        raise ValueError("C must be [M, N]")
-    P = bi_lse_partials_per_row(N)
-    if partials is None:
-        partials = torch.empty((M, P, 2), dtype=torch.float32, device=a.device)
-    _need_cuda(partials, "partials", (torch.float32,))
-    _contig(partials, "partials")
-    if tuple(partials.shape) != (M, P, 2):
-        raise ValueError(f"partials must be [M, {P}, 2]")
-    st = load().bi_matmul_lse(a.data_ptr(), _ld(a, "A"), b.data_ptr(), _ld(b, "B"),
-                              BI_B_KN if b_layout == "kn" else BI_B_NK, out.data_ptr(), _ld(out, "C"),
-                              _DT[out.dtype], partials.data_ptr(), M, N, K, _stream(stream))
-    _check("bi_matmul_lse", st)
-    return out, partials
-
-
-def bi_log_softmax_partials(x: torch.Tensor, partials: torch.Tensor, out: torch.Tensor | None = None,
-                            row_stats: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """y = log_softmax(x) over the last dimension from the pairs bi_matmul_lse wrote with x.
-    row_stats ([M, 2] fp32, optional) receives each row's (max, log sum exp(x - max))."""
-    _need_cuda(x, "x", tuple(_DT))
-    _need_cuda(partials, "partials", (torch.float32,))
-    _contig(partials, "partials")
-    M, V = x.shape
-    if tuple(partials.shape) != (M, bi_lse_partials_per_row(V), 2):
-        raise ValueError("partials do not match x")
-    if out is None:
-        out = torch.empty((M, V), dtype=torch.float32, device=x.device)
-    _need_cuda(out, "y", (torch.float32,))
-    _contig(out, "y")
-    if tuple(out.shape) != (M, V):
-        raise ValueError("y must be [M, V]")
-    if row_stats is None:
-        row_stats = torch.empty((M, 2), dtype=torch.float32, device=x.device)
-    _need_cuda(row_stats, "row_stats", (torch.float32,))
-    _contig(row_stats, "row_stats")
-    if tuple(row_stats.shape) != (M, 2):
-        raise ValueError("row_stats must be [M, 2]")
-    _check("bi_log_softmax_partials", load().bi_log_softmax_partials(
-        x.data_ptr(), _ld(x, "x"), _DT[x.dtype], partials.data_ptr(), row_stats.data_ptr(), out.data_ptr(),
-        M, V, _stream(stream)))
-    return out
-
-
 def bi_rmsnorm(x: torch.Tensor, w: torch.Tensor, eps: float = 1e-6, out: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
     """y = x / sqrt(mean(x^2) + eps) * w over the last dimension (bf16)."""
@@ -342,6 +294,7 @@ def bi_log_softmax_split(x: torch.Tensor, scratch: torch.Tensor | None = None,
         scratch = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
     if not scratch.is_cuda:
         raise ValueError("scratch must be device memory")
+    _same_device(scratch.get_device(), "scratch")
     nbytes = scratch.numel() * scratch.element_size()
     _check("bi_log_softmax_split", load().bi_log_softmax_split(
         x.data_ptr(), _DT[x.dtype], out.data_ptr(), M, V, scratch.data_ptr(), nbytes, _stream(stream)))
@@ -402,9 +355,15 @@ def bi_decode_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.T
     if out is None:
         out = torch.empty_like(q)
     _need_cuda(out, "out", (torch.bfloat16,))
+    _contig(out, "out")
+    if tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must be [B, Hq, D]")
     if scratch is None:
         scratch = torch.empty(max(bi_decode_attention_scratch_bytes(B, Hq, D, Lmax), 16), dtype=torch.uint8,
                               device=q.device)
+    if not scratch.is_cuda:
+        raise ValueError("scratch must be device memory")
+    _same_device(scratch.get_device(), "scratch")
     nbytes = scratch.numel() * scratch.element_size()
     _check("bi_decode_attention", load().bi_decode_attention(
         q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seq_lens.data_ptr(), out.data_ptr(),

@@ -122,8 +122,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 
 // 2-D bf16 tensor map over a row-major matrix: `inner` contiguous elements per row,
 // `outer` rows `ld` elements apart, box inner x outer, 128-byte swizzle, zero fill.
-bi_status encode_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint64_t ld,
-                     uint32_t box_inner, uint32_t box_outer)
+bi_status encode_map_uncached(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint64_t ld,
+                              uint32_t box_inner, uint32_t box_outer)
 {
     auto enc = tensor_map_encoder();
     if (!enc) return BI_ERR_CUDA;
@@ -137,7 +137,75 @@ bi_status encode_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_
     return r == CUDA_SUCCESS ? BI_OK : BI_ERR_CUDA;
 }
 
-bi_status launched() { return cudaGetLastError() == cudaSuccess ? BI_OK : BI_ERR_CUDA; }
+// Encoded tensor maps, keyed by everything the encoding reads (base address, extents, row
+// stride, box).  A map is a pure function of its key, so a hit returns exactly the map a fresh
+// encoding would; a freed and re-allocated buffer at the same address with the same shape gets
+// the same, still correct, map.  Direct-mapped with kMapCacheSlots slots under one mutex: a
+// colliding key replaces the slot.  A GEMM call looks up two maps.
+struct MapKey {
+    uint64_t base, inner, outer, ld;
+    uint32_t box_inner, box_outer;
+    bool operator==(const MapKey &o) const
+    {
+        return base == o.base && inner == o.inner && outer == o.outer && ld == o.ld &&
+               box_inner == o.box_inner && box_outer == o.box_outer;
+    }
+};
+struct MapSlot {
+    bool used = false;
+    MapKey key{};
+    CUtensorMap map{};
+};
+constexpr int kMapCacheSlots = 256;
+std::mutex g_map_mu;
+MapSlot g_map_cache[kMapCacheSlots];
+uint64_t g_map_hits = 0, g_map_misses = 0;
+
+inline uint32_t map_slot(const MapKey &k)
+{
+    uint64_t h = 0x9E3779B97F4A7C15ull;
+    for (uint64_t v : {k.base, k.inner, k.outer, k.ld, (uint64_t)k.box_inner << 32 | k.box_outer}) {
+        h ^= v + 0x9E3779B97F4A7C15ull + (h << 6) + (h >> 2);
+    }
+    return (uint32_t)(h % kMapCacheSlots);
+}
+
+bi_status encode_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint64_t ld,
+                     uint32_t box_inner, uint32_t box_outer)
+{
+    const MapKey key{reinterpret_cast<uint64_t>(base), inner, outer, ld, box_inner, box_outer};
+    const uint32_t slot = map_slot(key);
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    MapSlot &e = g_map_cache[slot];
+    if (e.used && e.key == key) {
+        ++g_map_hits;
+        *map = e.map;
+        return BI_OK;
+    }
+    ++g_map_misses;
+    const bi_status st = encode_map_uncached(map, base, inner, outer, ld, box_inner, box_outer);
+    if (st != BI_OK) return st;
+    e.used = true;
+    e.key = key;
+    e.map = *map;
+    return BI_OK;
+}
+
+// Launch `kernel` on `s` and report the launch's own result.  cudaLaunchKernelEx returns the
+// error of this launch, so a failure left behind by some other library's launch on this thread
+// is neither reported as ours nor cleared.
+template <typename... KArgs, typename... Args>
+bi_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? BI_OK : BI_ERR_CUDA;
+}
 
 // Launch `kernel` with programmatic stream serialization: it may start while the previous kernel
 // in the stream finishes, and waits (griddep_wait) for it before touching global memory.
@@ -184,15 +252,13 @@ bi_status launch_row_clusters(void (*kernel)(KArgs...), int64_t M, size_t smem, 
 // the output is silu(A . gate^T) * (A . up^T).
 bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, const void *A, int64_t lda,
                       const void *B, int64_t ldb, int b_layout, void *C, int64_t ldc, int c_dtype,
-                      int64_t M, int64_t N, int64_t K, void *stream, int fuse_silu = 0,
-                      float *lse_partial = nullptr)
+                      int64_t M, int64_t N, int64_t K, void *stream, int fuse_silu = 0)
 {
     if (M < 0 || N < 0 || K < 0) return BI_ERR_INVALID_ARG;
     if (b_layout != BI_B_KN && b_layout != BI_B_NK) return BI_ERR_INVALID_ARG;
     if (c_dtype != BI_BF16 && c_dtype != BI_F32) return BI_ERR_INVALID_ARG;
     if (M > kI32Max || (fuse_silu ? 2 * N : N) > kI32Max || K > kI32Max) return BI_ERR_UNSUPPORTED;
     if (M == 0 || N == 0) return BI_OK;
-    if (lse_partial && (fuse_silu || reinterpret_cast<uintptr_t>(lse_partial) % 8 != 0)) return BI_ERR_ALIGNMENT;
     const int64_t b_rows = fuse_silu ? 2 * N : N;  // extent of B along the output dimension
     if (!C || ldc < N) return BI_ERR_INVALID_ARG;
     if (addend_mode != bi::kAddNone) {
@@ -231,21 +297,13 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
     p.addend = static_cast<const __nv_bfloat16 *>(input);
     p.status = dev->status;
     p.wait_limit_ns = kWaitLimitNs;
-    p.lse_partial = reinterpret_cast<float2 *>(lse_partial);
-    p.lse_per_row = p.n_blocks;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
     if (K == 0 && !fuse_silu) {
         const int64_t total = M * N;
         int64_t blocks = (total + 255) / 256;
         if (blocks > (int64_t)dev->sms * 16) blocks = (int64_t)dev->sms * 16;
-        bi::gemm_k0_fill_kernel<<<(unsigned)blocks, 256, 0, s>>>(p);
-        if (lse_partial) {
-            int64_t pb = (M * p.lse_per_row + 127) / 128;
-            if (pb > (int64_t)dev->sms * 16) pb = (int64_t)dev->sms * 16;
-            bi::gemm_k0_partials_kernel<<<(unsigned)pb, 128, 0, s>>>(p);
-        }
-        return launched();
+        return launch(bi::gemm_k0_fill_kernel, dim3((unsigned)blocks), dim3(256), 0, s, p);
     }
 
     const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
@@ -263,9 +321,8 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
 
     const int64_t pairs = dev->gemm_clusters;
     const int grid = 2 * (int)(tiles < pairs ? tiles : pairs);
-    st = launch_pdl(bi::gemm_bf16_pair_kernel, dim3(grid), dim3(bi::kGemmThreads), (size_t)bi::kPairSmem, s, tm_a,
-                    tm_b, p);
-    return st != BI_OK ? st : launched();
+    return launch_pdl(bi::gemm_bf16_pair_kernel, dim3(grid), dim3(bi::kGemmThreads), (size_t)bi::kPairSmem, s,
+                      tm_a, tm_b, p);
 }
 
 __global__ void selftest_wait_kernel(int32_t *status, uint64_t limit_ns)
@@ -281,6 +338,20 @@ __global__ void selftest_wait_kernel(int32_t *status, uint64_t limit_ns)
     // Phase 0 of `bar` never completes: nothing arrives on it.
     if (threadIdx.x == 0) bi::wait_bounded(&bar, 0, &abort_flag, status, limit_ns);
     __syncthreads();
+}
+
+// The two launches of the split log_softmax: per-(row, chunk) partials, then the merge and write.
+bi_status split_launches(bool bf16, dim3 grid, cudaStream_t s, const uint8_t *xb, float2 *part, float *y, int64_t V)
+{
+    bi_status st = bf16 ? launch(bi::log_softmax_split_stats_kernel<true>, grid, dim3(bi::kSplitThreads), 0, s, xb,
+                                 part, V)
+                        : launch(bi::log_softmax_split_stats_kernel<false>, grid, dim3(bi::kSplitThreads), 0, s, xb,
+                                 part, V);
+    if (st != BI_OK) return st;
+    return bf16 ? launch(bi::log_softmax_split_write_kernel<true>, grid, dim3(bi::kSplitThreads), 0, s, xb,
+                         static_cast<const float2 *>(part), y, V)
+                : launch(bi::log_softmax_split_write_kernel<false>, grid, dim3(bi::kSplitThreads), 0, s, xb,
+                         static_cast<const float2 *>(part), y, V);
 }
 
 inline unsigned elementwise_blocks(int64_t work, int sms)
@@ -321,55 +392,6 @@ bi_status bi_matmul_silu_mul(const void *A, int64_t lda, const void *B, int64_t 
                        1);
 }
 
-int64_t bi_lse_partials_per_row(int64_t N)
-{
-    return N <= 0 ? 0 : (N + bi::kPairBN - 1) / bi::kPairBN;
-}
-
-bi_status bi_matmul_lse(const void *A, int64_t lda, const void *B, int64_t ldb, bi_b_layout b_layout, void *C,
-                        int64_t ldc, bi_dtype c_dtype, float *partials, int64_t M, int64_t N, int64_t K,
-                        void *stream)
-{
-    if (M > 0 && N > 0 && !partials) return BI_ERR_INVALID_ARG;
-    return gemm_common(nullptr, 0, bi::kAddNone, A, lda, B, ldb, b_layout, C, ldc, c_dtype, M, N, K, stream, 0,
-                       partials);
-}
-
-bi_status bi_log_softmax_partials(const void *x, int64_t ldx, bi_dtype x_dtype, const float *partials,
-                                  float *row_stats, float *y, int64_t M, int64_t V, void *stream)
-{
-    if (M < 0 || V < 0) return BI_ERR_INVALID_ARG;
-    if (x_dtype != BI_BF16 && x_dtype != BI_F32) return BI_ERR_INVALID_ARG;
-    if (M > kI32Max || V > kI32Max) return BI_ERR_UNSUPPORTED;
-    if (M == 0) return BI_OK;
-    if (V == 0 || !x || !y || !partials || !row_stats || ldx < V) return BI_ERR_INVALID_ARG;
-    if (reinterpret_cast<uintptr_t>(partials) % 8 != 0 || reinterpret_cast<uintptr_t>(row_stats) % 8 != 0)
-        return BI_ERR_ALIGNMENT;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool bf16 = x_dtype == BI_BF16;
-    const int64_t P = bi_lse_partials_per_row(V);
-    const float2 *part = reinterpret_cast<const float2 *>(partials);
-    float2 *rs = reinterpret_cast<float2 *>(row_stats);
-    bi::lse_row_stats_kernel<<<(unsigned)((M + bi::kRowStatWarps - 1) / bi::kRowStatWarps),
-                               bi::kRowStatWarps * 32, 0, s>>>(part, P, rs, M);
-    const bool vec = V % 8 == 0 && ldx % (bf16 ? 8 : 4) == 0 && aligned16(x) && aligned16(y);
-    const unsigned chunks = (unsigned)bi::apply_chunks(V);
-    for (int64_t row0 = 0; row0 < M; row0 += 65535) {  // rows on grid.y
-        const dim3 grid(chunks, (unsigned)(M - row0 < 65535 ? M - row0 : 65535));
-        if (vec && bf16)
-            bi::log_softmax_apply_vec_kernel<true><<<grid, bi::kApplyThreads, 0, s>>>(
-                static_cast<const uint8_t *>(x), ldx, rs, y, V, row0);
-        else if (vec)
-            bi::log_softmax_apply_vec_kernel<false><<<grid, bi::kApplyThreads, 0, s>>>(
-                static_cast<const uint8_t *>(x), ldx, rs, y, V, row0);
-        else if (bf16)
-            bi::log_softmax_apply_scalar_kernel<true><<<grid, bi::kApplyThreads, 0, s>>>(x, ldx, rs, y, V, row0);
-        else
-            bi::log_softmax_apply_scalar_kernel<false><<<grid, bi::kApplyThreads, 0, s>>>(x, ldx, rs, y, V, row0);
-    }
-    return launched();
-}
-
 bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H, float eps,
                      void *stream)
 {
@@ -392,17 +414,15 @@ bi_status bi_rmsnorm(const void *x, const void *w, void *y, int64_t M, int64_t H
         case 3: st = launch_pdl(bi::rmsnorm_vec_kernel<3>, dim3((unsigned)M), dim3(T), 0, s, xv, wv, yv, H, eps); break;
         case 4: st = launch_pdl(bi::rmsnorm_vec_kernel<4>, dim3((unsigned)M), dim3(T), 0, s, xv, wv, yv, H, eps); break;
         default:
-            bi::rmsnorm_scalar_kernel<<<(unsigned)M, T, 0, s>>>(
-                static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w),
-                static_cast<__nv_bfloat16 *>(y), H, eps);
+            st = launch(bi::rmsnorm_scalar_kernel, dim3((unsigned)M), dim3(T), 0, s,
+                        static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w),
+                        static_cast<__nv_bfloat16 *>(y), H, eps);
         }
-        if (st != BI_OK) return st;
-    } else {
-        bi::rmsnorm_scalar_kernel<<<(unsigned)M, T, 0, s>>>(
-            static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w),
-            static_cast<__nv_bfloat16 *>(y), H, eps);
+        return st;
     }
-    return launched();
+    return launch(bi::rmsnorm_scalar_kernel, dim3((unsigned)M), dim3(T), 0, s,
+                  static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w),
+                  static_cast<__nv_bfloat16 *>(y), H, eps);
 }
 
 bi_status bi_mean(const float *x, float *y, int64_t M, int64_t H, void *stream)
@@ -422,11 +442,9 @@ bi_status bi_mean(const float *x, float *y, int64_t M, int64_t H, void *stream)
         else
             st = launch_pdl(bi::mean_vec_kernel<false>, dim3((unsigned)M), dim3(T), 0, s,
                             reinterpret_cast<const float4 *>(x), y, H);
-        if (st != BI_OK) return st;
-    } else {
-        bi::mean_scalar_kernel<<<(unsigned)M, T, 0, s>>>(x, y, H);
+        return st;
     }
-    return launched();
+    return launch(bi::mean_scalar_kernel, dim3((unsigned)M), dim3(T), 0, s, x, y, H);
 }
 
 bi_status bi_log_softmax(const void *x, bi_dtype x_dtype, float *y, int64_t M, int64_t V, void *stream)
@@ -450,14 +468,10 @@ bi_status bi_log_softmax(const void *x, bi_dtype x_dtype, float *y, int64_t M, i
                                (size_t)bi::kLsmSmem, s, xb, y, V, dev->status, kWaitLimitNs)
                   : launch_pdl(bi::log_softmax_stream_kernel<false>, dim3((unsigned)M), dim3(bi::kLsmThreads),
                                (size_t)bi::kLsmSmem, s, xb, y, V, dev->status, kWaitLimitNs);
-        if (st != BI_OK) return st;
-    } else {
-        if (bf16)
-            bi::log_softmax_scalar_kernel<true><<<(unsigned)M, T, 0, s>>>(x, y, V);
-        else
-            bi::log_softmax_scalar_kernel<false><<<(unsigned)M, T, 0, s>>>(x, y, V);
+        return st;
     }
-    return launched();
+    return bf16 ? launch(bi::log_softmax_scalar_kernel<true>, dim3((unsigned)M), dim3(T), 0, s, x, y, V)
+                : launch(bi::log_softmax_scalar_kernel<false>, dim3((unsigned)M), dim3(T), 0, s, x, y, V);
 }
 
 bi_status bi_log_softmax_cluster(const void *x, bi_dtype x_dtype, float *y, int64_t M, int64_t V, void *stream)
@@ -482,7 +496,7 @@ bi_status bi_log_softmax_cluster(const void *x, bi_dtype x_dtype, float *y, int6
                                     dev->status, kWaitLimitNs)
               : launch_row_clusters(bi::log_softmax_cluster_kernel<false>, M, (size_t)slice_bytes, s, xb, y, V,
                                     dev->status, kWaitLimitNs);
-    return st != BI_OK ? st : launched();
+    return st;
 }
 
 size_t bi_log_softmax_split_scratch_bytes(int64_t M, int64_t V)
@@ -506,14 +520,7 @@ bi_status bi_log_softmax_split(const void *x, bi_dtype x_dtype, float *y, int64_
     const dim3 grid((unsigned)bi::split_chunks(V), (unsigned)M);
     const uint8_t *xb = static_cast<const uint8_t *>(x);
     float2 *part = static_cast<float2 *>(scratch);
-    if (x_dtype == BI_BF16) {
-        bi::log_softmax_split_stats_kernel<true><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, V);
-        bi::log_softmax_split_write_kernel<true><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, y, V);
-    } else {
-        bi::log_softmax_split_stats_kernel<false><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, V);
-        bi::log_softmax_split_write_kernel<false><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, y, V);
-    }
-    return launched();
+    return split_launches(x_dtype == BI_BF16, grid, s, xb, part, y, V);
 }
 
 }  // extern "C"
@@ -576,14 +583,7 @@ bi_status bi_log_softmax_split_noalloc(const void *x, bi_dtype x_dtype, float *y
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const dim3 grid((unsigned)bi::split_chunks(V), (unsigned)M);
     const uint8_t *xb = static_cast<const uint8_t *>(x);
-    if (x_dtype == BI_BF16) {
-        bi::log_softmax_split_stats_kernel<true><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, V);
-        bi::log_softmax_split_write_kernel<true><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, y, V);
-    } else {
-        bi::log_softmax_split_stats_kernel<false><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, V);
-        bi::log_softmax_split_write_kernel<false><<<grid, bi::kSplitThreads, 0, s>>>(xb, part, y, V);
-    }
-    return launched();
+    return split_launches(x_dtype == BI_BF16, grid, s, xb, part, y, V);
 }
 
 size_t bi_decode_attention_scratch_bytes(int64_t B, int64_t Hq, int64_t D, int64_t Lmax)
@@ -635,8 +635,7 @@ bi_status bi_decode_attention(const void *q, const void *k_cache, const void *v_
     st = launch_pdl(bi::decode_attention_combine_kernel, dim3((unsigned)Hq, (unsigned)B), dim3(bi::kAttnD), 0, s,
                     static_cast<const float2 *>(part_ms), static_cast<const float *>(part_acc), seq_lens,
                     static_cast<__nv_bfloat16 *>(out), (int)Hq, Lmax);
-    if (st != BI_OK) return st;
-    return launched();
+    return st;
 }
 
 bi_status bi_silu_mul(const void *gu, void *h, int64_t M, int64_t F, void *stream)
@@ -652,13 +651,11 @@ bi_status bi_silu_mul(const void *gu, void *h, int64_t M, int64_t F, void *strea
     if (F % 8 == 0) {
         if (!aligned16(gu) || !aligned16(h)) return BI_ERR_ALIGNMENT;
         const int64_t work = M * (F / 8);
-        bi::silu_mul_vec_kernel<<<elementwise_blocks(work, dev->sms), 256, 0, s>>>(
-            static_cast<const uint4 *>(gu), static_cast<uint4 *>(h), M, F);
-    } else {
-        bi::silu_mul_scalar_kernel<<<elementwise_blocks(M * F, dev->sms), 256, 0, s>>>(
-            static_cast<const __nv_bfloat16 *>(gu), static_cast<__nv_bfloat16 *>(h), M, F);
+        return launch(bi::silu_mul_vec_kernel, dim3(elementwise_blocks(work, dev->sms)), dim3(256), 0, s,
+                      static_cast<const uint4 *>(gu), static_cast<uint4 *>(h), M, F);
     }
-    return launched();
+    return launch(bi::silu_mul_scalar_kernel, dim3(elementwise_blocks(M * F, dev->sms)), dim3(256), 0, s,
+                  static_cast<const __nv_bfloat16 *>(gu), static_cast<__nv_bfloat16 *>(h), M, F);
 }
 
 bi_status bi_get_device_status(void *stream, int32_t *out)
@@ -679,9 +676,8 @@ bi_status bi_selftest_wait_timeout(int64_t limit_ns, void *stream)
     DeviceState *dev = nullptr;
     bi_status st = device_state(&dev);
     if (st != BI_OK) return st;
-    selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev->status,
-                                                                          (uint64_t)limit_ns);
-    return launched();
+    return launch(selftest_wait_kernel, dim3(1), dim3(32), 0, static_cast<cudaStream_t>(stream), dev->status,
+                  (uint64_t)limit_ns);
 }
 
 const char *bi_status_string(bi_status status)

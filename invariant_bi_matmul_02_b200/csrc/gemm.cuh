@@ -6,7 +6,6 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
-#include "maxsum.cuh"
 #include "ptx.cuh"
 
 namespace bi {
@@ -34,8 +33,6 @@ struct GemmParams {
     const __nv_bfloat16 *addend;
     int32_t *status;        // device status word
     uint64_t wait_limit_ns;
-    float2 *lse_partial;    // non-null: (max, sum of exp) of each row over each output tile
-    int64_t lse_per_row;    // partials per row = n_blocks
 };
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float(b16 << 16); }
@@ -96,19 +93,6 @@ __device__ __forceinline__ void store_row_chunk(const GemmParams &p, int64_t row
             for (int j = 0; j < 32 && col0 + j < p.N; ++j) dst[j] = __float2bfloat16_rn(v[j]);
         }
     }
-}
-
-// Fold one stored row chunk (columns col0 .. col0+31, those below N) into the tile's running
-// (max, sum of exp) pair.  The values folded are the ones stored in C: rounded to bf16 when C
-// is bf16, so that the pair describes exactly the logits a later pass reads back.
-__device__ __forceinline__ void lse_fold_chunk(const GemmParams &p, int64_t col0, float (&v)[32], MaxSum &acc)
-{
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const float r = p.c_f32 ? v[j] : __bfloat162float(__float2bfloat16_rn(v[j]));
-        v[j] = col0 + j < p.N ? r : kNegInf;
-    }
-    lsm_accumulate(acc, v);
 }
 
 // silu(g) * u of one row chunk, fp32 inside, stored as bf16 (columns col0 .. col0+31 of h).

@@ -230,7 +230,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     store_silu_chunk(p, row, col0, gv, uv);
                 }
             }
-            MaxSum tile_lse{kNegInf, 0.0f};
 #pragma unroll 1
             for (int c = 0; !p.fuse_silu && c < kPairBN / 32; ++c) {
                 uint32_t r[32];
@@ -244,12 +243,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     const bool full_chunk = col0 + 32 <= p.N;
                     add_addend(p, row, col0, full_chunk, v);
                     store_row_chunk(p, row, col0, full_chunk, v);
-                    if (p.lse_partial) lse_fold_chunk(p, col0, v, tile_lse);
                 }
             }
-            // The row's pair for this tile: its 8 chunks folded in ascending column order.
-            if (p.lse_partial && row < p.M)
-                p.lse_partial[row * p.lse_per_row + tile / m_blocks] = make_float2(tile_lse.m, tile_lse.s);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tempty_leader0 + acc * sizeof(uint64_t));
@@ -263,32 +258,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     if (warp == 1) {
         tc_fence_after_sync();
         tmem_dealloc_pair(tmem_base, kPairTmemCols);
-    }
-}
-
-// K = 0 with per-tile partials: C is the addend (or 0), so each tile's pair is folded from it
-// by the same per-chunk sequence as the GEMM epilogue, one thread per (row, tile).
-__global__ void gemm_k0_partials_kernel(const GemmParams p)
-{
-    const int64_t total = (int64_t)p.M * p.lse_per_row;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-         e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t i = e / p.lse_per_row, t = e % p.lse_per_row;
-        MaxSum acc{kNegInf, 0.0f};
-        for (int c = 0; c < kPairBN / 32; ++c) {
-            const int64_t col0 = t * kPairBN + 32 * c;
-            if (col0 >= p.N) break;
-            float v[32];
-            for (int j = 0; j < 32; ++j) {
-                float a = 0.0f;
-                if (col0 + j < p.N && p.addend_mode == kAddBias) a = __bfloat162float(p.addend[col0 + j]);
-                if (col0 + j < p.N && p.addend_mode == kAddMatrix)
-                    a = __bfloat162float(p.addend[i * p.ld_addend + col0 + j]);
-                v[j] = a;
-            }
-            lse_fold_chunk(p, col0, v, acc);
-        }
-        p.lse_partial[e] = make_float2(acc.m, acc.s);
     }
 }
 

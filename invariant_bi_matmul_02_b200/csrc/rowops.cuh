@@ -653,92 +653,6 @@ __global__ void __launch_bounds__(kSplitThreads) log_softmax_split_write_kernel(
     }
 }
 
-// --------------------------------------------------------------- log_softmax from tile partials
-
-// Second half of the LM-head log_softmax whose first half runs in the GEMM epilogue: the GEMM
-// leaves, per row, one (max, sum of exp) pair for each of its P output tiles.
-//   Launch 1 (one warp per row): lane l folds pairs l, l+32, ... in ascending order, then a
-//            fixed xor butterfly gives the row's (m, log s).
-//   Launch 2 (block (c, i)): y = (x - m) - log(s) for chunk c of row i, kApplyChunk elements;
-//            every load of the chunk is issued before the row's (m, log s) is read.
-// x rows are ldx elements apart; y is [M, V] contiguous.
-constexpr int kRowStatWarps = 8;
-constexpr int kApplyThreads = 256;
-constexpr int kApplyGroups = 4;                                   // 8-element groups per thread
-constexpr int kApplyChunk = kApplyThreads * kApplyGroups * 8;    // 8192 elements per block
-
-__host__ __device__ inline int64_t apply_chunks(int64_t V) { return (V + kApplyChunk - 1) / kApplyChunk; }
-
-__global__ void __launch_bounds__(kRowStatWarps * 32) lse_row_stats_kernel(
-    const float2 *__restrict__ partial, int64_t P, float2 *__restrict__ row_stats, int64_t M)
-{
-    const int64_t row = (int64_t)blockIdx.x * kRowStatWarps + (threadIdx.x >> 5);
-    if (row >= M) return;
-    const int lane = threadIdx.x & 31;
-    const float2 *pr = partial + row * P;
-    MaxSum acc{kNegInf, 0.0f};
-    int64_t k = lane;
-    for (; k + 96 < P; k += 128) {  // four pairs in flight per lane, folded in ascending order
-        const float2 p0 = __ldg(pr + k), p1 = __ldg(pr + k + 32), p2 = __ldg(pr + k + 64), p3 = __ldg(pr + k + 96);
-        acc = merge(acc, MaxSum{p0.x, p0.y});
-        acc = merge(acc, MaxSum{p1.x, p1.y});
-        acc = merge(acc, MaxSum{p2.x, p2.y});
-        acc = merge(acc, MaxSum{p3.x, p3.y});
-    }
-    for (; k < P; k += 32) {
-        const float2 pk = __ldg(pr + k);
-        acc = merge(acc, MaxSum{pk.x, pk.y});
-    }
-    acc = warp_merge(acc);
-    if (lane == 0) row_stats[row] = make_float2(acc.m, __logf(acc.s));
-}
-
-// V % 8 == 0, x 16-byte aligned with ldx % 8 == 0 (bf16) or ldx % 4 == 0 (fp32).
-template <bool BF16>
-__global__ void __launch_bounds__(kApplyThreads) log_softmax_apply_vec_kernel(
-    const uint8_t *__restrict__ x, int64_t ldx, const float2 *__restrict__ row_stats,
-    float *__restrict__ y, int64_t V, int64_t row0)
-{
-    constexpr int kElem = BF16 ? 2 : 4;
-    const int64_t row = row0 + blockIdx.y;
-    const int64_t e0 = blockIdx.x * (int64_t)kApplyChunk;
-    const uint8_t *xr = x + row * ldx * kElem;
-    float v[kApplyGroups][8];
-#pragma unroll
-    for (int g = 0; g < kApplyGroups; ++g) {
-        const int64_t e = e0 + 8 * (int64_t)(g * kApplyThreads + threadIdx.x);
-        if (e < V) split_load8<BF16>(xr, e, v[g]);
-    }
-    const float2 st = __ldg(row_stats + row);
-    const float m = st.x, ls = st.y;
-    float *yr = y + row * V;
-#pragma unroll
-    for (int g = 0; g < kApplyGroups; ++g) {
-        const int64_t e = e0 + 8 * (int64_t)(g * kApplyThreads + threadIdx.x);
-        if (e >= V) break;
-        float4 *dst = reinterpret_cast<float4 *>(yr + e);
-        __stcs(dst, make_float4((v[g][0] - m) - ls, (v[g][1] - m) - ls, (v[g][2] - m) - ls, (v[g][3] - m) - ls));
-        __stcs(dst + 1, make_float4((v[g][4] - m) - ls, (v[g][5] - m) - ls, (v[g][6] - m) - ls, (v[g][7] - m) - ls));
-    }
-}
-
-// Any V and ldx: element e0 + g * T + t belongs to thread t.
-template <bool BF16>
-__global__ void __launch_bounds__(kApplyThreads) log_softmax_apply_scalar_kernel(
-    const void *__restrict__ xv, int64_t ldx, const float2 *__restrict__ row_stats,
-    float *__restrict__ y, int64_t V, int64_t row0)
-{
-    const int64_t row = row0 + blockIdx.y;
-    const int64_t e0 = blockIdx.x * (int64_t)kApplyChunk;
-    const float2 st = __ldg(row_stats + row);
-    const float m = st.x, ls = st.y;
-    for (int64_t e = e0 + threadIdx.x; e < V && e < e0 + kApplyChunk; e += kApplyThreads) {
-        const float xe = BF16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(xv)[row * ldx + e])
-                              : static_cast<const float *>(xv)[row * ldx + e];
-        y[row * V + e] = (xe - m) - ls;
-    }
-}
-
 // --------------------------------------------------------------- SiLU * up
 
 __device__ __forceinline__ float silu_mul1(float g, float u)

@@ -221,39 +221,6 @@ int oracle_log_softmax_bf16(const uint16_t *x, double *y, int64_t M, int64_t V, 
 }
 
 /*
- * Per-tile statistics of a log_softmax: for each row i of x [M, V] (bf16 bit patterns) and
- * each tile t of `tile` consecutive columns [t*tile, min((t+1)*tile, V)),
- *   m_it = max over the tile of x_ij,   s_it = sum over the tile of exp(x_ij - m_it).
- * These are the (max, sum of exp) pairs a log_softmax reduces a row to before merging them
- * (the two-pass form of log_softmax above, cut into tiles); they carry the whole row's
- * statistics, because max_t m_t is the row maximum m and
- * sum_t s_t * exp(m_t - m) = sum_j exp(x_j - m).  m and s are [M, P], P = ceil(V / tile).
- */
-int oracle_tile_max_sumexp_bf16(const uint16_t *x, double *m, double *s, int64_t M, int64_t V,
-                                int64_t tile, int nthreads)
-{
-    if (M < 0 || V <= 0 || tile <= 0) return (M == 0 && V >= 0 && tile > 0) ? 0 : -1;
-    if (M > 0 && (x == 0 || m == 0 || s == 0)) return -1;
-    const int64_t P = (V + tile - 1) / tile;
-#pragma omp parallel for num_threads(threads_or_one(nthreads)) schedule(static)
-    for (int64_t i = 0; i < M; ++i) {
-        for (int64_t t = 0; t < P; ++t) {
-            const int64_t j0 = t * tile, j1 = (j0 + tile < V) ? j0 + tile : V;
-            double mt = -INFINITY;
-            for (int64_t j = j0; j < j1; ++j) {
-                const double v = bf16_to_double(x[i * V + j]);
-                if (v > mt) mt = v;
-            }
-            double st = 0.0;
-            for (int64_t j = j0; j < j1; ++j) st += exp(bf16_to_double(x[i * V + j]) - mt);
-            m[i * P + t] = mt;
-            s[i * P + t] = st;
-        }
-    }
-    return 0;
-}
-
-/*
  * Gated-MLP glue: gu is [M, 2F] bf16 with the gate in columns [0, F) and the
  * up projection in columns [F, 2F).  h_ij = silu(g_ij) * u_ij with
  * silu(g) = g / (1 + exp(-g)).

@@ -41,8 +41,6 @@ def _lib():
         lib.oracle_log_softmax_bf16.argtypes = [_ptr, _ptr, _i64, _i64, ctypes.c_int]
         lib.oracle_silu_mul.argtypes = [_ptr, _ptr, _i64, _i64, ctypes.c_int]
         lib.oracle_silu_mul_f64.argtypes = [_ptr, _ptr, _i64, _i64, ctypes.c_int]
-        lib.oracle_tile_max_sumexp_bf16.restype = ctypes.c_int
-        lib.oracle_tile_max_sumexp_bf16.argtypes = [_ptr, _ptr, _ptr, _i64, _i64, _i64, ctypes.c_int]
         lib.oracle_decode_attention.restype = ctypes.c_int
         lib.oracle_decode_attention.argtypes = [_ptr, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _i64, _i64,
                                                 ctypes.c_double, ctypes.c_int]
@@ -164,19 +162,6 @@ def log_softmax(x, nthreads=None) -> np.ndarray:
         raise TypeError("x must be float32 or bf16 bits (uint16)")
     _check(rc, "oracle_log_softmax")
     return y
-
-
-def tile_max_sumexp(x_bits, tile: int, nthreads=None) -> tuple[np.ndarray, np.ndarray]:
-    """Per row and per tile of `tile` columns: (max, sum of exp(x - max)) of bf16 x.
-    Returns m, s as [M, ceil(V / tile)] float64."""
-    x = np.ascontiguousarray(_as(x_bits, np.uint16, "x"))
-    M, V = x.shape
-    P = -(-V // tile) if V else 0
-    m = np.zeros((M, P), dtype=np.float64)
-    s = np.zeros((M, P), dtype=np.float64)
-    _check(_lib().oracle_tile_max_sumexp_bf16(x.ctypes.data, m.ctypes.data, s.ctypes.data, M, V, int(tile),
-                                               _threads(nthreads)), "oracle_tile_max_sumexp")
-    return m, s
 
 
 def silu_mul(gu_bits, nthreads=None) -> np.ndarray:

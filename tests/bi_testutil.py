@@ -46,6 +46,22 @@ def assert_lsm_close(gpu: torch.Tensor, ref: np.ndarray, what: str = ""):
     assert worst <= LSM_ABS, f"{what}: max |err| {worst} > {LSM_ABS}"
 
 
+def assert_lsm_close_ieee(gpu: torch.Tensor, ref: np.ndarray, what: str = ""):
+    """log_softmax parity on rows with masked (-inf) or non-finite entries: where the oracle's
+    value is finite the kernel's must be within LSM_ABS of it; where it is +-inf the kernel's
+    must be the same infinity; where it is NaN the kernel's must be NaN."""
+    g = to_np64(gpu)
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.isfinite(g), fin), f"{what}: finite entries differ from the oracle's"
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(g), nan), f"{what}: NaN entries differ from the oracle's"
+    inf = ~fin & ~nan
+    assert np.array_equal(g[inf], ref[inf]), f"{what}: infinite entries differ from the oracle's"
+    if fin.any():
+        worst = float(np.abs(g[fin] - ref[fin]).max())
+        assert worst <= LSM_ABS, f"{what}: max |err| {worst} > {LSM_ABS}"
+
+
 def mean_chain_depth(H: int) -> int:
     """Longest chain of fp32 additions in bi_mean's order for rows of H elements: one block of
     T threads per row (T = 32 ceil(((H / 4 + 3) / 4) / 32), clamped to [32, 1024]).

@@ -84,18 +84,6 @@ def test_host_validation_without_a_gpu(lib):
     assert lib.bi_silu_mul(NULL, NULL, 2, 8, NULL) == I
     # fused gate/up with [K, 2F] weights: the up half's first column F must be a multiple of 8
     assert lib.bi_matmul_silu_mul(fake, 200, fake, 1000, 0, fake, 504, 77, 500, 200, NULL) == A
-    # LM-head log_softmax halves: null or misaligned pairs, short row stride
-    assert lib.bi_matmul_lse(fake, 8, fake, 8, 1, fake, 8, 0, NULL, 2, 8, 8, NULL) == I
-    assert lib.bi_matmul_lse(fake, 8, fake, 8, 1, fake, 8, 0, fake + 4, 2, 8, 8, NULL) == A
-    assert lib.bi_matmul_lse(NULL, 8, NULL, 8, 1, NULL, 8, 0, NULL, 0, 8, 8, NULL) == binding.BI_OK
-    assert lib.bi_log_softmax_partials(fake, 7, 0, fake, fake, fake, 2, 8, NULL) == I
-    assert lib.bi_log_softmax_partials(fake, 8, 0, NULL, fake, fake, 2, 8, NULL) == I
-    assert lib.bi_log_softmax_partials(fake, 8, 0, fake, NULL, fake, 2, 8, NULL) == I
-    assert lib.bi_log_softmax_partials(fake, 8, 0, fake + 4, fake, fake, 2, 8, NULL) == A
-    assert lib.bi_log_softmax_partials(fake, 8, 0, fake, fake + 4, fake, 2, 8, NULL) == A
-    assert lib.bi_log_softmax_partials(fake, 8, 3, fake, fake, fake, 2, 8, NULL) == I
-    assert lib.bi_log_softmax_partials(NULL, 8, 0, NULL, NULL, NULL, 0, 8, NULL) == binding.BI_OK
-    assert [lib.bi_lse_partials_per_row(n) for n in (0, 1, 256, 257, 151936)] == [0, 1, 1, 2, 594]
     assert lib.bi_selftest_wait_timeout(10, NULL) == I
     v = ctypes.c_int32(0)
     assert lib.bi_get_device_status(NULL, None) == I
@@ -108,6 +96,15 @@ def test_binding_refuses_cpu_tensors():
         binding.bi_matmul(a, a, "nk")
     with pytest.raises(ValueError):
         binding.bi_mean(a.float())
+
+
+def test_binding_refuses_a_tensor_or_stream_off_the_current_device(monkeypatch):
+    """The C ABI runs on the current device; a tensor or stream of another device is refused in
+    the binding before anything is launched."""
+    monkeypatch.setattr(binding, "_current_device", lambda: 1)
+    binding._same_device(1, "x")
+    with pytest.raises(ValueError, match="current device is cuda:1"):
+        binding._same_device(0, "x")
 
 
 def test_missing_library_fails_loudly(tmp_path):

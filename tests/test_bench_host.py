@@ -29,7 +29,7 @@ def test_traffic_record_is_used_only_for_its_source_case_and_rows(tmp_path, monk
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(path))
     assert bench.measured_traffic(1024, "gemm_lm_head") == 123456789
     assert bench.measured_traffic(2048, "gemm_lm_head") is None
-    assert bench.measured_traffic(1024, "gemm_lm_head_lse") is None
+    assert bench.measured_traffic(1024, "gemm_qo_m256") is None
     rec["gemm_source_sha"] = "0" * 16  # captured on another kernel source
     path.write_text(json.dumps(rec))
     assert bench.measured_traffic(1024, "gemm_lm_head") is None

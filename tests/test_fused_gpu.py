@@ -70,6 +70,15 @@ def test_fused_batch_invariance(layout):
             assert same_bits(bi.bi_matmul_silu_mul(pool[idx], w, layout), ref[idx]), f"M={M}"
 
 
+def test_fused_repeatable_100_runs():
+    M, F, K = 2048, 12288, 4096
+    a = inputs.rows_normal(409, 0, M, K).to(DEV)
+    w = gate_up(416, F, K, "nk").to(DEV)
+    first = bi.bi_matmul_silu_mul(a, w)
+    for _ in range(100):
+        assert same_bits(bi.bi_matmul_silu_mul(a, w), first)
+
+
 def test_fused_k0_and_empty():
     a0 = torch.empty(5, 0, dtype=torch.bfloat16, device=DEV)
     w0 = torch.empty(16, 0, dtype=torch.bfloat16, device=DEV)

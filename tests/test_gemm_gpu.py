@@ -204,6 +204,53 @@ def test_batch_invariance_sweep(name, layout):
             assert same_bits(out, ref[idx]), f"{name} {layout} M={M}: a row differs from M=1"
 
 
+@pytest.mark.parametrize("K,N", [(4096, 12288), (4096, 24576), (12288, 4096)])
+def test_batch_invariance_sweep_wide_and_deep(K, N):
+    """gate/up (N = 12288, and the fused [gate; up] N = 24576) and down (K = 12288) over the
+    whole M sweep up to 2048: every row of every batch, at every position of three windows of
+    a random permutation of the pool, equals the same row computed alone, bit for bit."""
+    pool = inputs.rows_normal(238, 0, 2048, K).to(DEV)
+    w = weight(239, N, K, "nk").to(DEV)
+    ref = torch.empty(2048, N, dtype=torch.bfloat16, device=DEV)
+    for i in range(2048):
+        bi.bi_matmul(pool[i:i + 1], w, "nk", out=ref[i:i + 1])
+    perm = inputs.permutation(240, 2048).to(DEV)
+    for M in M_SWEEP:
+        for start in (0, 2048 - M, (2048 - M) // 2):
+            idx = perm[start:start + M]
+            out = bi.bi_matmul(pool[idx], w, "nk")
+            assert same_bits(out, ref[idx]), f"K={K} N={N} M={M}: a row differs from M=1"
+
+
+def test_lm_head_logits_invariance():
+    """LM-head logits [M, 151936] at M in {1, 8, 64, 256, 1024}: each row equals the row
+    computed alone, bit for bit, at every position of two windows of a permutation."""
+    K, N, P = 4096, 151936, 1024
+    pool = inputs.rows_normal(241, 0, P, K).to(DEV)
+    w = weight(242, N, K, "nk").to(DEV)
+    ref = torch.empty(P, N, dtype=torch.bfloat16, device=DEV)
+    for i in range(P):
+        bi.bi_matmul(pool[i:i + 1], w, "nk", out=ref[i:i + 1])
+    perm = inputs.permutation(243, P).to(DEV)
+    for M in (1, 8, 64, 256, 1024):
+        for start in (0, P - M):
+            idx = perm[start:start + M]
+            assert same_bits(bi.bi_matmul(pool[idx], w, "nk"), ref[idx]), f"LM head M={M}"
+
+
+def test_addmm_repeatable_100_runs():
+    K, N, M = 4096, 4096, 2048
+    a = inputs.rows_normal(244, 0, M, K).to(DEV)
+    w = weight(245, N, K, "nk").to(DEV)
+    bias = inputs.bias(246, N).to(DEV)
+    resid = inputs.rows_normal(247, 0, M, N).to(DEV)
+    first_b = bi.bi_addmm(bias, a, w)
+    first_r = bi.bi_addmm(resid, a, w)
+    for _ in range(100):
+        assert same_bits(bi.bi_addmm(bias, a, w), first_b)
+        assert same_bits(bi.bi_addmm(resid, a, w), first_r)
+
+
 def test_addmm_residual_invariance_positions():
     K, N = 12288, 4096
     pool = inputs.rows_normal(233, 0, 512, K).to(DEV)

@@ -360,72 +360,3 @@ def test_empty_batches():
     assert oracle.matmul(np.zeros((0, 8), np.uint16), np.zeros((8, 4), np.uint16), "kn").shape == (0, 4)
     assert oracle.mean(np.zeros((0, 8), np.float32)).shape == (0,)
     assert oracle.log_softmax(np.zeros((0, 8), np.float32)).shape == (0, 8)
-
-
-# ----------------------------------------------------------------------------- per-tile (max, sum exp)
-
-def test_tile_stats_constant_row_counts():
-    """Constant rows: every tile's max is the constant and its sum is its column count."""
-    for V, tile in ((1000, 256), (256, 256), (257, 256), (151936, 256), (5, 2)):
-        for c in (0.0, -3.5, 7.0):
-            x = bits(torch.full((2, V), c, dtype=torch.bfloat16))
-            m, s = oracle.tile_max_sumexp(x, tile)
-            counts = [min(tile, V - t * tile) for t in range(-(-V // tile))]
-            assert np.array_equal(m, np.full((2, len(counts)), c))
-            assert np.array_equal(s, np.array([counts, counts], dtype=np.float64))
-
-
-def test_tile_stats_planted_maxima_closed_form():
-    """Row of -1 with one entry t + 1 planted at a different offset in each tile t: the max of
-    tile t is t + 1 and its sum is 1 + (n_t - 1) e^(-(t + 2)); a wrong tile index or boundary
-    moves a planted maximum into the wrong tile."""
-    V, tile = 1000, 256
-    row = torch.full((V,), -1.0)
-    P = -(-V // tile)
-    for t in range(P):
-        n_t = min(tile, V - t * tile)
-        row[t * tile + (37 * t + 5) % n_t] = t + 1
-    m, s = oracle.tile_max_sumexp(bits(row.to(torch.bfloat16)[None]), tile)
-    for t in range(P):
-        n_t = min(tile, V - t * tile)
-        assert m[0, t] == t + 1
-        assert abs(s[0, t] - (1 + (n_t - 1) * math.exp(-(t + 2)))) <= 1e-15 * n_t
-
-
-def test_tile_stats_underflowing_terms_count_exactly():
-    """Entries 0 and -1000: exp(-1000) underflows to 0 in binary64, so s counts the zeros."""
-    g = torch.Generator().manual_seed(41)
-    mask = torch.rand(3, 777, generator=g) < 0.3
-    x = torch.where(mask, torch.tensor(0.0), torch.tensor(-1000.0)).to(torch.bfloat16)
-    x[:, ::256] = 0.0  # every tile holds at least one zero
-    m, s = oracle.tile_max_sumexp(bits(x), 256)
-    zeros = (x == 0).numpy()
-    for t in range(m.shape[1]):
-        assert np.all(m[:, t] == 0.0)
-        assert np.array_equal(s[:, t], zeros[:, t * 256:(t + 1) * 256].sum(axis=1).astype(np.float64))
-
-
-@pytest.mark.parametrize("V", [1000, 151936])
-def test_tile_stats_merge_to_the_row_log_softmax(V):
-    """The tiles together hold the row's statistics: max_t m_t is the row max, and
-    m + log(sum_t s_t e^(m_t - m)) is the row's log-sum-exp, i.e. x_j - y_j of the
-    (separately pinned) log_softmax in every column."""
-    x = inputs.rows_normal(42, 0, 3, V, std=1.3)
-    xb = bits(x)
-    m, s = oracle.tile_max_sumexp(xb, 256)
-    y = oracle.log_softmax(xb)
-    x64 = x.to(torch.float64).numpy()
-    for i in range(3):
-        mm = m[i].max()
-        assert mm == x64[i].max()
-        lse = mm + math.log(math.fsum(s[i] * np.exp(m[i] - mm)))
-        assert np.max(np.abs((x64[i] - y[i]) - lse)) <= 1e-12 * max(1.0, abs(lse))
-
-
-def test_tile_stats_pin_detects_wrong_tile_boundary():
-    """Planted mistake: tiles that overlap by one column (j1 = j0 + tile + 1) miscount."""
-    V, tile = 1000, 256
-    x = np.zeros((1, V))
-    wrong = [float(np.exp(x[0, t * tile:min(V, t * tile + tile + 1)]).sum()) for t in range(-(-V // tile))]
-    counts = [min(tile, V - t * tile) for t in range(-(-V // tile))]
-    assert wrong != counts

@@ -206,6 +206,29 @@ def test_row_ops_repeatable_100_runs():
         assert same_bits(bi.bi_mean(xf), first_m)
 
 
+def test_log_softmax_repeatable_100_runs():
+    """The streamed kernel of the LM-head step: bulk copies complete on mbarriers, a stage is
+    refilled right after the block has read it, and the second pass reads stages still
+    resident.  A missing fence there would show up as a rare bit flip, so the step's own shape
+    (bf16, M = 1024, V = 151936: 10 ring chunks, the last one partial) runs 100 times, and an
+    fp32 row length whose last chunk holds 8 elements (98312 = 12 x 8192 + 8) as well."""
+    x = inputs.rows_normal(152, 0, 1024, 151936, std=1.3).to(DEV)
+    first = bi.bi_log_softmax(x)
+    for _ in range(100):
+        assert same_bits(bi.bi_log_softmax(x), first)
+    xf = inputs.rows_normal(153, 0, 64, 98312, dtype=torch.float32).to(DEV)
+    first = bi.bi_log_softmax(xf)
+    for _ in range(100):
+        assert same_bits(bi.bi_log_softmax(xf), first)
+
+
+def test_silu_mul_repeatable_100_runs():
+    gu = inputs.rows_normal(154, 0, 512, 2 * 12288, std=2.0).to(DEV)
+    first = bi.bi_silu_mul(gu)
+    for _ in range(100):
+        assert same_bits(bi.bi_silu_mul(gu), first)
+
+
 # ----------------------------------------------------------------------------- edge cases
 
 def test_empty_batch_is_noop():

@@ -38,6 +38,7 @@ def reference(x):
 @pytest.mark.parametrize("first,second", [
     ((5, 151936, torch.bfloat16), (33, 4096, torch.float32)),
     ((1724, 151936, torch.bfloat16), (2, 1000, torch.bfloat16)),
+    ((2, 1000, torch.bfloat16), (1724, 151936, torch.bfloat16)),  # the second call writes more partials
 ])
 def test_noalloc_matches_scratch_entry_point_on_two_calls(first, second):
     for seed, (M, V, dt) in enumerate((first, second)):
@@ -48,6 +49,18 @@ def test_noalloc_matches_scratch_entry_point_on_two_calls(first, second):
         torch.cuda.synchronize()
         assert float((y - ref).abs().max()) <= LSM_ABS
         assert same_bits(y, ref)
+
+
+def test_noalloc_python_wrapper():
+    """The binding's wrapper passes its arguments in the C function's order and checks the
+    output's shape before it calls anything."""
+    x = inputs.rows_normal(610, 0, 9, 151936, std=1.3).to(DEV)
+    y = torch.empty(9, 151936, dtype=torch.float32, device=DEV)
+    for _ in range(2):
+        assert bi.bi_log_softmax_split_noalloc(x, y) is y
+        assert same_bits(y, reference(x))
+    with pytest.raises(ValueError):
+        bi.bi_log_softmax_split_noalloc(x, torch.empty(9, 151928, dtype=torch.float32, device=DEV))
 
 
 def test_noalloc_refuses_sizes_beyond_its_array():
