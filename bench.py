@@ -445,6 +445,8 @@ def run_bi(args):
     row_gbs = {op: round(b * M / (per_op[op] / 1e3) / 1e9, 1) for op, b in row_bytes.items()
                if op in per_op}
 
+    # The per-kernel M sweep runs after every timed region, on this GPU alone (N = 1).
+    sweep = metric_sweep(device, peaks) if world == 1 and not args.no_metric_sweep else None
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -488,6 +490,7 @@ def run_bi(args):
             "gpu_launches": len(OPS) * args.steps,
             "clocks": clocks,
             "device_status": status,
+            "metric_sweep": sweep,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -559,6 +562,142 @@ def _rows_differing(t, ref1):
     n = ref1.shape[0]
     view = torch.int16 if t.element_size() == 2 else torch.int32
     return int((t[:n].contiguous().view(view) != ref1.contiguous().view(view)).any(dim=1).sum())
+
+
+# ----------------------------------------------------------------------------- metric sweep (in the JSON line)
+
+SWEEP_GEMMS = [("q/o", HIDDEN, HIDDEN), ("k/v", HIDDEN, KV), ("gate/up", HIDDEN, FFN), ("down", FFN, HIDDEN),
+               ("lm_head", HIDDEN, VOCAB)]
+SWEEP_M = [1, 64, 256, 1024, 2048]
+SWEEP_ROW_OPS = [("rmsnorm", HIDDEN, (1024, 16384)), ("mean", HIDDEN, (1024, 16384)),
+                 ("log_softmax", VOCAB, (1, 64, 1024))]
+
+
+def roofline_point(flop: float, nbytes: float, us: float, peaks: dict) -> dict:
+    """Fraction of the roofline for one launch: the roofline time is the larger of the FLOPs at the
+    tensor peak and the algorithmic bytes at the HBM peak; `bound` names the larger term."""
+    t_tensor = flop / (peaks["bf16_tflops"] * 1e12) if flop else 0.0
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_roof = max(t_tensor, t_hbm)
+    return {"bound": "tensor" if t_tensor >= t_hbm else "hbm", "roofline_frac": round(t_roof / (us * 1e-6), 3)}
+
+
+def metric_sweep(device, peaks: dict, reps: int = 10) -> dict:
+    """The metric's M sweep, per kernel, on synthetic inputs shaped like the workload: each bi
+    kernel and torch's default kernel for the same op, timed alone (median of `reps` launches, a
+    256 MB write before each to flush L2); TFLOP/s, algorithmic GB/s and the fraction of the
+    roofline, and how many of the first 8 rows differ bit-wise from the same rows computed
+    alone (M = 1)."""
+    import torch
+    import torch.nn.functional as F
+    from invariant_bi_matmul_02_b200 import binding as bi
+    g = torch.Generator(device=device)
+    g.manual_seed(7)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    counter = [0]
+
+    def flush():
+        counter[0] += 1
+        flush_buf.fill_(counter[0] & 0xFF)
+
+    def us(fn):
+        fn()
+        return _timed(fn, flush, reps) * 1e3
+
+    out = {"protocol": f"median of {reps} launches, 256 MB written before each (L2 flushed); inputs "
+                       "N(0,1), weights N(0,0.02) [N,K]; peaks: burst", "gemm": [], "row_ops": []}
+    for name, K, N in SWEEP_GEMMS:
+        w = (torch.randn(N, K, generator=g, device=device) * 0.02).to(torch.bfloat16)
+        a = torch.randn(max(SWEEP_M), K, generator=g, device=device).to(torch.bfloat16)
+        ref = torch.cat([bi.bi_matmul(a[i:i + 1], w) for i in range(8)])
+        tref = torch.cat([F.linear(a[i:i + 1], w) for i in range(8)])
+        for M in SWEEP_M:
+            am = a[:M]
+            c = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+            t_bi = us(lambda: bi.bi_matmul(am, w, out=c))
+            t_t = us(lambda: F.linear(am, w))
+            n = min(M, 8)
+            flop, nbytes = 2.0 * M * N * K, float(gemm_bytes(M, K, N))
+            out["gemm"].append({"shape": name, "M": M, "K": K, "N": N, "bi_us": round(t_bi, 1),
+                                "tflops": round(flop / t_bi / 1e6, 1), "gbs": round(nbytes / t_bi / 1e3, 1),
+                                **roofline_point(flop, nbytes, t_bi, peaks), "torch_us": round(t_t, 1),
+                                "rows_differing_from_m1": _rows_differing(c, ref[:n]),
+                                "torch_rows_differing_from_m1": _rows_differing(F.linear(am, w), tref[:n])})
+        del w, a, ref, tref
+    for op, H, ms in SWEEP_ROW_OPS:
+        Mmax = max(ms)
+        if op == "rmsnorm":
+            x = torch.randn(Mmax, H, generator=g, device=device).to(torch.bfloat16)
+            wn = (1 + 0.1 * torch.randn(H, generator=g, device=device)).to(torch.bfloat16)
+            fb = lambda xm, y: bi.bi_rmsnorm(xm, wn, EPS, out=y)
+            ft = lambda xm: F.rms_norm(xm, (H,), wn, EPS)
+            y_of = lambda M: torch.empty(M, H, dtype=torch.bfloat16, device=device)
+            per_row = 4 * H
+        elif op == "mean":
+            x = torch.randn(Mmax, H, generator=g, device=device)
+            fb = lambda xm, y: bi.bi_mean(xm, out=y)
+            ft = lambda xm: xm.mean(-1)
+            y_of = lambda M: torch.empty(M, dtype=torch.float32, device=device)
+            per_row = 4 * H + 4
+        else:
+            x = (1.3 * torch.randn(Mmax, H, generator=g, device=device)).to(torch.bfloat16)
+            fb = lambda xm, y: bi.bi_log_softmax(xm, out=y)
+            ft = lambda xm: torch.log_softmax(xm, -1, dtype=torch.float32)
+            y_of = lambda M: torch.empty(M, H, dtype=torch.float32, device=device)
+            per_row = 6 * H
+        ref = torch.cat([fb(x[i:i + 1], y_of(1)).reshape(1, -1) for i in range(8)])
+        tref = torch.cat([ft(x[i:i + 1]).reshape(1, -1) for i in range(8)])
+        for M in ms:
+            xm, y = x[:M], y_of(M)
+            t_bi = us(lambda: fb(xm, y))
+            t_t = us(lambda: ft(xm))
+            n = min(M, 8)
+            nbytes = float(per_row * M)
+            out["row_ops"].append({"op": op, "M": M, "H": H, "bi_us": round(t_bi, 1),
+                                   "gbs": round(nbytes / t_bi / 1e3, 1),
+                                   "hbm_frac": round(nbytes / t_bi / 1e3 / peaks["hbm_gbs"], 3),
+                                   "torch_us": round(t_t, 1),
+                                   "rows_differing_from_m1": _rows_differing(y.reshape(M, -1), ref[:n]),
+                                   "torch_rows_differing_from_m1": _rows_differing(ft(xm).reshape(M, -1),
+                                                                                   tref[:n])})
+        del x, ref, tref
+    del flush_buf
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_host_overhead(args):
+    """Host time per bi_matmul call at M = 1 (K = N = 256) through the binding, with the tensor-map
+    cache hitting (the same buffers every call) and missing (a new activation address each call,
+    so one of the two maps is encoded), and the device time of the same launch for scale."""
+    import torch
+    from invariant_bi_matmul_02_b200 import binding as bi
+    dev = torch.device("cuda", 0)
+    K = N = 256
+    w = torch.randn(N, K, device=dev).to(torch.bfloat16)
+    pool = torch.randn(4096, K, device=dev).to(torch.bfloat16)  # 4096 distinct row addresses
+    c = torch.empty(1, N, dtype=torch.bfloat16, device=dev)
+    calls = 4000
+
+    def host_us(rows):
+        for i in range(50):
+            bi.bi_matmul(rows(i), w, out=c)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for i in range(calls):
+            bi.bi_matmul(rows(i), w, out=c)
+        t = (time.perf_counter() - t0) / calls * 1e6
+        torch.cuda.synchronize()
+        return t
+
+    h0, m0 = bi.bi_tensor_map_cache_stats()
+    hit = host_us(lambda i: pool[:1])
+    h1, m1 = bi.bi_tensor_map_cache_stats()
+    miss = host_us(lambda i: pool[(i * 7) % 4096:(i * 7) % 4096 + 1])
+    h2, m2 = bi.bi_tensor_map_cache_stats()
+    print(json.dumps({"host_overhead": "bi_matmul M=1 K=N=256 through the binding",
+                      "host_us_per_call_cache_hit": round(hit, 2), "host_us_per_call_one_miss": round(miss, 2),
+                      "hits_misses_hit_loop": [h1 - h0, m1 - m0], "hits_misses_miss_loop": [h2 - h1, m2 - m1]}))
 
 
 def run_sweep(args):
@@ -1001,6 +1140,10 @@ def main():
                     help="gate/up + SiLU*up as one fused GEMM (default) or GEMM then bi_silu_mul")
     ap.add_argument("--cpu-budget", type=float, default=25.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--host-overhead", action="store_true",
+                    help="host time per small GEMM call with and without tensor-map cache hits")
+    ap.add_argument("--no-metric-sweep", action="store_true",
+                    help="leave out the per-kernel M sweep that the JSON line carries at N=1")
     ap.add_argument("--sweep", action="store_true", help="per-kernel M sweeps (table, not JSON line)")
     ap.add_argument("--sweep-shapes", default="",
                     help="comma list of sweep groups (q/o,k/v,gate/up,down,lm_head,rows; attention only when named)")
@@ -1020,6 +1163,9 @@ def main():
         return
     if args.kernel_case:
         run_kernel_case(args)
+        return
+    if args.host_overhead:
+        run_host_overhead(args)
         return
     if args.uniqueness:
         run_uniqueness(args)

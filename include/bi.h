@@ -313,6 +313,15 @@ const char *bi_status_string(bi_status status);
  */
 void bi_gemm_config(int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int32_t *mma_k);
 
+/*
+ * bi_tensor_map_cache_stats -- how many TMA tensor-map look-ups of the GEMM entry points were
+ * served from the library's cache (*hits) and how many had to be encoded (*misses) since the
+ * library was loaded.  A GEMM call looks up two maps (weights and activations), keyed by
+ * (base address, extents, row stride, box); a repeated call with the same buffers hits twice.
+ * Either pointer may be NULL.
+ */
+void bi_tensor_map_cache_stats(int64_t *hits, int64_t *misses);
+
 /* Library version as major*10000 + minor*100 + patch. */
 int32_t bi_version(void);
 

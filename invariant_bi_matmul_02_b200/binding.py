@@ -45,6 +45,7 @@ SIGNATURES = {
     "bi_selftest_wait_timeout": (ctypes.c_int, [_i64, _p]),
     "bi_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bi_gemm_config": (None, [ctypes.POINTER(_i32)] * 5),
+    "bi_tensor_map_cache_stats": (None, [ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
     "bi_version": (ctypes.c_int32, []),
 }
 
@@ -386,6 +387,13 @@ def bi_gemm_config() -> dict:
     vals = [_i32(0) for _ in range(5)]
     load().bi_gemm_config(*[ctypes.byref(v) for v in vals])
     return dict(zip(("bm", "bn", "bk", "stages", "mma_k"), (int(v.value) for v in vals)))
+
+
+def bi_tensor_map_cache_stats() -> tuple[int, int]:
+    """(hits, misses) of the library's TMA tensor-map cache since it was loaded."""
+    h, m = _i64(0), _i64(0)
+    load().bi_tensor_map_cache_stats(ctypes.byref(h), ctypes.byref(m))
+    return int(h.value), int(m.value)
 
 
 def bi_version() -> int:

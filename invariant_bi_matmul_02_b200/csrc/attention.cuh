@@ -1,18 +1,27 @@
 // attention.cuh -- batch-invariant decode attention (one query token per sequence).
 //
 // The key/value cache of a sequence is cut into splits of kAttnSplit tokens, a cut fixed
-// by the sequence's own length.  Launch 1 gives every (split, kv head, sequence) one block,
-// which produces, for each query head of the kv head's group, the split's maximum score,
-// its sum of exp(score - max) and the matching weighted sum of value rows.  Launch 2
-// folds the splits of each (sequence, query head) in ascending split order.  Every
-// reduction is a fixed sequence or a fixed tree, so a sequence's output depends on its own
-// query, cache and length only -- not on the batch it is decoded in or its position there.
+// by the sequence's own length.  Launch 1 produces, for every (split, kv head, sequence) and
+// each query head of the kv head's group, the split's maximum score, its sum of
+// exp(score - max) and the matching weighted sum of value rows.  Launch 2 folds the splits of
+// each (sequence, query head) in ascending split order.  Every reduction is a fixed sequence
+// or a fixed tree, so a sequence's output depends on its own query, cache and length only --
+// not on the batch it is decoded in, its position there, or which CTA computes a split.
+//
+// Launch 1 is a persistent, warp-specialised kernel: one CTA per SM walks the (split, kv head,
+// sequence) work items round-robin.  Its producer warp stages each item's query rows (bulk
+// copies) and its K and V tiles (4-D TMA tensor loads, 128-byte swizzle) into a ring of
+// kAttnStages shared-memory stages, each completing on mbarriers.  Two groups of four consumer
+// warps take the CTA's items alternately, so one group's compute overlaps the other's and the
+// loads of the next items.  The cache streams from HBM without a gap between items.  The
+// arithmetic of an item is fixed and does not depend on the ring, the group or the CTA.
 //
 // Layouts (row-major, bf16): q [B, Hq, D]; k, v [B, Lmax, Hkv, D]; out [B, Hq, D].  Query
 // head h reads kv head h / (Hq / Hkv).  D = 128.
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 
 #include "rowops.cuh"
@@ -20,21 +29,32 @@
 namespace bi {
 
 constexpr int kAttnD = 128;
-constexpr int kAttnSplit = 128;       // tokens per split (one per thread in the score phase)
-constexpr int kAttnThreads = 128;
-constexpr int kAttnMaxGroup = 8;      // query heads per kv head
-constexpr int kAttnStride = kAttnD + 8;  // padded row (bf16): conflict-free ldmatrix rows
-constexpr int kAttnWarps = kAttnThreads / 32;
+constexpr int kAttnSplit = 128;                         // tokens per split
+constexpr int kAttnConsumers = 4;                       // consumer warps per group, 32 tokens each
+constexpr int kAttnGroups = 2;                          // consumer groups, alternate items
+constexpr int kAttnThreads = 32 * (1 + kAttnGroups * kAttnConsumers);  // warp 0 produces
+constexpr int kAttnMaxGroup = 8;                        // query heads per kv head
+constexpr int kAttnStages = 3;
+constexpr int kAttnQStride = kAttnD + 8;                // padded query row (bf16): conflict-free ldmatrix
+constexpr int kAttnBoxBytes = kAttnSplit * 64 * 2;      // one TMA box: 128 tokens x 64 d (16 KB)
+constexpr int kAttnTileBytes = 2 * kAttnBoxBytes;       // K or V of one split: 32 KB
+constexpr int kAttnQBytes = 16 * kAttnQStride * 2;      // query rows of a group, padded to 16 rows
+constexpr int kAttnStageBytes = 2 * kAttnTileBytes + ((kAttnQBytes + 1023) / 1024) * 1024;
+constexpr int kAttnSmem = kAttnStages * kAttnStageBytes + 1024;  // + alignment slack
 
-struct AttnSmem {
-    __nv_bfloat16 q[16][kAttnStride];           // the group's query heads, rows >= G zero
-    union {
-        __nv_bfloat16 k[kAttnSplit][kAttnStride];
-        float o[kAttnWarps][kAttnMaxGroup][kAttnD];  // per-warp partial outputs, after the scores
-    } ko;
-    __nv_bfloat16 v[kAttnSplit][kAttnStride];
-    float red[kAttnWarps][16];
-    float stat[16][2];
+static_assert(kAttnConsumers * kAttnMaxGroup * kAttnD * 4 <= kAttnTileBytes,
+              "per-warp partial outputs fit in the K tile they replace");
+
+struct AttnParams {
+    const __nv_bfloat16 *q;
+    const int32_t *lens;
+    float2 *part_ms;  // [B, Hq, S] (max, sum)
+    float *part_acc;  // [B, Hq, S, D]
+    int32_t Hq, Hkv, B;
+    int64_t Lmax, S;  // S = splits of Lmax
+    float scale;
+    int32_t *status;
+    uint64_t wait_limit_ns;
 };
 
 __host__ __device__ inline int64_t attn_splits(int64_t L) { return (L + kAttnSplit - 1) / kAttnSplit; }
@@ -45,198 +65,344 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&p);
 }
 
-// Launch 1: grid (ceil(Lmax / kAttnSplit), Hkv, B), kAttnThreads threads, sizeof(AttnSmem)
-// bytes of dynamic shared memory.  part_ms: [B, Hq, S] float2 (max, sum); part_acc:
-// [B, Hq, S, D] float, S = ceil(Lmax / kAttnSplit).
-//
-// Tensor-core form (mma.sync m16n8k16, bf16 in, fp32 accumulate).  Warp w owns tokens
-// 32w .. 32w+31 of the split.  Scores: S = Q . K^T with Q the group's heads padded to 16 rows;
-// every score accumulates its eight 16-wide D steps in ascending order.  Then, per head, the
-// split's maximum and sum of exp(s - max) (fp32) come from fixed trees: a thread's own values
-// in order, the lane quad (xor 1, 2), the warps in order.  Weighted sums: O_w = P_w . V_w with
-// P split into two bf16 terms (about 16 significant bits), two 16-token steps in ascending
-// order; the four warps' O_w are added in warp order.
-template <int G>  // query heads per kv head (1, 2, 4 or 8)
-__global__ void __launch_bounds__(kAttnThreads, 3)
-    decode_attention_split_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                                  const __nv_bfloat16 *__restrict__ v, const int32_t *__restrict__ lens,
-                                  float2 *__restrict__ part_ms, float *__restrict__ part_acc, int Hq, int Hkv,
-                                  int64_t Lmax, float scale, int32_t *status)
+// Shared-memory address of 16-byte chunk `chunk` (0..15) of token row `row` of a K or V tile as
+// the TMA writes it: two boxes of 64 d each (chunks 0..7 and 8..15), rows of 128 bytes, with the
+// 128-byte swizzle (chunk c of row r lands at chunk c ^ (r mod 8)).
+__device__ __forceinline__ const uint8_t *kv_chunk(const uint8_t *tile, int row, int chunk)
 {
-    extern __shared__ __align__(16) uint8_t attn_raw[];
-    AttnSmem &sm = *reinterpret_cast<AttnSmem *>(attn_raw);
+    return tile + (chunk >> 3) * kAttnBoxBytes + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
+}
+
+// Sequence length as the kernels use it: a value outside 1 .. Lmax is clamped (and reported).
+__device__ __forceinline__ int64_t attn_len(const AttnParams &p, int b, bool report)
+{
+    int64_t L = p.lens[b];
+    if (L < 1 || L > p.Lmax) {
+        if (report) *reinterpret_cast<volatile int32_t *>(p.status) = 1;  // BI_ERR_INVALID_ARG
+        L = L < 1 ? 1 : p.Lmax;
+    }
+    return L;
+}
+
+// 4-D tiled TMA load (coordinates innermost first), completion on `bar`.
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, uint64_t *bar, int32_t c0,
+                                            int32_t c1, int32_t c2, int32_t c3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
+// All threads of one consumer group (named barrier `id`, 128 threads): true iff every one passes
+// `ok`.
+__device__ __forceinline__ bool consumers_all(int id, bool ok)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %2, 0;\n\t"
+        "barrier.red.and.pred q, %1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(id), "r"(ok ? 1u : 0u)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void consumers_sync(int id) { asm volatile("barrier.sync %0, 128;" ::"r"(id) : "memory"); }
+
+// Bounded wait until *flag >= v (a shared-memory progress counter written by another warp).
+// On time-out it records BI_ERR_TIMEOUT and raises the abort flag, like wait_bounded.
+__device__ __forceinline__ bool wait_flag_at_least(volatile int *flag, int v, volatile int *abort_flag,
+                                                   int32_t *status, uint64_t limit_ns)
+{
+    if (*flag >= v) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (*flag >= v) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+            *reinterpret_cast<volatile int32_t *>(status) = 5;  // BI_ERR_TIMEOUT
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+// Launch 1: grid = min(work items, SMs) CTAs of kAttnThreads threads, kAttnSmem bytes of dynamic
+// shared memory.  Work item i: split i % S, kv head (i / S) % Hkv, sequence i / (S Hkv); items
+// past their sequence's length have no partial and are skipped by every role alike.
+//
+// Arithmetic per item (mma.sync m16n8k16, bf16 in, fp32 accumulate; warp w owns tokens
+// 32w .. 32w+31 of the split).  Scores: S = Q . K^T with Q the group's heads padded to 16 rows;
+// every score accumulates its eight 16-wide D steps in ascending order.  Per head, the split's
+// maximum and sum of exp(s - max) (fp32) come from fixed trees: a thread's own values in
+// order, the lane quad (xor 1, 2), the warps in order.  Weighted sums: O_w = P_w . V_w with P
+// split into two bf16 terms (about 16 significant bits), two 16-token steps in ascending order;
+// the four warps' O_w are added in warp order.  Value rows past the sequence's end are zeroed in
+// shared memory before use, so stale cache contents never reach the sums.
+template <int G>  // query heads per kv head (1, 2, 4 or 8)
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    decode_attention_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                                  const AttnParams p)
+{
+    extern __shared__ uint8_t attn_raw[];
+    uint8_t *smem = attn_raw + ((1024u - (smem_addr(attn_raw) & 1023u)) & 1023u);
+    __shared__ uint64_t kfull[kAttnStages], vfull[kAttnStages], empty[kAttnStages];
+    __shared__ float red_all[kAttnGroups][kAttnConsumers][16];
+    __shared__ float stat_all[kAttnGroups][16][2];
+    __shared__ int abort_flag_s;
+    __shared__ int progress_s[kAttnGroups];  // items a consumer group has started (local index + 1)
+    volatile int *abort_flag = &abort_flag_s;
+    volatile int *progress = progress_s;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto k_tile = [&](int s) { return smem + s * kAttnStageBytes; };
+    auto v_tile = [&](int s) { return smem + s * kAttnStageBytes + kAttnTileBytes; };
+    auto q_rows = [&](int s) { return reinterpret_cast<__nv_bfloat16 *>(smem + s * kAttnStageBytes + 2 * kAttnTileBytes); };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kAttnStages; ++s) {
+            mbar_init(&kfull[s], 1);
+            mbar_init(&vfull[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        abort_flag_s = 0;
+        for (int g = 0; g < kAttnGroups; ++g) progress_s[g] = 0;
+        fence_mbar_init();
+    }
+    // Query rows G .. 15 of every stage stay zero (the copies fill rows 0 .. G-1 only).
+    for (int i = threadIdx.x; i < kAttnStages * (16 - G) * kAttnQStride / 2; i += kAttnThreads) {
+        const int s = i / ((16 - G) * kAttnQStride / 2), r = i % ((16 - G) * kAttnQStride / 2);
+        reinterpret_cast<uint32_t *>(q_rows(s) + G * kAttnQStride)[r] = 0u;
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
     griddep_wait();  // the previous kernel's output (q, the caches, the lengths) is complete
     griddep_launch_dependents();
-    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gid = lane >> 2, tig = lane & 3;
-    const int64_t S = attn_splits(Lmax);
-    int64_t L = lens[b];
-    if (L < 1 || L > Lmax) {
-        if (tid == 0) *reinterpret_cast<volatile int32_t *>(status) = 1;  // BI_ERR_INVALID_ARG
-        L = L < 1 ? 1 : Lmax;
-    }
-    const int64_t t0 = (int64_t)split * kAttnSplit;
-    if (t0 >= L) return;  // this split is past the sequence's end: it has no partial
-    const int n_tok = (int)(L - t0 < kAttnSplit ? L - t0 : kAttnSplit);
 
-    // Stage Q (rows >= G zero) and K in copy group 1, V in copy group 2 (16-byte async
-    // copies; rows past the sequence zero-filled).  The scores wait for group 1 only.
-    for (int c = tid; c < 16 * (kAttnD / 8); c += kAttnThreads) {
-        const int j = c / (kAttnD / 8), col = (c % (kAttnD / 8)) * 8;
-        const bool in = j < G;
-        cp_async16(&sm.q[j][col], q + (in ? ((int64_t)b * Hq + (int64_t)g * G + j) * kAttnD + col : 0),
-                   in ? 16u : 0u);
-    }
-    for (int c = tid; c < kAttnSplit * (kAttnD / 8); c += kAttnThreads) {
-        const int row = c / (kAttnD / 8), col = (c % (kAttnD / 8)) * 8;
-        const bool in = row < n_tok;
-        const int64_t off = in ? (((int64_t)b * Lmax + t0 + row) * Hkv + g) * kAttnD + col : 0;
-        cp_async16(&sm.ko.k[row][col], k + off, in ? 16u : 0u);
-    }
-    cp_async_commit();
-    for (int c = tid; c < kAttnSplit * (kAttnD / 8); c += kAttnThreads) {
-        const int row = c / (kAttnD / 8), col = (c % (kAttnD / 8)) * 8;
-        const bool in = row < n_tok;
-        const int64_t off = in ? (((int64_t)b * Lmax + t0 + row) * Hkv + g) * kAttnD + col : 0;
-        cp_async16(&sm.v[row][col], v + off, in ? 16u : 0u);
-    }
-    cp_async_commit();
-    cp_async_wait_pending<1>();
-    __syncthreads();
+    const int64_t items = (int64_t)p.B * p.Hkv * p.S;
+    const uint64_t lim = p.wait_limit_ns;
 
-    // ---- scores: acc[nt] is the 16 x 8 tile (heads x tokens 32w + 8nt ..)
-    float acc[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
-#pragma unroll
-    for (int kk = 0; kk < kAttnD / 16; ++kk) {
-        uint32_t af[4];
-        ldsm_x4(af, &sm.q[(lane & 7) + 8 * ((lane >> 3) & 1)][16 * kk + 8 * (lane >> 4)]);
-#pragma unroll
-        for (int nt = 0; nt < 4; nt += 2) {
-            // matrices: (tile nt, d 0-7), (nt, d 8-15), (nt+1, d 0-7), (nt+1, d 8-15) of this step
-            uint32_t bf[4];
-            ldsm_x4(bf, &sm.ko.k[32 * warp + 8 * (nt + (lane >> 4)) + (lane & 7)][16 * kk + 8 * ((lane >> 3) & 1)]);
-            mma_16816_bf16(acc[nt], af, bf[0], bf[1]);
-            mma_16816_bf16(acc[nt + 1], af, bf[2], bf[3]);
-        }
-    }
-    // scale and mask: element (row gid / gid+8, token 32w + 8nt + 2tig + {0,1})
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int tok = 32 * warp + 8 * nt + 2 * tig + (e & 1);
-            acc[nt][e] = tok < n_tok ? acc[nt][e] * scale : kNegInf;
-        }
-
-    // ---- per-head max: own values in order, quad butterfly, warps in order
-    float mx[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        float m = acc[0][2 * h];
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) m = fmaxf(fmaxf(m, acc[nt][2 * h]), acc[nt][2 * h + 1]);
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        mx[h] = m;
-    }
-    if (tig == 0) {
-        sm.red[warp][gid] = mx[0];
-        sm.red[warp][gid + 8] = mx[1];
-    }
-    __syncthreads();
-    if (tid < 16) {
-        float m = sm.red[0][tid];
-        for (int w = 1; w < kAttnWarps; ++w) m = fmaxf(m, sm.red[w][tid]);
-        sm.stat[tid][0] = m;
-    }
-    __syncthreads();
-    // ---- p = exp(s - max); per-head sums by the same trees
-    float sum[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const float m = sm.stat[gid + 8 * h][0];
-        float l = 0.0f;
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float &x = acc[nt][2 * h + e];
-                x = x == kNegInf ? 0.0f : __expf(x - m);
-                l = __fadd_rn(l, x);
+    if (warp == 0) {
+        // ------------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+                const int split = (int)(it % p.S), g = (int)((it / p.S) % p.Hkv), b = (int)(it / (p.S * p.Hkv));
+                const int64_t t0 = (int64_t)split * kAttnSplit;
+                if (t0 >= attn_len(p, b, false)) continue;
+                if (!(ok = wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim))) break;
+                mbar_arrive_expect_tx(&kfull[stage], G * kAttnD * 2 + kAttnTileBytes);
+                for (int j = 0; j < G; ++j)
+                    bulk_load(q_rows(stage) + j * kAttnQStride, p.q + ((int64_t)b * p.Hq + (int64_t)g * G + j) * kAttnD,
+                              kAttnD * 2, &kfull[stage]);
+                tma_load_4d(k_tile(stage), &tm_k, &kfull[stage], 0, g, (int32_t)t0, b);
+                tma_load_4d(k_tile(stage) + kAttnBoxBytes, &tm_k, &kfull[stage], 64, g, (int32_t)t0, b);
+                mbar_arrive_expect_tx(&vfull[stage], kAttnTileBytes);
+                tma_load_4d(v_tile(stage), &tm_v, &vfull[stage], 0, g, (int32_t)t0, b);
+                tma_load_4d(v_tile(stage) + kAttnBoxBytes, &tm_v, &vfull[stage], 64, g, (int32_t)t0, b);
+                ++issued;
+                advance(stage, phase, kAttnStages);
             }
-        l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 1));
-        l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 2));
-        sum[h] = l;
-    }
-    __syncthreads();  // every warp has read sm.stat / sm.red
-    if (tig == 0) {
-        sm.red[warp][gid] = sum[0];
-        sm.red[warp][gid + 8] = sum[1];
-    }
-    cp_async_wait_pending<0>();  // V has landed
-    __syncthreads();
-    if (tid < 16) {
-        float l = sm.red[0][tid];
-        for (int w = 1; w < kAttnWarps; ++w) l = __fadd_rn(l, sm.red[w][tid]);
-        sm.stat[tid][1] = l;
-    }
+            if (!ok) {
+                // A wait ran out: let every copy already issued land before shared memory goes
+                // away (the last kAttnStages items at most).
+                for (int j = issued > kAttnStages ? issued - kAttnStages : 0; j < issued; ++j) {
+                    const uint32_t par = (uint32_t)(j / kAttnStages) & 1u;
+                    const uint64_t t0 = global_timer_ns();
+                    while ((!mbar_try_wait(smem_addr(&kfull[j % kAttnStages]), par) ||
+                            !mbar_try_wait(smem_addr(&vfull[j % kAttnStages]), par)) &&
+                           global_timer_ns() - t0 < lim) {
+                    }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------ consumers
+        // Group grp takes the CTA's items with local index i = grp, grp + 2, ...; item i sits in
+        // stage i % kAttnStages, that stage's use i / kAttnStages.
+        const int grp = (warp - 1) / kAttnConsumers;
+        const int cw = (warp - 1) % kAttnConsumers, ct = threadIdx.x - 32 - 32 * kAttnConsumers * grp;
+        const int bar_id = 1 + grp;
+        const int gid = lane >> 2, tig = lane & 3;
+        float (*red)[16] = red_all[grp];
+        float (*stat)[2] = stat_all[grp];
+        uint32_t local = 0;
+        for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+            const int split = (int)(it % p.S), g = (int)((it / p.S) % p.Hkv), b = (int)(it / (p.S * p.Hkv));
+            const int64_t t0 = (int64_t)split * kAttnSplit;
+            const int64_t L = attn_len(p, b, ct == 0 && grp == 0 && split == 0);
+            if (t0 >= L) continue;
+            const uint32_t mine = local++;
+            if (mine % kAttnGroups != (uint32_t)grp) continue;
+            const int stage = (int)(mine % kAttnStages);
+            const uint32_t use = mine / kAttnStages;
+            const int n_tok = (int)(L - t0 < kAttnSplit ? L - t0 : kAttnSplit);
+            const uint8_t *ks = k_tile(stage);
+            uint8_t *vs = v_tile(stage);
+            const __nv_bfloat16 *qs = q_rows(stage);
+            // The stage's previous use belongs to the other group.  Once that group has started
+            // this group's preceding item it has finished that previous use, so the stage's
+            // barriers are at most one phase from the one wanted and a parity wait is exact.
+            bool ok = mine == 0 || wait_flag_at_least(&progress[grp ^ 1], (int)mine, abort_flag, p.status, lim);
+            ok = ok && wait_bounded(&kfull[stage], use & 1u, abort_flag, p.status, lim);
+            if (!consumers_all(bar_id, ok)) break;
+            if (ct == 0) progress[grp] = (int)mine + 1;
 
-    // ---- O_w = P_w . V_w: A from the score tiles (two 8-token tiles per 16-token step)
-    float o[kAttnD / 8][4];
+            // ---- scores: acc[nt] is the 16 x 8 tile (heads x tokens 32 cw + 8 nt ..)
+            float acc[4][4];
 #pragma unroll
-    for (int dt = 0; dt < kAttnD / 8; ++dt)
+            for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[dt][e] = 0.0f;
-    // P enters the tensor cores as two bf16 terms, hi = bf16(p) and lo = bf16(p - hi), so the
-    // weights keep about 16 significant bits; per 16-token step the hi product is added first.
+                for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const float *p0 = acc[2 * j], *p1 = acc[2 * j + 1];
-        const float pv[8] = {p0[0], p0[1], p0[2], p0[3], p1[0], p1[1], p1[2], p1[3]};
-        float hi[8], lo[8];
+            for (int kk = 0; kk < kAttnD / 16; ++kk) {
+                uint32_t af[4];
+                ldsm_x4(af, qs + ((lane & 7) + 8 * ((lane >> 3) & 1)) * kAttnQStride + 16 * kk + 8 * (lane >> 4));
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            hi[e] = __bfloat162float(__float2bfloat16_rn(pv[e]));
-            lo[e] = pv[e] - hi[e];
-        }
-        const uint32_t pa_hi[4] = {pack_bf16(hi[0], hi[1]), pack_bf16(hi[2], hi[3]), pack_bf16(hi[4], hi[5]),
-                                   pack_bf16(hi[6], hi[7])};
-        const uint32_t pa_lo[4] = {pack_bf16(lo[0], lo[1]), pack_bf16(lo[2], lo[3]), pack_bf16(lo[4], lo[5]),
-                                   pack_bf16(lo[6], lo[7])};
-        const int tok0 = 32 * warp + 16 * j;
+                for (int nt = 0; nt < 4; nt += 2) {
+                    // matrices: (tile nt, d 0-7), (nt, d 8-15), (nt+1, d 0-7), (nt+1, d 8-15) of this step
+                    uint32_t bf[4];
+                    ldsm_x4(bf, kv_chunk(ks, 32 * cw + 8 * (nt + (lane >> 4)) + (lane & 7), 2 * kk + ((lane >> 3) & 1)));
+                    mma_16816_bf16(acc[nt], af, bf[0], bf[1]);
+                    mma_16816_bf16(acc[nt + 1], af, bf[2], bf[3]);
+                }
+            }
+            // scale and mask: element (row gid / gid+8, token 32 cw + 8 nt + 2 tig + {0,1})
 #pragma unroll
-        for (int dt = 0; dt < kAttnD / 8; dt += 2) {
-            // matrices (transposed): (tokens 0-7, d tile dt), (tokens 8-15, dt), (0-7, dt+1), (8-15, dt+1)
-            uint32_t vf[4];
-            ldsm_x4_trans(vf, &sm.v[tok0 + (lane & 7) + 8 * ((lane >> 3) & 1)][8 * (dt + (lane >> 4))]);
-            mma_16816_bf16(o[dt], pa_hi, vf[0], vf[1]);
-            mma_16816_bf16(o[dt], pa_lo, vf[0], vf[1]);
-            mma_16816_bf16(o[dt + 1], pa_hi, vf[2], vf[3]);
-            mma_16816_bf16(o[dt + 1], pa_lo, vf[2], vf[3]);
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int tok = 32 * cw + 8 * nt + 2 * tig + (e & 1);
+                    acc[nt][e] = tok < n_tok ? acc[nt][e] * p.scale : kNegInf;
+                }
+
+            // ---- per-head max: own values in order, quad butterfly, warps in order
+            float mx[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float m = acc[0][2 * h];
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) m = fmaxf(fmaxf(m, acc[nt][2 * h]), acc[nt][2 * h + 1]);
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+                mx[h] = m;
+            }
+            if (tig == 0) {
+                red[cw][gid] = mx[0];
+                red[cw][gid + 8] = mx[1];
+            }
+            consumers_sync(bar_id);
+            if (ct < 16) {
+                float m = red[0][ct];
+                for (int w = 1; w < kAttnConsumers; ++w) m = fmaxf(m, red[w][ct]);
+                stat[ct][0] = m;
+            }
+            consumers_sync(bar_id);
+            // ---- p = exp(s - max); per-head sums by the same trees
+            float sum[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float m = stat[gid + 8 * h][0];
+                float l = 0.0f;
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float &x = acc[nt][2 * h + e];
+                        x = x == kNegInf ? 0.0f : __expf(x - m);
+                        l = __fadd_rn(l, x);
+                    }
+                l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 1));
+                l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 2));
+                sum[h] = l;
+            }
+            consumers_sync(bar_id);  // every warp has read stat / red
+            if (tig == 0) {
+                red[cw][gid] = sum[0];
+                red[cw][gid + 8] = sum[1];
+            }
+            if (!consumers_all(bar_id, wait_bounded(&vfull[stage], use & 1u, abort_flag, p.status, lim))) break;
+            if (ct < 16) {
+                float l = red[0][ct];
+                for (int w = 1; w < kAttnConsumers; ++w) l = __fadd_rn(l, red[w][ct]);
+                stat[ct][1] = l;
+            }
+            if (n_tok < kAttnSplit) {
+                // Value rows past the sequence's end: zero, whatever the cache holds there.
+                for (int i = ct; i < (kAttnSplit - n_tok) * 16; i += 32 * kAttnConsumers)
+                    *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(kv_chunk(vs, n_tok + i / 16, i % 16))) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                consumers_sync(bar_id);
+            }
+
+            // ---- O_w = P_w . V_w: A from the score tiles (two 8-token tiles per 16-token step)
+            float o[kAttnD / 8][4];
+#pragma unroll
+            for (int dt = 0; dt < kAttnD / 8; ++dt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[dt][e] = 0.0f;
+            // P enters the tensor cores as two bf16 terms, hi = bf16(p) and lo = bf16(p - hi), so
+            // the weights keep about 16 significant bits; per 16-token step hi is added first.
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const float *p0 = acc[2 * j], *p1 = acc[2 * j + 1];
+                const float pv[8] = {p0[0], p0[1], p0[2], p0[3], p1[0], p1[1], p1[2], p1[3]};
+                float hi[8], lo[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    hi[e] = __bfloat162float(__float2bfloat16_rn(pv[e]));
+                    lo[e] = pv[e] - hi[e];
+                }
+                const uint32_t pa_hi[4] = {pack_bf16(hi[0], hi[1]), pack_bf16(hi[2], hi[3]), pack_bf16(hi[4], hi[5]),
+                                           pack_bf16(hi[6], hi[7])};
+                const uint32_t pa_lo[4] = {pack_bf16(lo[0], lo[1]), pack_bf16(lo[2], lo[3]), pack_bf16(lo[4], lo[5]),
+                                           pack_bf16(lo[6], lo[7])};
+                const int tok0 = 32 * cw + 16 * j;
+#pragma unroll
+                for (int dt = 0; dt < kAttnD / 8; dt += 2) {
+                    // matrices (transposed): (tokens 0-7, d tile dt), (8-15, dt), (0-7, dt+1), (8-15, dt+1)
+                    uint32_t vf[4];
+                    ldsm_x4_trans(vf, kv_chunk(vs, tok0 + (lane & 7) + 8 * ((lane >> 3) & 1), dt + (lane >> 4)));
+                    mma_16816_bf16(o[dt], pa_hi, vf[0], vf[1]);
+                    mma_16816_bf16(o[dt], pa_lo, vf[0], vf[1]);
+                    mma_16816_bf16(o[dt + 1], pa_hi, vf[2], vf[3]);
+                    mma_16816_bf16(o[dt + 1], pa_lo, vf[2], vf[3]);
+                }
+            }
+            consumers_sync(bar_id);  // the K tile is no longer read: it holds the per-warp outputs now
+            float *so = reinterpret_cast<float *>(const_cast<uint8_t *>(ks));
+#pragma unroll
+            for (int dt = 0; dt < kAttnD / 8; ++dt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int row = gid + 8 * (e >> 1), col = 8 * dt + 2 * tig + (e & 1);
+                    if (row < G) so[(cw * kAttnMaxGroup + row) * kAttnD + col] = o[dt][e];
+                }
+            consumers_sync(bar_id);
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+                float r = so[j * kAttnD + ct];
+                for (int w = 1; w < kAttnConsumers; ++w) r = __fadd_rn(r, so[(w * kAttnMaxGroup + j) * kAttnD + ct]);
+                const int64_t bh = (int64_t)b * p.Hq + (int64_t)g * G + j;
+                p.part_acc[(bh * p.S + split) * kAttnD + ct] = r;
+                if (ct == 0) p.part_ms[bh * p.S + split] = make_float2(stat[j][0], stat[j][1]);
+            }
+            // Release the stage: the generic-proxy writes above (partial outputs, zeroed rows) are
+            // ordered before the next TMA writes into it.
+            fence_proxy_async_smem();
+            consumers_sync(bar_id);
+            if (ct == 0) mbar_arrive(&empty[stage]);
         }
     }
-    __syncthreads();  // K is no longer read: its space holds the per-warp outputs
-#pragma unroll
-    for (int dt = 0; dt < kAttnD / 8; ++dt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int row = gid + 8 * (e >> 1), col = 8 * dt + 2 * tig + (e & 1);
-            if (row < G) sm.ko.o[warp][row][col] = o[dt][e];
-        }
     __syncthreads();
-#pragma unroll
-    for (int j = 0; j < G; ++j) {
-        float r = sm.ko.o[0][j][tid];
-        for (int w = 1; w < kAttnWarps; ++w) r = __fadd_rn(r, sm.ko.o[w][j][tid]);
-        const int64_t bh = (int64_t)b * Hq + (int64_t)g * G + j;
-        part_acc[(bh * S + split) * kAttnD + tid] = r;
-        if (tid == 0) part_ms[bh * S + split] = make_float2(sm.stat[j][0], sm.stat[j][1]);
-    }
 }
 
 // Launch 2: grid (Hq, B), kAttnD threads.  Fold the sequence's splits in ascending order.

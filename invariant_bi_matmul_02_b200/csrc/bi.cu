@@ -75,14 +75,14 @@ bi_status device_state(DeviceState **out)
                 return BI_ERR_CUDA;
             d.gemm_clusters = n;
         }
-        if (cudaFuncSetAttribute(bi::decode_attention_split_kernel<1>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(bi::AttnSmem)) != cudaSuccess ||
-            cudaFuncSetAttribute(bi::decode_attention_split_kernel<2>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(bi::AttnSmem)) != cudaSuccess ||
-            cudaFuncSetAttribute(bi::decode_attention_split_kernel<4>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(bi::AttnSmem)) != cudaSuccess ||
-            cudaFuncSetAttribute(bi::decode_attention_split_kernel<8>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(bi::AttnSmem)) != cudaSuccess)
+        if (cudaFuncSetAttribute(bi::decode_attention_split_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 bi::kAttnSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(bi::decode_attention_split_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 bi::kAttnSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(bi::decode_attention_split_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 bi::kAttnSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(bi::decode_attention_split_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 bi::kAttnSmem) != cudaSuccess)
             return BI_ERR_CUDA;
         if (cudaFuncSetAttribute(bi::log_softmax_stream_kernel<true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kLsmSmem) != cudaSuccess ||
@@ -189,6 +189,23 @@ bi_status encode_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_
     e.key = key;
     e.map = *map;
     return BI_OK;
+}
+
+// 4-D bf16 tensor map over a decode cache [B, Lmax, Hkv, D] (row-major): dims innermost first
+// (D, Hkv, Lmax, B); box 64 d x 1 head x 128 tokens x 1 sequence, 128-byte swizzle, zero fill
+// past Lmax.
+bi_status encode_kv_map(CUtensorMap *map, const void *base, uint64_t D, uint64_t Hkv, uint64_t Lmax, uint64_t B)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return BI_ERR_CUDA;
+    const cuuint64_t dims[4] = {D, Hkv, Lmax, B};
+    const cuuint64_t strides[3] = {D * 2, Hkv * D * 2, Lmax * Hkv * D * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)bi::kAttnSplit, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? BI_OK : BI_ERR_CUDA;
 }
 
 // Launch `kernel` on `s` and report the launch's own result.  cudaLaunchKernelEx returns the
@@ -311,7 +328,10 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
     if (tiles > kI32Max) return BI_ERR_UNSUPPORTED;
 
     CUtensorMap tm_a, tm_b;
-    st = encode_map(&tm_a, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda, bi::kBK, bi::kBM);
+    // The A box copies the rows that exist: M rounded up to 8, at most the CTA's 128.  The tile,
+    // the MMA shape and every element's K order are the same for every M.
+    p.a_box_rows = (int32_t)(M >= bi::kBM ? bi::kBM : (M + 7) / 8 * 8);
+    st = encode_map(&tm_a, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda, bi::kBK, (uint32_t)p.a_box_rows);
     if (st != BI_OK) return st;
     if (b_layout == BI_B_NK)
         st = encode_map(&tm_b, B, (uint64_t)K, (uint64_t)b_rows, (uint64_t)ldb, bi::kBK, b_rows_box);
@@ -612,30 +632,41 @@ bi_status bi_decode_attention(const void *q, const void *k_cache, const void *v_
     bi_status st = device_state(&dev);
     if (st != BI_OK) return st;
     const int64_t S = bi::attn_splits(Lmax);
-    float *part_acc = static_cast<float *>(scratch);
-    float2 *part_ms = reinterpret_cast<float2 *>(part_acc + (size_t)B * Hq * S * D);
+    CUtensorMap tm_k, tm_v;
+    st = encode_kv_map(&tm_k, k_cache, (uint64_t)D, (uint64_t)Hkv, (uint64_t)Lmax, (uint64_t)B);
+    if (st != BI_OK) return st;
+    st = encode_kv_map(&tm_v, v_cache, (uint64_t)D, (uint64_t)Hkv, (uint64_t)Lmax, (uint64_t)B);
+    if (st != BI_OK) return st;
+    bi::AttnParams p{};
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.lens = seq_lens;
+    p.part_acc = static_cast<float *>(scratch);
+    p.part_ms = reinterpret_cast<float2 *>(p.part_acc + (size_t)B * Hq * S * D);
+    p.Hq = (int32_t)Hq;
+    p.Hkv = (int32_t)Hkv;
+    p.B = (int32_t)B;
+    p.Lmax = Lmax;
+    p.S = S;
+    p.scale = scale;
+    p.status = dev->status;
+    p.wait_limit_ns = kWaitLimitNs;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const auto *qb = static_cast<const __nv_bfloat16 *>(q);
-    const auto *kb = static_cast<const __nv_bfloat16 *>(k_cache);
-    const auto *vb = static_cast<const __nv_bfloat16 *>(v_cache);
-    const dim3 grid((unsigned)S, (unsigned)Hkv, (unsigned)B);
-    const size_t smem = sizeof(bi::AttnSmem);
+    // Persistent: one CTA per SM walks the (split, kv head, sequence) items; the grid size only
+    // decides which CTA computes an item, never an item's arithmetic.
+    const int64_t items = B * Hkv * S;
+    const dim3 grid((unsigned)(items < dev->sms ? items : dev->sms));
+    const size_t smem = (size_t)bi::kAttnSmem;
     switch (Hq / Hkv) {  // the group size is a property of the model, not of the batch
-    case 1: st = launch_pdl(bi::decode_attention_split_kernel<1>, grid, dim3(bi::kAttnThreads), smem, s, qb, kb, vb,
-                            seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
-    case 2: st = launch_pdl(bi::decode_attention_split_kernel<2>, grid, dim3(bi::kAttnThreads), smem, s, qb, kb, vb,
-                            seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
-    case 4: st = launch_pdl(bi::decode_attention_split_kernel<4>, grid, dim3(bi::kAttnThreads), smem, s, qb, kb, vb,
-                            seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
-    case 8: st = launch_pdl(bi::decode_attention_split_kernel<8>, grid, dim3(bi::kAttnThreads), smem, s, qb, kb, vb,
-                            seq_lens, part_ms, part_acc, (int)Hq, (int)Hkv, Lmax, scale, dev->status); break;
+    case 1: st = launch_pdl(bi::decode_attention_split_kernel<1>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
+    case 2: st = launch_pdl(bi::decode_attention_split_kernel<2>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
+    case 4: st = launch_pdl(bi::decode_attention_split_kernel<4>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
+    case 8: st = launch_pdl(bi::decode_attention_split_kernel<8>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
     default: return BI_ERR_UNSUPPORTED;
     }
     if (st != BI_OK) return st;
-    st = launch_pdl(bi::decode_attention_combine_kernel, dim3((unsigned)Hq, (unsigned)B), dim3(bi::kAttnD), 0, s,
-                    static_cast<const float2 *>(part_ms), static_cast<const float *>(part_acc), seq_lens,
-                    static_cast<__nv_bfloat16 *>(out), (int)Hq, Lmax);
-    return st;
+    return launch_pdl(bi::decode_attention_combine_kernel, dim3((unsigned)Hq, (unsigned)B), dim3(bi::kAttnD), 0, s,
+                      static_cast<const float2 *>(p.part_ms), static_cast<const float *>(p.part_acc), seq_lens,
+                      static_cast<__nv_bfloat16 *>(out), (int)Hq, Lmax);
 }
 
 bi_status bi_silu_mul(const void *gu, void *h, int64_t M, int64_t F, void *stream)
@@ -702,6 +733,13 @@ void bi_gemm_config(int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int3
     if (mma_k) *mma_k = bi::kMmaK;
 }
 
-int32_t bi_version(void) { return 100; }
+void bi_tensor_map_cache_stats(int64_t *hits, int64_t *misses)
+{
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    if (hits) *hits = (int64_t)g_map_hits;
+    if (misses) *misses = (int64_t)g_map_misses;
+}
+
+int32_t bi_version(void) { return 200; }
 
 }  // extern "C"

@@ -33,6 +33,7 @@ struct GemmParams {
     const __nv_bfloat16 *addend;
     int32_t *status;        // device status word
     uint64_t wait_limit_ns;
+    int32_t a_box_rows;     // rows of A one TMA box copies: M rounded up to 8, at most 128
 };
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float(b16 << 16); }

@@ -119,17 +119,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             for (int tile = first; ok && tile < num_tiles; tile += stride) {
-                const int m0 = (tile % m_blocks) * kPairBM + 128 * (int)rank;
+                const int m_pair = (tile % m_blocks) * kPairBM;
+                const int m0 = m_pair + 128 * (int)rank;
                 const int nh0 = p.fuse_silu ? (tile / m_blocks) * kHalfBN + (rank ? p.N : 0)
                                             : (tile / m_blocks) * kPairBN + kHalfBN * (int)rank;
+                // A rows are copied only where they exist: the box holds p.a_box_rows rows (M
+                // rounded up to 8, at most 128), and the second CTA's half is not copied at all
+                // when no row of it is below M.  Shared-memory rows left uncopied feed only
+                // accumulator rows at or beyond M, which are never stored.
+                const bool a_hi = m_pair + 128 < p.M;
+                const uint32_t a_bytes = (uint32_t)p.a_box_rows * (kBK * 2);
+                const uint32_t stage_bytes = (a_hi ? 2u : 1u) * a_bytes + 2u * kPBBytes;
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim)) {
                         ok = false;
                         break;
                     }
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kPStageBytes);
+                    if (leader) mbar_arrive_expect_tx(&full[stage], stage_bytes);
                     const uint32_t bar = map_to_rank(smem_addr(&full[stage]), 0);
-                    tma_load_2d_pair(sA + stage * kPABytes, &tm_a, bar, kb * kBK, m0);
+                    if (leader || a_hi) tma_load_2d_pair(sA + stage * kPABytes, &tm_a, bar, kb * kBK, m0);
                     uint8_t *dstB = sB + stage * kPBBytes;
                     if (p.b_mn_major) {
 #pragma unroll
@@ -159,7 +167,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ---------------------------------------------------------- MMA issuer (leader)
-            const uint32_t idesc = mma_idesc_bf16(kPairBM, kPairBN, p.b_mn_major ? 1u : 0u);
+            const uint32_t idesc = mma_idesc_bf16(kPairBM, kPairBN, 0u, p.b_mn_major ? 1u : 0u);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             bool ok = true;
             for (int tile = first; ok && tile < num_tiles; tile += stride) {

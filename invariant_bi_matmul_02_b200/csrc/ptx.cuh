@@ -183,14 +183,15 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_byte_addr, uint32_t
     return d;
 }
 
-// Instruction descriptor of tcgen05.mma kind::f16: bf16 x bf16 -> fp32, A K-major,
-// B K-major (b_mn_major = 0) or MN-major (1), shape M x N.
-__host__ __device__ constexpr uint32_t mma_idesc_bf16(uint32_t m, uint32_t n, uint32_t b_mn_major)
+// Instruction descriptor of tcgen05.mma kind::f16: bf16 x bf16 -> fp32, A and B each K-major
+// (0) or MN-major (1), shape M x N.
+__host__ __device__ constexpr uint32_t mma_idesc_bf16(uint32_t m, uint32_t n, uint32_t a_mn_major,
+                                                      uint32_t b_mn_major)
 {
     return (1u << 4)              // D format: f32
            | (1u << 7)            // A format: bf16
            | (1u << 10)           // B format: bf16
-           | (0u << 15)           // A major: K
+           | (a_mn_major << 15)   // A major
            | (b_mn_major << 16)   // B major
            | ((n >> 3) << 17)     // N / 8
            | ((m >> 4) << 24);    // M / 16

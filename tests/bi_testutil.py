@@ -104,5 +104,7 @@ def bf16_bits_np(t: torch.Tensor) -> np.ndarray:
     return inputs.bf16_bits(t)
 
 
-# The M values of the GEMM sweep (powers of two up to 2048 plus the odd sizes).
-M_SWEEP = [1, 2, 3, 4, 8, 16, 32, 64, 77, 128, 256, 512, 1000, 1024, 2048]
+# The M values of the GEMM sweep: powers of two up to 2048, the odd sizes, and the sizes on
+# either side of the GEMM's 128-token half-tile (a tile whose second half holds no token skips
+# that half's MMAs): 129, 384, 385.
+M_SWEEP = [1, 2, 3, 4, 8, 16, 32, 64, 77, 128, 129, 256, 384, 385, 512, 1000, 1024, 2048]

@@ -61,6 +61,22 @@ def test_attention_batch_invariance_over_compositions():
         assert same_bits(o, ref[idx]), f"trial {t}: batch of {b} changed a sequence's output"
 
 
+def test_attention_ignores_cache_contents_past_each_length():
+    """Cache rows past a sequence's length may hold anything (a reused buffer, NaN or infinity
+    bit patterns); the output must not change by a bit."""
+    B, Hq, Hkv, Lmax = 4, 32, 8, 300
+    q, k, v = make(809, B, Hq, Hkv, Lmax)
+    lens = [1, 130, 255, 300]
+    sl = torch.tensor(lens, dtype=torch.int32).to(DEV)
+    clean = bi.bi_decode_attention(q.to(DEV), k.to(DEV), v.to(DEV), sl)
+    k2, v2 = k.clone(), v.clone()
+    for b, L in enumerate(lens):
+        k2[b, L:] = float("nan")
+        v2[b, L:] = float("inf") if b % 2 else float("nan")
+    dirty = bi.bi_decode_attention(q.to(DEV), k2.to(DEV), v2.to(DEV), sl)
+    assert same_bits(clean, dirty)
+
+
 def test_attention_repeatable_100_runs():
     B, Hq, Hkv, Lmax = 16, 32, 8, 700
     q, k, v = make(806, B, Hq, Hkv, Lmax)

@@ -278,6 +278,23 @@ def test_matmul_repeatable_100_runs():
         assert same_bits(bi.bi_matmul(a, w), first)
 
 
+def test_tensor_map_cache_hits_on_repeated_calls():
+    """A repeated call with the same buffers is served two tensor maps from the cache; a new
+    activation buffer is one miss (its map) and one hit (the weights' map); results agree."""
+    a = inputs.rows_normal(248, 0, 4, 256).to(DEV)
+    w = weight(249, 512, 256, "nk").to(DEV)
+    first = bi.bi_matmul(a, w)
+    h0, m0 = bi.bi_tensor_map_cache_stats()
+    again = bi.bi_matmul(a, w)
+    h1, m1 = bi.bi_tensor_map_cache_stats()
+    assert (h1 - h0, m1 - m0) == (2, 0)
+    a2 = a.clone()
+    other = bi.bi_matmul(a2, w)
+    h2, m2 = bi.bi_tensor_map_cache_stats()
+    assert (h2 - h1, m2 - m1) == (1, 1)
+    assert same_bits(first, again) and same_bits(first, other)
+
+
 # ----------------------------------------------------------------------------- errors
 
 def test_invalid_arguments_are_rejected():
