@@ -42,7 +42,8 @@ constexpr int kAttnQBytes = 16 * kAttnQStride * 2;      // query rows of a group
 constexpr int kAttnStageBytes = 2 * kAttnTileBytes + ((kAttnQBytes + 1023) / 1024) * 1024;
 constexpr int kAttnSmem = kAttnStages * kAttnStageBytes + 1024;  // + alignment slack
 
-static_assert(kAttnConsumers * kAttnMaxGroup * kAttnD * 4 <= kAttnTileBytes,
+constexpr int kAttnOStride = kAttnD + 4;                // per-warp output rows in shared memory (floats)
+static_assert(kAttnConsumers * kAttnMaxGroup * kAttnOStride * 4 <= kAttnTileBytes,
               "per-warp partial outputs fit in the K tile they replace");
 
 struct AttnParams {
@@ -153,8 +154,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     extern __shared__ uint8_t attn_raw[];
     uint8_t *smem = attn_raw + ((1024u - (smem_addr(attn_raw) & 1023u)) & 1023u);
     __shared__ uint64_t kfull[kAttnStages], vfull[kAttnStages], empty[kAttnStages];
-    __shared__ float red_all[kAttnGroups][kAttnConsumers][16];
-    __shared__ float stat_all[kAttnGroups][16][2];
+    __shared__ float red_m_all[kAttnGroups][kAttnConsumers][16];  // per-warp maxima of the 16 rows
+    __shared__ float red_s_all[kAttnGroups][kAttnConsumers][16];  // per-warp sums of exp
     __shared__ int abort_flag_s;
     __shared__ int progress_s[kAttnGroups];  // items a consumer group has started (local index + 1)
     volatile int *abort_flag = &abort_flag_s;
@@ -169,7 +170,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int s = 0; s < kAttnStages; ++s) {
             mbar_init(&kfull[s], 1);
             mbar_init(&vfull[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], kAttnConsumers);  // one arrival per consumer warp
         }
         abort_flag_s = 0;
         for (int g = 0; g < kAttnGroups; ++g) progress_s[g] = 0;
@@ -232,8 +233,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int cw = (warp - 1) % kAttnConsumers, ct = threadIdx.x - 32 - 32 * kAttnConsumers * grp;
         const int bar_id = 1 + grp;
         const int gid = lane >> 2, tig = lane & 3;
-        float (*red)[16] = red_all[grp];
-        float (*stat)[2] = stat_all[grp];
+        float (*red_m)[16] = red_m_all[grp];
+        float (*red_s)[16] = red_s_all[grp];
         uint32_t local = 0;
         for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
             const int split = (int)(it % p.S), g = (int)((it / p.S) % p.Hkv), b = (int)(it / (p.S * p.Hkv));
@@ -296,21 +297,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 mx[h] = m;
             }
             if (tig == 0) {
-                red[cw][gid] = mx[0];
-                red[cw][gid + 8] = mx[1];
+                red_m[cw][gid] = mx[0];
+                red_m[cw][gid + 8] = mx[1];
             }
-            consumers_sync(bar_id);
-            if (ct < 16) {
-                float m = red[0][ct];
-                for (int w = 1; w < kAttnConsumers; ++w) m = fmaxf(m, red[w][ct]);
-                stat[ct][0] = m;
-            }
-            consumers_sync(bar_id);
-            // ---- p = exp(s - max); per-head sums by the same trees
+            consumers_sync(bar_id);  // every warp's maxima are posted; the K tile is no longer read
+            // ---- p = exp(s - max); per-head sums by the same trees.  Each thread folds the warps'
+            // maxima of its two heads itself, in warp order.
             float sum[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const float m = stat[gid + 8 * h][0];
+                float m = red_m[0][gid + 8 * h];
+#pragma unroll
+                for (int w = 1; w < kAttnConsumers; ++w) m = fmaxf(m, red_m[w][gid + 8 * h]);
                 float l = 0.0f;
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt)
@@ -324,17 +322,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 2));
                 sum[h] = l;
             }
-            consumers_sync(bar_id);  // every warp has read stat / red
             if (tig == 0) {
-                red[cw][gid] = sum[0];
-                red[cw][gid + 8] = sum[1];
+                red_s[cw][gid] = sum[0];
+                red_s[cw][gid + 8] = sum[1];
             }
             if (!consumers_all(bar_id, wait_bounded(&vfull[stage], use & 1u, abort_flag, p.status, lim))) break;
-            if (ct < 16) {
-                float l = red[0][ct];
-                for (int w = 1; w < kAttnConsumers; ++w) l = __fadd_rn(l, red[w][ct]);
-                stat[ct][1] = l;
-            }
             if (n_tok < kAttnSplit) {
                 // Value rows past the sequence's end: zero, whatever the cache holds there.
                 for (int i = ct; i < (kAttnSplit - n_tok) * 16; i += 32 * kAttnConsumers)
@@ -377,29 +369,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     mma_16816_bf16(o[dt + 1], pa_lo, vf[2], vf[3]);
                 }
             }
-            consumers_sync(bar_id);  // the K tile is no longer read: it holds the per-warp outputs now
+            // The K tile (read by every warp before the maxima barrier) holds the per-warp outputs,
+            // rows kAttnOStride floats apart so that the eight rows of a store hit different banks.
             float *so = reinterpret_cast<float *>(const_cast<uint8_t *>(ks));
 #pragma unroll
             for (int dt = 0; dt < kAttnD / 8; ++dt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int row = gid + 8 * (e >> 1), col = 8 * dt + 2 * tig + (e & 1);
-                    if (row < G) so[(cw * kAttnMaxGroup + row) * kAttnD + col] = o[dt][e];
+                    if (row < G) so[(cw * kAttnMaxGroup + row) * kAttnOStride + col] = o[dt][e];
                 }
             consumers_sync(bar_id);
 #pragma unroll
             for (int j = 0; j < G; ++j) {
-                float r = so[j * kAttnD + ct];
-                for (int w = 1; w < kAttnConsumers; ++w) r = __fadd_rn(r, so[(w * kAttnMaxGroup + j) * kAttnD + ct]);
+                float r = so[j * kAttnOStride + ct];
+                for (int w = 1; w < kAttnConsumers; ++w)
+                    r = __fadd_rn(r, so[(w * kAttnMaxGroup + j) * kAttnOStride + ct]);
                 const int64_t bh = (int64_t)b * p.Hq + (int64_t)g * G + j;
                 p.part_acc[(bh * p.S + split) * kAttnD + ct] = r;
-                if (ct == 0) p.part_ms[bh * p.S + split] = make_float2(stat[j][0], stat[j][1]);
+                if (ct == 0) {
+                    float m = red_m[0][j], l = red_s[0][j];
+                    for (int w = 1; w < kAttnConsumers; ++w) {
+                        m = fmaxf(m, red_m[w][j]);
+                        l = __fadd_rn(l, red_s[w][j]);
+                    }
+                    p.part_ms[bh * p.S + split] = make_float2(m, l);
+                }
             }
-            // Release the stage: the generic-proxy writes above (partial outputs, zeroed rows) are
-            // ordered before the next TMA writes into it.
+            // Release the stage, one arrival per warp: the generic-proxy writes into it (partial
+            // outputs, zeroed rows) are ordered before the next TMA writes.
             fence_proxy_async_smem();
-            consumers_sync(bar_id);
-            if (ct == 0) mbar_arrive(&empty[stage]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
         }
     }
     __syncthreads();
