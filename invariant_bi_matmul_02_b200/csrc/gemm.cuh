@@ -86,12 +86,10 @@ __device__ __forceinline__ void store_row_chunk(const GemmParams &p, int64_t row
         if (full) {
             uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 w = make_uint4(pack2_bf16(v[8 * q], v[8 * q + 1]), pack2_bf16(v[8 * q + 2], v[8 * q + 3]),
-                                           pack2_bf16(v[8 * q + 4], v[8 * q + 5]),
-                                           pack2_bf16(v[8 * q + 6], v[8 * q + 7]));
-                d4[q] = w;
-            }
+            for (int q = 0; q < 4; ++q)
+                d4[q] = make_uint4(pack2_bf16(v[8 * q], v[8 * q + 1]), pack2_bf16(v[8 * q + 2], v[8 * q + 3]),
+                                   pack2_bf16(v[8 * q + 4], v[8 * q + 5]),
+                                   pack2_bf16(v[8 * q + 6], v[8 * q + 7]));
         } else {
             for (int j = 0; j < 32 && col0 + j < p.N; ++j) dst[j] = __float2bfloat16_rn(v[j]);
         }
