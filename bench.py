@@ -666,6 +666,15 @@ def metric_sweep(device, peaks: dict, reps: int = 10) -> dict:
     return out
 
 
+def run_mma_probe(args):
+    """Cycles per back-to-back tcgen05.mma for several instruction shapes (the stand-alone probe
+    built by csrc/build.py); one JSON line per shape."""
+    from invariant_bi_matmul_02_b200.csrc import build as libbuild
+    exe = libbuild.build_probe()
+    out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
+    print(out, end="", flush=True)
+
+
 def run_host_overhead(args):
     """Host time per bi_matmul call at M = 1 (K = N = 256) through the binding, with the tensor-map
     cache hitting (the same buffers every call) and missing (a new activation address each call,
@@ -878,6 +887,8 @@ KERNEL_CASES = {
     "gemm_gate_up": "bi_matmul M=1024 K=4096 N=24576 (B [N, K])",
     "gemm_lm_head": "bi_matmul M=1024 K=4096 N=151936 (B [N, K])",
     "gemm_qo_m256": "bi_matmul M=256 K=4096 N=4096 (B [N, K])",
+    "gemm_kv_m1": "bi_matmul M=1 K=4096 N=1024 (B [N, K])",
+    "gemm_down_m64": "bi_matmul M=64 K=12288 N=4096 (B [N, K])",
     "gemm_gate_up_silu": "bi_matmul_silu_mul M=1024 K=4096 F=12288 (B [2F, K])",
     "rmsnorm": "bi_rmsnorm M=16384 H=4096 bf16",
     "mean": "bi_mean M=16384 H=4096 fp32",
@@ -905,7 +916,8 @@ def run_kernel_case(args):
         work, unit = 2 * 1024 * 2 * FFN * HIDDEN, "TFLOP/s"
     elif name.startswith("gemm"):
         M, K, N = {"gemm_gate_up": (1024, HIDDEN, 2 * FFN), "gemm_lm_head": (1024, HIDDEN, VOCAB),
-                   "gemm_qo_m256": (256, HIDDEN, HIDDEN)}[name]
+                   "gemm_qo_m256": (256, HIDDEN, HIDDEN), "gemm_kv_m1": (1, HIDDEN, KV),
+                   "gemm_down_m64": (64, FFN, HIDDEN)}[name]
         a = inputs.rows_normal(50, 0, M, K).to(dev)
         w = inputs.weight_normal(51, (N, K)).to(dev)
         c = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
@@ -1140,6 +1152,8 @@ def main():
                     help="gate/up + SiLU*up as one fused GEMM (default) or GEMM then bi_silu_mul")
     ap.add_argument("--cpu-budget", type=float, default=25.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mma-probe", action="store_true",
+                    help="cycles per tcgen05.mma for several instruction shapes")
     ap.add_argument("--host-overhead", action="store_true",
                     help="host time per small GEMM call with and without tensor-map cache hits")
     ap.add_argument("--no-metric-sweep", action="store_true",
@@ -1166,6 +1180,9 @@ def main():
         return
     if args.host_overhead:
         run_host_overhead(args)
+        return
+    if args.mma_probe:
+        run_mma_probe(args)
         return
     if args.uniqueness:
         run_uniqueness(args)

@@ -42,7 +42,7 @@ constexpr int kAttnQBytes = 16 * kAttnQStride * 2;      // query rows of a group
 constexpr int kAttnStageBytes = 2 * kAttnTileBytes + ((kAttnQBytes + 1023) / 1024) * 1024;
 constexpr int kAttnSmem = kAttnStages * kAttnStageBytes + 1024;  // + alignment slack
 
-constexpr int kAttnOStride = kAttnD + 4;                // per-warp output rows in shared memory (floats)
+constexpr int kAttnOStride = kAttnD + 8;                // per-warp output rows in shared memory (floats)
 static_assert(kAttnConsumers * kAttnMaxGroup * kAttnOStride * 4 <= kAttnTileBytes,
               "per-warp partial outputs fit in the K tile they replace");
 
@@ -370,7 +370,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
             }
             // The K tile (read by every warp before the maxima barrier) holds the per-warp outputs,
-            // rows kAttnOStride floats apart so that the eight rows of a store hit different banks.
+            // rows kAttnOStride floats apart: a store's lanes cover rows 0..3 (x 4 columns two
+            // apart) in distinct banks; rows 4..7 (group size 8) share banks with rows 0..3.
             float *so = reinterpret_cast<float *>(const_cast<uint8_t *>(ks));
 #pragma unroll
             for (int dt = 0; dt < kAttnD / 8; ++dt)

@@ -42,5 +42,20 @@ def build(force: bool = False, out: str = LIB, defines=(), verbose: bool = False
     return out
 
 
+PROBE_SRC = os.path.join(CSRC, "mma_probe.cu")
+PROBE = os.path.join(PKG, "mma_probe")
+
+
+def build_probe(force: bool = False) -> str:
+    """The tcgen05 MMA cost probe (a stand-alone program, not part of libbi.so)."""
+    deps = [PROBE_SRC, os.path.join(CSRC, "ptx.cuh")]
+    if not force and os.path.exists(PROBE) and os.path.getmtime(PROBE) >= max(os.path.getmtime(p) for p in deps):
+        return PROBE
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-I" + CSRC, "-o", PROBE,
+           PROBE_SRC]
+    subprocess.run(cmd, check=True)
+    return PROBE
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
