@@ -249,9 +249,10 @@ __global__ void __launch_bounds__(1024, 1) log_softmax_scalar_kernel(const void 
 // builds the row's (max, sum of exp); pass 2 writes y = (x - max) - log(sum), starting
 // with the last chunks of the row, which are still in the ring, and streaming the rest
 // again in descending order, so the chunk read most recently (the likeliest to be still in
-// L2) comes first.  Pass-1 copies ask L2 to keep their lines (they are read again in pass 2),
-// pass-2 copies ask it to drop theirs, and y is written with streaming stores so that it does
-// not push the rows' inputs out of L2 before their second read.  (B200, M = 1024, V = 151936
+// L2) comes first.  Pass-1 copies of the chunks pass 2 reads again ask L2 to keep their lines;
+// every other copy (the chunks that stay in the ring, and the second reads) asks it to drop
+// them, and y is written with streaming stores, so that neither pushes the rows' inputs out of
+// L2 before their second read.  (B200, M = 1024, V = 151936
 // bf16 with L2 flushed: 180 us, against 186 us with ascending re-reads and default-policy y
 // stores; the same bits.)
 //
@@ -314,8 +315,9 @@ __global__ void __launch_bounds__(kLsmThreads, 2)
         const uint32_t bytes = (uint32_t)(row_bytes - off < kLsmChunk ? row_bytes - off : kLsmChunk);
         uint64_t *bar = &full[j % kLsmStages];
         mbar_arrive_expect_tx(bar, bytes);
+        // Only the chunks pass 2 reads again (0 .. R-1) ask L2 to keep their lines.
         bulk_load_hint(ring[j % kLsmStages], xr + off, bytes, bar,
-                       j < n ? l2_policy_evict_last() : l2_policy_evict_first());
+                       j < R ? l2_policy_evict_last() : l2_policy_evict_first());
     };
     if (tid == 0)
         for (; issued < kLsmStages && issued < n; ++issued) issue(issued);
