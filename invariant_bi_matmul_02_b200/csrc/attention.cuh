@@ -408,11 +408,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // Launch 2: grid (Hq, B), kAttnD threads.  Fold the sequence's splits in ascending order.
+// The splits' maximum is exact in any order, so the block takes it in parallel; the weights
+// w_s = exp(m_s - max) and the split sums go to shared memory a chunk at a time, and each thread
+// folds l += sum_s w_s and o += acc_s w_s in ascending s with its value loads issued ahead.
+constexpr int kCombineChunk = kAttnD;
+
 __global__ void __launch_bounds__(kAttnD)
     decode_attention_combine_kernel(const float2 *__restrict__ part_ms, const float *__restrict__ part_acc,
                                     const int32_t *__restrict__ lens, __nv_bfloat16 *__restrict__ out,
                                     int Hq, int64_t Lmax)
 {
+    __shared__ float w_s[kCombineChunk], l_s[kCombineChunk], red[kAttnD / 32];
     griddep_wait();  // every split's partials are complete
     griddep_launch_dependents();
     const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
@@ -421,14 +427,42 @@ __global__ void __launch_bounds__(kAttnD)
     L = L < 1 ? 1 : (L > Lmax ? Lmax : L);
     const int64_t n = attn_splits(L);
     const int64_t bh = (int64_t)b * Hq + h;
+    const float2 *ms = part_ms + bh * S;
+    const float *acc = part_acc + bh * S * kAttnD + d;
     float m = kNegInf;
-    for (int64_t s = 0; s < n; ++s) m = fmaxf(m, part_ms[bh * S + s].x);
+    for (int64_t s = d; s < n; s += kAttnD) m = fmaxf(m, ms[s].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((d & 31) == 0) red[d >> 5] = m;
+    __syncthreads();
+    m = red[0];
+#pragma unroll
+    for (int w = 1; w < kAttnD / 32; ++w) m = fmaxf(m, red[w]);
     float l = 0.0f, o = 0.0f;
-    for (int64_t s = 0; s < n; ++s) {
-        const float2 ms = part_ms[bh * S + s];
-        const float w = __expf(ms.x - m);
-        l = fmaf(ms.y, w, l);
-        o = fmaf(part_acc[(bh * S + s) * kAttnD + d], w, o);
+    for (int64_t s0 = 0; s0 < n; s0 += kCombineChunk) {
+        const int cnt = (int)(n - s0 < kCombineChunk ? n - s0 : kCombineChunk);
+        __syncthreads();  // the previous chunk's weights have been read
+        if (d < cnt) {
+            const float2 v = ms[s0 + d];
+            w_s[d] = __expf(v.x - m);
+            l_s[d] = v.y;
+        }
+        __syncthreads();
+        int j = 0;
+        for (; j + 8 <= cnt; j += 8) {
+            float a[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) a[u] = acc[(s0 + j + u) * kAttnD];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                l = fmaf(l_s[j + u], w_s[j + u], l);
+                o = fmaf(a[u], w_s[j + u], o);
+            }
+        }
+        for (; j < cnt; ++j) {
+            l = fmaf(l_s[j], w_s[j], l);
+            o = fmaf(acc[(s0 + j) * kAttnD], w_s[j], o);
+        }
     }
     out[bh * kAttnD + d] = __float2bfloat16_rn(o / l);
 }
