@@ -66,3 +66,15 @@ def test_clock_sampler_reports_median_and_active_reasons():
     assert out["reasons"] == ["sw_power_cap"] and out["samples"] == 3
     s.proc = _FakeSmi("0, 900, 1965, 500.0, 0x8, Active, Not Active, Not Active, Not Active")
     assert s.stop()["reasons"] == ["hw_slowdown"]
+
+
+def test_roofline_point_takes_the_larger_bound():
+    """The roofline time of a launch is the larger of its FLOPs at the tensor peak and its
+    algorithmic bytes at the HBM peak; the fraction is that time over the measured one."""
+    peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
+    # 2 TFLOP at 1000 TFLOP/s = 2 ms; 1 GB at 5000 GB/s = 0.2 ms: tensor-bound
+    r = bench.roofline_point(2e12, 1e9, 4000.0, peaks)
+    assert r == {"bound": "tensor", "roofline_frac": 0.5}
+    # 1 GFLOP = 1 us of tensor time; 50 MB = 10 us of HBM time: HBM-bound, measured 20 us
+    r = bench.roofline_point(1e9, 50e6, 20.0, peaks)
+    assert r == {"bound": "hbm", "roofline_frac": 0.5}
