@@ -48,7 +48,8 @@ constexpr int kPairSmem = kPStages * kPStageBytes + kSmemMisc;
 constexpr uint32_t kPairTmemCols = pow2_at_least(2 * kPairBN);
 
 static_assert(kPairBN % 128 == 0 && kPairBN <= 256, "pair tile N must be 128 or 256");
-static_assert(kPStages >= 2, "need at least two pipeline stages");
+static_assert(kPStages >= 2 && kPStages <= 32, "two to 32 pipeline stages (one producer lane per stage at the tail)");
+static_assert(kPairSmem + 1024 <= 256 * 1024, "shared addresses fit the 14-bit descriptor address field");
 static_assert(kPairTmemCols <= 512, "accumulators must fit in tensor memory");
 static_assert(kPairSmem > 114 * 1024, "one CTA per SM keeps the TMEM allocation uncontended");
 
@@ -114,10 +115,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const uint64_t lim = p.wait_limit_ns;
 
     if (warp == 0) {
+        uint32_t stage = 0, phase = 0;
+        bool ok = true;
         if (lane == 0) {
             // ---------------------------------------------------------- TMA producer (both CTAs)
-            uint32_t stage = 0, phase = 0;
-            bool ok = true;
             for (int tile = first; ok && tile < num_tiles; tile += stride) {
                 const int m_pair = (tile % m_blocks) * kPairBM;
                 const int m0 = m_pair + 128 * (int)rank;
@@ -149,25 +150,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     advance(stage, phase, kPStages);
                 }
             }
-            if (ok) {
-                // Tail: every stage released by the leader's MMA, so no multicast arrival
-                // is still on its way to this CTA when it exits.
-                for (int s = 0; s < kPStages; ++s) {
-                    if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim)) break;
-                    advance(stage, phase, kPStages);
-                }
-            } else {
-                // Abort: loads already issued complete on the leader's barrier, which this
-                // CTA cannot observe; give them a bounded grace period to land.
-                const uint64_t t0 = global_timer_ns();
-                while (global_timer_ns() - t0 < 2000000ull) {
-                }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        stage = __shfl_sync(0xffffffffu, stage, 0);
+        phase = __shfl_sync(0xffffffffu, phase, 0);
+        if (ok) {
+            // Tail: every stage released by the leader's MMA, so no multicast arrival is still
+            // on its way to this CTA when it exits.  Lane j waits for the j-th stage after the
+            // last one filled (the same barriers and parities a sequential walk would take); a
+            // wait that completes still costs a few hundred cycles, so the lanes take them at once.
+            if (lane < kPStages) {
+                const uint32_t j = stage + (uint32_t)lane;
+                const uint32_t st = j < (uint32_t)kPStages ? j : j - kPStages;
+                const uint32_t ph = j < (uint32_t)kPStages ? phase : phase ^ 1u;
+                wait_bounded(&empty[st], ph ^ 1u, abort_flag, p.status, lim);
+            }
+            __syncwarp();
+        } else if (lane == 0) {
+            // Abort: loads already issued complete on the leader's barrier, which this CTA
+            // cannot observe; give them a bounded grace period to land.
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < 2000000ull) {
             }
         }
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ---------------------------------------------------------- MMA issuer (leader)
             const uint32_t idesc = mma_idesc_bf16(kPairBM, kPairBN, 0u, p.b_mn_major ? 1u : 0u);
+            // Descriptors of stage 0's first K step.  A stage or a K step moves only the start
+            // address field (address / 16 in the low 14 bits; every shared address of this CTA
+            // fits, so the sum never carries into the next field): one add per MMA instead of a
+            // descriptor rebuilt on the issuing thread's critical path.
+            const uint64_t a_desc0 = sw128_desc(smem_addr(sA), 16, 1024);
+            const uint64_t b_desc0 = p.b_mn_major ? sw128_desc(smem_addr(sB), 64 * kBK * 2, 1024)
+                                                  : sw128_desc(smem_addr(sB), 16, 1024);
+            const uint32_t b_step = p.b_mn_major ? (kMmaK * 128) >> 4 : (kMmaK * 2) >> 4;
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             bool ok = true;
             for (int tile = first; ok && tile < num_tiles; tile += stride) {
@@ -183,16 +200,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t a_base = smem_addr(sA + stage * kPABytes);
-                    const uint32_t b_base = smem_addr(sB + stage * kPBBytes);
+                    const uint64_t a_desc = a_desc0 + stage * (uint32_t)(kPABytes >> 4);
+                    const uint64_t b_desc = b_desc0 + stage * (uint32_t)(kPBBytes >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / kMmaK; ++kk) {
-                        const uint64_t a_desc = sw128_desc(a_base + kk * (kMmaK * 2), 16, 1024);
-                        const uint64_t b_desc =
-                            p.b_mn_major ? sw128_desc(b_base + kk * (kMmaK * 128), 64 * kBK * 2, 1024)
-                                         : sw128_desc(b_base + kk * (kMmaK * 2), 16, 1024);
-                        tc_mma_bf16_pair(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < kBK / kMmaK; ++kk)
+                        tc_mma_bf16_pair(d_tmem, a_desc + kk * ((kMmaK * 2) >> 4), b_desc + kk * b_step, idesc,
+                                         (kb | kk) != 0 ? 1u : 0u);
                     tc_commit_pair_mc(&empty[stage], 0x3);
                     advance(stage, phase, kPStages);
                 }
