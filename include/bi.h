@@ -18,9 +18,10 @@
  * and the SiLU-times-up glue of a gated MLP.
  *
  * How each entry point fixes its order (the same for every M):
- *   - bi_matmul / bi_addmm: one tcgen05/TMEM tile configuration fed by TMA for
- *     every shape; every output element accumulates its K products in fp32,
- *     16 at a time, in ascending K; no split-K, no stream-K, no tile switch.
+ *   - bi_matmul / bi_addmm: tcgen05/TMEM tiles fed by TMA; the tile width is a
+ *     function of the output width N alone (bi_gemm_config), never of M; every
+ *     output element accumulates its K products in fp32, 16 at a time, in
+ *     ascending K, in either configuration; no split-K, no stream-K.
  *   - bi_rmsnorm / bi_mean / bi_log_softmax: one thread block per row; the
  *     block size and each thread's element set depend only on the row length;
  *     partial results merge through a fixed warp-shuffle tree and a fixed
@@ -307,11 +308,15 @@ bi_status bi_selftest_wait_timeout(int64_t limit_ns, void *stream);
 const char *bi_status_string(bi_status status);
 
 /*
- * bi_gemm_config -- report the single tile configuration every bi_matmul / bi_addmm
- * call uses: output tile bm x bn, K-slice bk per pipeline stage, number of stages,
- * and the K step of one tensor-core instruction.  Any pointer may be NULL.
+ * bi_gemm_config -- report the tile configuration the GEMM entry points use for an
+ * output width n (the N of bi_matmul / bi_addmm, the F of bi_matmul_silu_mul): output
+ * tile bm x bn, K per pipeline stage bk, number of stages, and the K step of one
+ * tensor-core instruction.  The configuration depends on n alone -- every M of a
+ * given weight matrix runs the same one -- and both configurations take the same
+ * 16-wide K steps in ascending order, so an element's bits do not depend on it.
+ * n <= 0 reports the configuration of wide outputs.  Any pointer may be NULL.
  */
-void bi_gemm_config(int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int32_t *mma_k);
+void bi_gemm_config(int64_t n, int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int32_t *mma_k);
 
 /*
  * bi_tensor_map_cache_stats -- how many TMA tensor-map look-ups of the GEMM entry points were

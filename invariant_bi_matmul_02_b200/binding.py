@@ -44,7 +44,7 @@ SIGNATURES = {
     "bi_get_device_status": (ctypes.c_int, [_p, ctypes.POINTER(_i32)]),
     "bi_selftest_wait_timeout": (ctypes.c_int, [_i64, _p]),
     "bi_status_string": (ctypes.c_char_p, [ctypes.c_int]),
-    "bi_gemm_config": (None, [ctypes.POINTER(_i32)] * 5),
+    "bi_gemm_config": (None, [_i64] + [ctypes.POINTER(_i32)] * 5),
     "bi_tensor_map_cache_stats": (None, [ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
     "bi_version": (ctypes.c_int32, []),
 }
@@ -383,9 +383,10 @@ def bi_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
     _check("bi_selftest_wait_timeout", load().bi_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
 
-def bi_gemm_config() -> dict:
+def bi_gemm_config(n: int = 0) -> dict:
+    """Tile configuration of the GEMM entry points for output width n (n <= 0: wide outputs)."""
     vals = [_i32(0) for _ in range(5)]
-    load().bi_gemm_config(*[ctypes.byref(v) for v in vals])
+    load().bi_gemm_config(int(n), *[ctypes.byref(v) for v in vals])
     return dict(zip(("bm", "bn", "bk", "stages", "mma_k"), (int(v.value) for v in vals)))
 
 

@@ -33,7 +33,8 @@ constexpr int64_t kI32Max = 2147483647;
 struct DeviceState {
     bool ready = false;
     int sms = 0;
-    int gemm_clusters = 0;  // CTA pairs of the GEMM that fit on the device at once
+    int gemm_clusters_wide = 0;    // CTA pairs of each GEMM configuration that fit on the device at once
+    int gemm_clusters_narrow = 0;
     int32_t *status = nullptr;
 };
 
@@ -41,6 +42,30 @@ std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Opt the GEMM configuration T into its shared memory and count the CTA pairs that fit at once.
+template <typename T>
+bi_status pair_clusters(int sms, int *out)
+{
+    const void *fn = reinterpret_cast<const void *>(bi::gemm_bf16_pair_kernel<T::kBN, T::kStageK>);
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmem) != cudaSuccess)
+        return BI_ERR_CUDA;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * sms, 1, 1);
+    cfg.blockDim = dim3(bi::kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = T::kSmem;
+    cudaLaunchAttribute attr{};
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n < 1) return BI_ERR_CUDA;
+    *out = n;
+    return BI_OK;
+}
 
 bi_status device_state(DeviceState **out)
 {
@@ -55,26 +80,9 @@ bi_status device_state(DeviceState **out)
         void *sym = nullptr;
         if (cudaGetSymbolAddress(&sym, g_bi_status) != cudaSuccess) return BI_ERR_CUDA;
         d.status = static_cast<int32_t *>(sym);
-        if (cudaFuncSetAttribute(bi::gemm_bf16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 bi::kPairSmem) != cudaSuccess)
+        if (pair_clusters<bi::WideTile>(d.sms, &d.gemm_clusters_wide) != BI_OK ||
+            pair_clusters<bi::NarrowTile>(d.sms, &d.gemm_clusters_narrow) != BI_OK)
             return BI_ERR_CUDA;
-        {
-            cudaLaunchConfig_t cfg{};
-            cfg.gridDim = dim3(2 * d.sms, 1, 1);
-            cfg.blockDim = dim3(bi::kGemmThreads, 1, 1);
-            cfg.dynamicSmemBytes = bi::kPairSmem;
-            cudaLaunchAttribute attr{};
-            attr.id = cudaLaunchAttributeClusterDimension;
-            attr.val.clusterDim.x = 2;
-            attr.val.clusterDim.y = 1;
-            attr.val.clusterDim.z = 1;
-            cfg.attrs = &attr;
-            cfg.numAttrs = 1;
-            int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, bi::gemm_bf16_pair_kernel, &cfg) != cudaSuccess || n < 1)
-                return BI_ERR_CUDA;
-            d.gemm_clusters = n;
-        }
         if (cudaFuncSetAttribute(bi::decode_attention_split_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  bi::kAttnSmem) != cudaSuccess ||
             cudaFuncSetAttribute(bi::decode_attention_split_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -267,6 +275,35 @@ bi_status launch_row_clusters(void (*kernel)(KArgs...), int64_t M, size_t smem, 
 
 // N is the number of output columns.  With fuse_silu, B holds 2N rows ([gate; up]) and
 // the output is silu(A . gate^T) * (A . up^T).
+// Tile counts, tensor maps and the launch of the pair GEMM in configuration T.
+template <typename T>
+bi_status launch_pair(bi::GemmParams p, const void *A, int64_t lda, const void *B, int64_t ldb, int b_layout,
+                      int64_t b_rows, int pairs, cudaStream_t s)
+{
+    const int64_t M = p.M, N = p.N, K = p.K;
+    p.m_blocks = (int32_t)((M + bi::kPairBM - 1) / bi::kPairBM);
+    p.n_blocks = (int32_t)(p.fuse_silu ? (N + T::kHalf - 1) / T::kHalf : (N + T::kBN - 1) / T::kBN);
+    p.k_blocks = (int32_t)((K + T::kStageK - 1) / T::kStageK);
+    const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
+    if (tiles > kI32Max) return BI_ERR_UNSUPPORTED;
+
+    CUtensorMap tm_a, tm_b;
+    // The A box copies the rows that exist: M rounded up to 8, at most the CTA's 128.  The tile,
+    // the MMA shape and every element's K order are the same for every M.
+    p.a_box_rows = (int32_t)(M >= bi::kBM ? bi::kBM : (M + 7) / 8 * 8);
+    bi_status st = encode_map(&tm_a, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda, bi::kBK, (uint32_t)p.a_box_rows);
+    if (st != BI_OK) return st;
+    if (b_layout == BI_B_NK)
+        st = encode_map(&tm_b, B, (uint64_t)K, (uint64_t)b_rows, (uint64_t)ldb, bi::kBK, (uint32_t)T::kHalf);
+    else
+        st = encode_map(&tm_b, B, (uint64_t)b_rows, (uint64_t)K, (uint64_t)ldb, 64, (uint32_t)T::kStageK);
+    if (st != BI_OK) return st;
+
+    const int grid = 2 * (int)(tiles < pairs ? tiles : pairs);
+    return launch_pdl(bi::gemm_bf16_pair_kernel<T::kBN, T::kStageK>, dim3(grid), dim3(bi::kGemmThreads),
+                      (size_t)T::kSmem, s, tm_a, tm_b, p);
+}
+
 bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, const void *A, int64_t lda,
                       const void *B, int64_t ldb, int b_layout, void *C, int64_t ldc, int c_dtype,
                       int64_t M, int64_t N, int64_t K, void *stream, int fuse_silu = 0)
@@ -301,10 +338,7 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
     p.M = (int32_t)M;
     p.N = (int32_t)N;
     p.K = (int32_t)K;
-    p.m_blocks = (int32_t)((M + bi::kPairBM - 1) / bi::kPairBM);
-    p.n_blocks = (int32_t)(fuse_silu ? (N + bi::kHalfBN - 1) / bi::kHalfBN : (N + bi::kPairBN - 1) / bi::kPairBN);
     p.fuse_silu = fuse_silu;
-    p.k_blocks = (int32_t)((K + bi::kBK - 1) / bi::kBK);
     p.b_mn_major = b_layout == BI_B_KN ? 1 : 0;
     p.c_f32 = c_f32 ? 1 : 0;
     p.addend_mode = addend_mode;
@@ -323,26 +357,11 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
         return launch(bi::gemm_k0_fill_kernel, dim3((unsigned)blocks), dim3(256), 0, s, p);
     }
 
-    const int64_t tiles = (int64_t)p.m_blocks * p.n_blocks;
-    const uint32_t b_rows_box = bi::kHalfBN;
-    if (tiles > kI32Max) return BI_ERR_UNSUPPORTED;
-
-    CUtensorMap tm_a, tm_b;
-    // The A box copies the rows that exist: M rounded up to 8, at most the CTA's 128.  The tile,
-    // the MMA shape and every element's K order are the same for every M.
-    p.a_box_rows = (int32_t)(M >= bi::kBM ? bi::kBM : (M + 7) / 8 * 8);
-    st = encode_map(&tm_a, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda, bi::kBK, (uint32_t)p.a_box_rows);
-    if (st != BI_OK) return st;
-    if (b_layout == BI_B_NK)
-        st = encode_map(&tm_b, B, (uint64_t)K, (uint64_t)b_rows, (uint64_t)ldb, bi::kBK, b_rows_box);
-    else
-        st = encode_map(&tm_b, B, (uint64_t)b_rows, (uint64_t)K, (uint64_t)ldb, 64, bi::kBK);
-    if (st != BI_OK) return st;
-
-    const int64_t pairs = dev->gemm_clusters;
-    const int grid = 2 * (int)(tiles < pairs ? tiles : pairs);
-    return launch_pdl(bi::gemm_bf16_pair_kernel, dim3(grid), dim3(bi::kGemmThreads), (size_t)bi::kPairSmem, s,
-                      tm_a, tm_b, p);
+    // The tile configuration is a function of the output width N alone; every M of a given
+    // weight runs the same one.
+    if (N <= bi::kNarrowMaxN)
+        return launch_pair<bi::NarrowTile>(p, A, lda, B, ldb, b_layout, b_rows, dev->gemm_clusters_narrow, s);
+    return launch_pair<bi::WideTile>(p, A, lda, B, ldb, b_layout, b_rows, dev->gemm_clusters_wide, s);
 }
 
 __global__ void selftest_wait_kernel(int32_t *status, uint64_t limit_ns)
@@ -724,12 +743,13 @@ const char *bi_status_string(bi_status status)
     return "BI_ERR_UNKNOWN";
 }
 
-void bi_gemm_config(int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int32_t *mma_k)
+void bi_gemm_config(int64_t n, int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int32_t *mma_k)
 {
+    const bool narrow = n > 0 && n <= bi::kNarrowMaxN;
     if (bm) *bm = bi::kPairBM;
-    if (bn) *bn = bi::kPairBN;
-    if (stages) *stages = bi::kPStages;
-    if (bk) *bk = bi::kBK;
+    if (bn) *bn = narrow ? bi::NarrowTile::kBN : bi::WideTile::kBN;
+    if (stages) *stages = narrow ? bi::NarrowTile::kStages : bi::WideTile::kStages;
+    if (bk) *bk = narrow ? bi::NarrowTile::kStageK : bi::WideTile::kStageK;
     if (mma_k) *mma_k = bi::kMmaK;
 }
 
@@ -740,6 +760,6 @@ void bi_tensor_map_cache_stats(int64_t *hits, int64_t *misses)
     if (misses) *misses = (int64_t)g_map_misses;
 }
 
-int32_t bi_version(void) { return 200; }
+int32_t bi_version(void) { return 201; }
 
 }  // extern "C"

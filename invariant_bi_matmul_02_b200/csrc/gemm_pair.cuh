@@ -1,14 +1,20 @@
 // gemm_pair.cuh -- the batch-invariant bf16 GEMM: tcgen05 on CTA pairs (cta_group::2).
 //
-// One tile configuration for every call: a CTA pair (a 2-CTA cluster on one TPC)
-// owns a 256 x kPairBN output tile.  Each CTA stages, per 64-wide K slice, its own 128
-// rows of A and its own kPairBN/2 rows (columns of C) of B; the leader CTA issues
-// tcgen05.mma.cta_group::2 (M = 256, N = kPairBN, K = 16), which reads both CTAs'
-// shared memory and accumulates each CTA's 128 x kPairBN half of the tile in fp32 in
-// that CTA's tensor memory.  Per output element the order is the same as for any
-// single tcgen05 MMA: the first 16-wide K step overwrites the accumulator, every later
-// step adds in ascending K.  It depends only on K -- not on M, N, the row's position,
-// or which pair computes the tile.  No split-K, no stream-K, no tile switch.
+// A CTA pair (a 2-CTA cluster on one TPC) owns a 256 x BN output tile.  Each CTA stages,
+// per pipeline stage of SK values of K, its own 128 rows of A and its own BN/2 rows
+// (columns of C) of B; the leader CTA issues tcgen05.mma.cta_group::2 (M = 256, N = BN,
+// K = 16), which reads both CTAs' shared memory and accumulates each CTA's 128 x BN half
+// of the tile in fp32 in that CTA's tensor memory.  Per output element the order is the
+// same as for any single tcgen05 MMA: the first 16-wide K step overwrites the
+// accumulator, every later step adds in ascending K.  It depends only on K -- not on M,
+// N, the row's position, or which pair computes the tile.  No split-K, no stream-K.
+//
+// Two instantiations exist, and the host picks one from the weight's output width N
+// alone (never from M): the wide tile (BN = 256, SK = 64) and, for N <= 1024, the
+// narrow tile (BN = 128, SK = 128), whose more numerous tiles fill more of the GPU and
+// whose 8 MMAs per stage amortise the issuing thread's per-stage barrier wait and commit.
+// Both run the same 16-wide K steps in the same order, so a row's bits do not depend on
+// which one ran (the tests compare them).
 //
 // Pipeline, per CTA pair:
 //   full[s]   (leader)  armed by the leader's producer with both CTAs' bytes; both
@@ -30,33 +36,48 @@
 #include "gemm.cuh"
 #include "ptx.cuh"
 
-#ifndef BI_GEMM_PAIR_BN
-#define BI_GEMM_PAIR_BN 256  // the one tile width every call uses; other values exist for experiments only
-#endif
-
 namespace bi {
 
-constexpr int kPairBM = 256;                   // rows of C per CTA pair
-constexpr int kPairBN = BI_GEMM_PAIR_BN;       // columns of C per CTA pair
-constexpr int kHalfBN = kPairBN / 2;           // B rows staged by each CTA
-constexpr int kPABytes = 128 * kBK * 2;        // A slice per CTA
-constexpr int kPBBytes = kHalfBN * kBK * 2;    // B slice per CTA
-constexpr int kPStageBytes = kPABytes + kPBBytes;
-constexpr int kPStagesRaw = (kSmemBudget - kSmemMisc) / kPStageBytes;
-constexpr int kPStages = kPStagesRaw > 12 ? 12 : kPStagesRaw;
-constexpr int kPairSmem = kPStages * kPStageBytes + kSmemMisc;
-constexpr uint32_t kPairTmemCols = pow2_at_least(2 * kPairBN);
+constexpr int kPairBM = 256;  // rows of C per CTA pair
 
-static_assert(kPairBN % 128 == 0 && kPairBN <= 256, "pair tile N must be 128 or 256");
-static_assert(kPStages >= 2 && kPStages <= 32, "two to 32 pipeline stages (one producer lane per stage at the tail)");
-static_assert(kPairSmem + 1024 <= 256 * 1024, "shared addresses fit the 14-bit descriptor address field");
-static_assert(kPairTmemCols <= 512, "accumulators must fit in tensor memory");
-static_assert(kPairSmem > 114 * 1024, "one CTA per SM keeps the TMEM allocation uncontended");
+// Shared-memory layout of one tile configuration.  A stage holds SK / 64 swizzle atoms
+// (64 values of K, 128 bytes per row) of A and of B.
+template <int BN, int SK>
+struct PairTile {
+    static constexpr int kBN = BN;                      // columns of C per CTA pair
+    static constexpr int kHalf = BN / 2;                // B rows staged by each CTA
+    static constexpr int kStageK = SK;                  // K per pipeline stage
+    static constexpr int kAtoms = SK / kBK;             // 64-wide K atoms per stage
+    static constexpr int kAAtom = 128 * kBK * 2;        // one atom of A per CTA
+    static constexpr int kBAtom = kHalf * kBK * 2;      // one atom of B ([N, K] storage) per CTA
+    static constexpr int kABytes = kAtoms * kAAtom;     // A slice per CTA per stage
+    static constexpr int kBBytes = kAtoms * kBAtom;     // B slice per CTA per stage
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStagesRaw = (kSmemBudget - kSmemMisc) / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+    static constexpr int kSmem = kStages * kStageBytes + kSmemMisc;
+    static constexpr uint32_t kTmemCols = pow2_at_least(2 * BN);
 
+    static_assert(BN % 128 == 0 && BN <= 256, "pair tile N must be 128 or 256 ([K, N] B needs 64-column groups)");
+    static_assert(SK % kBK == 0 && SK >= kBK, "a stage holds whole swizzle atoms");
+    static_assert(kStages >= 2 && kStages <= 32, "two to 32 stages (one producer lane per stage at the tail)");
+    static_assert(kSmem + 1024 <= 256 * 1024, "shared addresses fit the 14-bit descriptor address field");
+    static_assert(kTmemCols <= 512, "accumulators must fit in tensor memory");
+    static_assert(kSmem > 114 * 1024, "one CTA per SM keeps the TMEM allocation uncontended");
+};
+
+using WideTile = PairTile<256, 64>;     // 7 stages of 64 K
+using NarrowTile = PairTile<128, 128>;  // 4 stages of 128 K
+constexpr int64_t kNarrowMaxN = 1024;   // output widths up to this use NarrowTile
+
+template <int BN, int SK>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
                           const __grid_constant__ CUtensorMap tm_b, const GemmParams p)
 {
+    using T = PairTile<BN, SK>;
+    constexpr int kPairBN = T::kBN, kHalfBN = T::kHalf, kPStages = T::kStages;
+    constexpr int kPABytes = T::kABytes, kPBBytes = T::kBBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     uint8_t *sA = smem;
@@ -91,7 +112,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         prefetch_tensor_map(&tm_b);
     }
     if (warp == 1) {
-        tmem_alloc_pair(tmem_holder, kPairTmemCols);
+        tmem_alloc_pair(tmem_holder, T::kTmemCols);
         tmem_relinquish_pair();
     }
     tc_fence_before_sync();
@@ -129,7 +150,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 // when no row of it is below M.  Shared-memory rows left uncopied feed only
                 // accumulator rows at or beyond M, which are never stored.
                 const bool a_hi = m_pair + 128 < p.M;
-                const uint32_t a_bytes = (uint32_t)p.a_box_rows * (kBK * 2);
+                const uint32_t a_bytes = (uint32_t)p.a_box_rows * (SK * 2);
                 const uint32_t stage_bytes = (a_hi ? 2u : 1u) * a_bytes + 2u * kPBBytes;
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim)) {
@@ -138,14 +159,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     }
                     if (leader) mbar_arrive_expect_tx(&full[stage], stage_bytes);
                     const uint32_t bar = map_to_rank(smem_addr(&full[stage]), 0);
-                    if (leader || a_hi) tma_load_2d_pair(sA + stage * kPABytes, &tm_a, bar, kb * kBK, m0);
+                    const int k0 = kb * SK;
+                    if (leader || a_hi) {
+#pragma unroll
+                        for (int at = 0; at < T::kAtoms; ++at)
+                            tma_load_2d_pair(sA + stage * kPABytes + at * T::kAAtom, &tm_a, bar, k0 + at * kBK, m0);
+                    }
                     uint8_t *dstB = sB + stage * kPBBytes;
                     if (p.b_mn_major) {
+                        // [K, N] storage: one box of 64 columns x SK values of K per 64-column group.
 #pragma unroll
                         for (int g = 0; g < kHalfBN / 64; ++g)
-                            tma_load_2d_pair(dstB + g * (64 * kBK * 2), &tm_b, bar, nh0 + g * 64, kb * kBK);
+                            tma_load_2d_pair(dstB + g * (64 * SK * 2), &tm_b, bar, nh0 + g * 64, k0);
                     } else {
-                        tma_load_2d_pair(dstB, &tm_b, bar, kb * kBK, nh0);
+#pragma unroll
+                        for (int at = 0; at < T::kAtoms; ++at)
+                            tma_load_2d_pair(dstB + at * T::kBAtom, &tm_b, bar, k0 + at * kBK, nh0);
                     }
                     advance(stage, phase, kPStages);
                 }
@@ -182,9 +211,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             // fits, so the sum never carries into the next field): one add per MMA instead of a
             // descriptor rebuilt on the issuing thread's critical path.
             const uint64_t a_desc0 = sw128_desc(smem_addr(sA), 16, 1024);
-            const uint64_t b_desc0 = p.b_mn_major ? sw128_desc(smem_addr(sB), 64 * kBK * 2, 1024)
+            const uint64_t b_desc0 = p.b_mn_major ? sw128_desc(smem_addr(sB), 64 * SK * 2, 1024)
                                                   : sw128_desc(smem_addr(sB), 16, 1024);
-            const uint32_t b_step = p.b_mn_major ? (kMmaK * 128) >> 4 : (kMmaK * 2) >> 4;
+            const bool b_mn = p.b_mn_major != 0;
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             bool ok = true;
             for (int tile = first; ok && tile < num_tiles; tile += stride) {
@@ -203,9 +232,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     const uint64_t a_desc = a_desc0 + stage * (uint32_t)(kPABytes >> 4);
                     const uint64_t b_desc = b_desc0 + stage * (uint32_t)(kPBBytes >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / kMmaK; ++kk)
-                        tc_mma_bf16_pair(d_tmem, a_desc + kk * ((kMmaK * 2) >> 4), b_desc + kk * b_step, idesc,
-                                         (kb | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < SK / kMmaK; ++kk) {
+                        // K step kk: atom kk / 4, 32-byte column (kk % 4) of its 128-byte rows;
+                        // [K, N] storage advances 16 rows of 128 bytes instead.
+                        constexpr int kPerAtom = kBK / kMmaK;
+                        const uint32_t in_atom = (kk % kPerAtom) * ((kMmaK * 2) >> 4);
+                        const uint32_t a_off = (kk / kPerAtom) * (T::kAAtom >> 4) + in_atom;
+                        const uint32_t b_off =
+                            b_mn ? kk * ((kMmaK * 128) >> 4) : (kk / kPerAtom) * (T::kBAtom >> 4) + in_atom;
+                        tc_mma_bf16_pair(d_tmem, a_desc + a_off, b_desc + b_off, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
                     tc_commit_pair_mc(&empty[stage], 0x3);
                     advance(stage, phase, kPStages);
                 }
@@ -278,7 +314,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     cluster_sync_all();  // no CTA leaves while its peer may still signal its barriers
     if (warp == 1) {
         tc_fence_after_sync();
-        tmem_dealloc_pair(tmem_base, kPairTmemCols);
+        tmem_dealloc_pair(tmem_base, T::kTmemCols);
     }
 }
 

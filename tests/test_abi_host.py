@@ -43,10 +43,17 @@ def test_status_strings_and_config(lib):
     assert binding.status_string(binding.BI_OK) == "BI_OK"
     assert binding.status_string(binding.BI_ERR_TIMEOUT) == "BI_ERR_TIMEOUT"
     assert binding.status_string(99) == "BI_ERR_UNKNOWN"
-    cfg = binding.bi_gemm_config()
-    assert cfg["bm"] == 256 and cfg["bk"] == 64 and cfg["mma_k"] == 16  # a CTA pair's tile
-    assert cfg["bn"] in (128, 256) and cfg["stages"] >= 2
-    assert binding.bi_version() >= 100
+    wide = binding.bi_gemm_config()
+    assert wide == binding.bi_gemm_config(151936) == binding.bi_gemm_config(1025)
+    assert wide["bm"] == 256 and wide["bn"] == 256 and wide["bk"] == 64 and wide["mma_k"] == 16
+    narrow = binding.bi_gemm_config(1024)
+    assert narrow == binding.bi_gemm_config(1)
+    assert narrow["bm"] == 256 and narrow["bn"] == 128 and narrow["bk"] == 128 and narrow["mma_k"] == 16
+    # every stage fits in the 227 KB a CTA may use, with room for the barriers
+    for cfg in (wide, narrow):
+        assert cfg["stages"] >= 2
+        assert cfg["stages"] * (128 + cfg["bn"] // 2) * cfg["bk"] * 2 <= 227 * 1024 - 1536
+    assert binding.bi_version() >= 201
 
 
 NULL = None

@@ -222,6 +222,36 @@ def test_batch_invariance_sweep_wide_and_deep(K, N):
             assert same_bits(out, ref[idx]), f"K={K} N={N} M={M}: a row differs from M=1"
 
 
+@pytest.mark.parametrize("layout", ["nk", "kn"])
+@pytest.mark.parametrize("K", [4096, 4104])
+def test_tile_width_does_not_change_bits(K, layout):
+    """Outputs up to 1024 columns wide run the 128-column tile with 128-deep stages, wider ones
+    the 256-column tile with 64-deep stages.  Both take the same 16-wide K steps in ascending
+    order, so the first 1024 columns of a 1280-column product (wide tile) equal, bit for bit,
+    the product with only those 1024 weight rows (narrow tile) -- for plain, bias and fused
+    SiLU * up outputs, at ragged M and K."""
+    assert bi.bi_gemm_config(1024)["bn"] != bi.bi_gemm_config(1280)["bn"]
+    w = weight(250, 1280, K, "nk").to(DEV)
+    gate, up = w, weight(251, 1280, K, "nk").to(DEV)
+    bias = inputs.bias(252, 1280).to(DEV)
+    wk = w if layout == "nk" else w.t().contiguous()
+    for M in (1, 77, 300):
+        a = inputs.rows_normal(253, 0, M, K).to(DEV)
+        wide = bi.bi_matmul(a, wk, layout)
+        narrow = bi.bi_matmul(a, wk[:1024] if layout == "nk" else wk[:, :1024], layout)
+        assert same_bits(wide[:, :1024], narrow), f"matmul M={M} K={K} {layout}"
+        wide_b = bi.bi_addmm(bias, a, wk, layout)
+        narrow_b = bi.bi_addmm(bias[:1024], a, wk[:1024] if layout == "nk" else wk[:, :1024], layout)
+        assert same_bits(wide_b[:, :1024], narrow_b), f"addmm M={M} K={K} {layout}"
+        gu_wide = torch.cat([gate, up])
+        gu_narrow = torch.cat([gate[:1024], up[:1024]])
+        if layout == "kn":
+            gu_wide, gu_narrow = gu_wide.t().contiguous(), gu_narrow.t().contiguous()
+        h_wide = bi.bi_matmul_silu_mul(a, gu_wide, layout)
+        h_narrow = bi.bi_matmul_silu_mul(a, gu_narrow, layout)
+        assert same_bits(h_wide[:, :1024], h_narrow), f"fused M={M} K={K} {layout}"
+
+
 def test_lm_head_logits_invariance():
     """LM-head logits [M, 151936] at M in {1, 8, 64, 256, 1024}: each row equals the row
     computed alone, bit for bit, at every position of two windows of a permutation."""
