@@ -142,8 +142,8 @@ __device__ __forceinline__ bool wait_flag_at_least(volatile int *flag, int v, vo
 // 32w .. 32w+31 of the split).  Scores: S = Q . K^T with Q the group's heads padded to 16 rows;
 // every score accumulates its eight 16-wide D steps in ascending order.  Per head, the split's
 // maximum and sum of exp(s - max) (fp32) come from fixed trees: a thread's own values in
-// order, the lane quad (xor 1, 2), the warps in order.  Weighted sums: O_w = P_w . V_w with P
-// split into two bf16 terms (about 16 significant bits), two 16-token steps in ascending order;
+// order, the lane quad (xor 1, 2), the warps in order.  Weighted sums: O_w^T = V_w^T . P_w^T with
+// P split into two bf16 terms (about 16 significant bits), two 16-token steps in ascending order;
 // the four warps' O_w are added in warp order.  Value rows past the sequence's end are zeroed in
 // shared memory before use, so stale cache contents never reach the sums.
 template <int G>  // query heads per kv head (1, 2, 4 or 8)
@@ -154,8 +154,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     extern __shared__ uint8_t attn_raw[];
     uint8_t *smem = attn_raw + ((1024u - (smem_addr(attn_raw) & 1023u)) & 1023u);
     __shared__ uint64_t kfull[kAttnStages], vfull[kAttnStages], empty[kAttnStages];
-    __shared__ float red_m_all[kAttnGroups][kAttnConsumers][16];  // per-warp maxima of the 16 rows
-    __shared__ float red_s_all[kAttnGroups][kAttnConsumers][16];  // per-warp sums of exp
+    __shared__ float red_m_all[kAttnGroups][kAttnConsumers][8];  // per-warp maxima of the 8 head rows
+    __shared__ float red_s_all[kAttnGroups][kAttnConsumers][8];  // per-warp sums of exp
     __shared__ int abort_flag_s;
     __shared__ int progress_s[kAttnGroups];  // items a consumer group has started (local index + 1)
     volatile int *abort_flag = &abort_flag_s;
@@ -233,8 +233,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int cw = (warp - 1) % kAttnConsumers, ct = threadIdx.x - 32 - 32 * kAttnConsumers * grp;
         const int bar_id = 1 + grp;
         const int gid = lane >> 2, tig = lane & 3;
-        float (*red_m)[16] = red_m_all[grp];
-        float (*red_s)[16] = red_s_all[grp];
+        float (*red_m)[8] = red_m_all[grp];
+        float (*red_s)[8] = red_s_all[grp];
         uint32_t local = 0;
         for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
             const int split = (int)(it % p.S), g = (int)((it / p.S) % p.Hkv), b = (int)(it / (p.S * p.Hkv));
@@ -249,10 +249,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const uint8_t *ks = k_tile(stage);
             uint8_t *vs = v_tile(stage);
             const __nv_bfloat16 *qs = q_rows(stage);
-            // The stage's previous use belongs to the other group.  Once that group has started
-            // this group's preceding item it has finished that previous use, so the stage's
-            // barriers are at most one phase from the one wanted and a parity wait is exact.
-            bool ok = mine == 0 || wait_flag_at_least(&progress[grp ^ 1], (int)mine, abort_flag, p.status, lim);
+            // Items are started in order: once the group before this one has started item mine - 1,
+            // every earlier item -- the stage's previous use among them -- has started, so that use's
+            // copies have landed and the stage's barriers are at most one phase from the one
+            // wanted: a parity wait is exact.
+            const int prev_grp = grp == 0 ? kAttnGroups - 1 : grp - 1;
+            bool ok = mine == 0 || wait_flag_at_least(&progress[prev_grp], (int)mine, abort_flag, p.status, lim);
             ok = ok && wait_bounded(&kfull[stage], use & 1u, abort_flag, p.status, lim);
             if (!consumers_all(bar_id, ok)) break;
             if (ct == 0) progress[grp] = (int)mine + 1;
@@ -285,46 +287,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     acc[nt][e] = tok < n_tok ? acc[nt][e] * p.scale : kNegInf;
                 }
 
-            // ---- per-head max: own values in order, quad butterfly, warps in order
-            float mx[2];
+            // ---- per-head max: own values in order, quad butterfly, warps in order.  Only rows
+            // 0..7 (e = 0, 1) hold heads; rows 8..15 are padding and are not used.
+            {
+                float m = acc[0][0];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float m = acc[0][2 * h];
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) m = fmaxf(fmaxf(m, acc[nt][2 * h]), acc[nt][2 * h + 1]);
+                for (int nt = 0; nt < 4; ++nt) m = fmaxf(fmaxf(m, acc[nt][0]), acc[nt][1]);
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-                mx[h] = m;
-            }
-            if (tig == 0) {
-                red_m[cw][gid] = mx[0];
-                red_m[cw][gid + 8] = mx[1];
+                if (tig == 0) red_m[cw][gid] = m;
             }
             consumers_sync(bar_id);  // every warp's maxima are posted; the K tile is no longer read
             // ---- p = exp(s - max); per-head sums by the same trees.  Each thread folds the warps'
             // maxima of its two heads itself, in warp order.
-            float sum[2];
+            {
+                float m = red_m[0][gid];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float m = red_m[0][gid + 8 * h];
-#pragma unroll
-                for (int w = 1; w < kAttnConsumers; ++w) m = fmaxf(m, red_m[w][gid + 8 * h]);
+                for (int w = 1; w < kAttnConsumers; ++w) m = fmaxf(m, red_m[w][gid]);
                 float l = 0.0f;
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        float &x = acc[nt][2 * h + e];
+                        float &x = acc[nt][e];
                         x = x == kNegInf ? 0.0f : __expf(x - m);
                         l = __fadd_rn(l, x);
                     }
                 l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 1));
                 l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 2));
-                sum[h] = l;
-            }
-            if (tig == 0) {
-                red_s[cw][gid] = sum[0];
-                red_s[cw][gid + 8] = sum[1];
+                if (tig == 0) red_s[cw][gid] = l;
             }
             if (!consumers_all(bar_id, wait_bounded(&vfull[stage], use & 1u, abort_flag, p.status, lim))) break;
             if (n_tok < kAttnSplit) {
@@ -335,50 +326,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 consumers_sync(bar_id);
             }
 
-            // ---- O_w = P_w . V_w: A from the score tiles (two 8-token tiles per 16-token step)
-            float o[kAttnD / 8][4];
+            // ---- O_w^T = V_w^T . P_w^T: d on the MMA's M (8 tiles of 16 rows), the group's heads on
+            // N (8 columns; columns G .. 7 are padding), tokens on K in two 16-token steps in
+            // ascending order.  Rows 0..7 of the score tiles (e = 0, 1: head gid, tokens 2 tig and
+            // 2 tig + 1 of tiles 2j and 2j + 1) are exactly the B fragments of P^T for step j, and
+            // the transposed ldmatrix of V yields the A fragments of V^T, so nothing is reshuffled.
+            // P enters as two bf16 terms, hi = bf16(p) and lo = bf16(p - hi), so the weights keep
+            // about 16 significant bits; per 16-token step hi is added first.
+            float o[kAttnD / 16][4];  // o[mt]: d 16 mt + gid (+ 8), heads 2 tig, 2 tig + 1
 #pragma unroll
-            for (int dt = 0; dt < kAttnD / 8; ++dt)
+            for (int mt = 0; mt < kAttnD / 16; ++mt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) o[dt][e] = 0.0f;
-            // P enters the tensor cores as two bf16 terms, hi = bf16(p) and lo = bf16(p - hi), so
-            // the weights keep about 16 significant bits; per 16-token step hi is added first.
+                for (int e = 0; e < 4; ++e) o[mt][e] = 0.0f;
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const float *p0 = acc[2 * j], *p1 = acc[2 * j + 1];
-                const float pv[8] = {p0[0], p0[1], p0[2], p0[3], p1[0], p1[1], p1[2], p1[3]};
-                float hi[8], lo[8];
+                const float pv[4] = {acc[2 * j][0], acc[2 * j][1], acc[2 * j + 1][0], acc[2 * j + 1][1]};
+                float hi[4], lo[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
+                for (int e = 0; e < 4; ++e) {
                     hi[e] = __bfloat162float(__float2bfloat16_rn(pv[e]));
                     lo[e] = pv[e] - hi[e];
                 }
-                const uint32_t pa_hi[4] = {pack_bf16(hi[0], hi[1]), pack_bf16(hi[2], hi[3]), pack_bf16(hi[4], hi[5]),
-                                           pack_bf16(hi[6], hi[7])};
-                const uint32_t pa_lo[4] = {pack_bf16(lo[0], lo[1]), pack_bf16(lo[2], lo[3]), pack_bf16(lo[4], lo[5]),
-                                           pack_bf16(lo[6], lo[7])};
+                const uint32_t pb_hi0 = pack_bf16(hi[0], hi[1]), pb_hi1 = pack_bf16(hi[2], hi[3]);
+                const uint32_t pb_lo0 = pack_bf16(lo[0], lo[1]), pb_lo1 = pack_bf16(lo[2], lo[3]);
                 const int tok0 = 32 * cw + 16 * j;
 #pragma unroll
                 for (int dt = 0; dt < kAttnD / 8; dt += 2) {
-                    // matrices (transposed): (tokens 0-7, d tile dt), (8-15, dt), (0-7, dt+1), (8-15, dt+1)
+                    // matrices (transposed): (tokens 0-7, d tile dt), (8-15, dt), (0-7, dt+1), (8-15, dt+1);
+                    // as A of V^T (rows d, columns tokens): a0 = (dt, 0-7), a1 = (dt+1, 0-7),
+                    // a2 = (dt, 8-15), a3 = (dt+1, 8-15).
                     uint32_t vf[4];
                     ldsm_x4_trans(vf, kv_chunk(vs, tok0 + (lane & 7) + 8 * ((lane >> 3) & 1), dt + (lane >> 4)));
-                    mma_16816_bf16(o[dt], pa_hi, vf[0], vf[1]);
-                    mma_16816_bf16(o[dt], pa_lo, vf[0], vf[1]);
-                    mma_16816_bf16(o[dt + 1], pa_hi, vf[2], vf[3]);
-                    mma_16816_bf16(o[dt + 1], pa_lo, vf[2], vf[3]);
+                    const uint32_t va[4] = {vf[0], vf[2], vf[1], vf[3]};
+                    mma_16816_bf16(o[dt / 2], va, pb_hi0, pb_hi1);
+                    mma_16816_bf16(o[dt / 2], va, pb_lo0, pb_lo1);
                 }
             }
             // The K tile (read by every warp before the maxima barrier) holds the per-warp outputs,
-            // rows kAttnOStride floats apart: a store's lanes cover rows 0..3 (x 4 columns two
-            // apart) in distinct banks; rows 4..7 (group size 8) share banks with rows 0..3.
+            // rows kAttnOStride floats apart.  A store's lanes cover d 16 mt + gid (+ 8) of heads
+            // 2 tig (+ 1): for up to four heads, rows 0 and 2 (or 1 and 3) sit 16 banks apart, so the
+            // 16 lanes that store land in distinct banks; eight heads share banks two ways.
             float *so = reinterpret_cast<float *>(const_cast<uint8_t *>(ks));
 #pragma unroll
-            for (int dt = 0; dt < kAttnD / 8; ++dt)
+            for (int mt = 0; mt < kAttnD / 16; ++mt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int row = gid + 8 * (e >> 1), col = 8 * dt + 2 * tig + (e & 1);
-                    if (row < G) so[(cw * kAttnMaxGroup + row) * kAttnOStride + col] = o[dt][e];
+                    const int head = 2 * tig + (e & 1), col = 16 * mt + gid + 8 * (e >> 1);
+                    if (head < G) so[(cw * kAttnMaxGroup + head) * kAttnOStride + col] = o[mt][e];
                 }
             consumers_sync(bar_id);
 #pragma unroll
