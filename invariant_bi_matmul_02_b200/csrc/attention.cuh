@@ -74,10 +74,13 @@ __device__ __forceinline__ const uint8_t *kv_chunk(const uint8_t *tile, int row,
     return tile + (chunk >> 3) * kAttnBoxBytes + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
 }
 
+constexpr int kAttnLensCached = 4096;  // sequence lengths launch 1 keeps in shared memory
+
 // Sequence length as the kernels use it: a value outside 1 .. Lmax is clamped (and reported).
-__device__ __forceinline__ int64_t attn_len(const AttnParams &p, int b, bool report)
+// `cached` holds lens[0 .. kAttnLensCached) when non-null.
+__device__ __forceinline__ int64_t attn_len(const AttnParams &p, int b, bool report, const int32_t *cached = nullptr)
 {
-    int64_t L = p.lens[b];
+    int64_t L = cached && b < kAttnLensCached ? cached[b] : p.lens[b];
     if (L < 1 || L > p.Lmax) {
         if (report) *reinterpret_cast<volatile int32_t *>(p.status) = 1;  // BI_ERR_INVALID_ARG
         L = L < 1 ? 1 : p.Lmax;
@@ -158,6 +161,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __shared__ float red_s_all[kAttnGroups][kAttnConsumers][8];  // per-warp sums of exp
     __shared__ int abort_flag_s;
     __shared__ int progress_s[kAttnGroups];  // items a consumer group has started (local index + 1)
+    // Every role walks all of the CTA's items and needs each one's sequence length: read once here
+    // rather than from global memory per item.
+    __shared__ int32_t lens_s[kAttnLensCached];
     volatile int *abort_flag = &abort_flag_s;
     volatile int *progress = progress_s;
 
@@ -185,8 +191,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncthreads();
     griddep_wait();  // the previous kernel's output (q, the caches, the lengths) is complete
     griddep_launch_dependents();
+    for (int i = threadIdx.x; i < p.B && i < kAttnLensCached; i += kAttnThreads) lens_s[i] = p.lens[i];
+    __syncthreads();
 
-    const int64_t items = (int64_t)p.B * p.Hkv * p.S;
+    // The host guarantees B * Hkv * S < 2^31, so item indices and their coordinates are 32-bit.
+    const uint32_t items = (uint32_t)p.B * (uint32_t)p.Hkv * (uint32_t)p.S;
+    const uint32_t n_splits = (uint32_t)p.S, n_kv = (uint32_t)p.Hkv;
     const uint64_t lim = p.wait_limit_ns;
 
     if (warp == 0) {
@@ -195,10 +205,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t stage = 0, phase = 0;
             int issued = 0;
             bool ok = true;
-            for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
-                const int split = (int)(it % p.S), g = (int)((it / p.S) % p.Hkv), b = (int)(it / (p.S * p.Hkv));
+            for (uint32_t it = blockIdx.x; it < items; it += gridDim.x) {
+                const uint32_t sg = it / n_splits;
+                const int split = (int)(it - sg * n_splits), g = (int)(sg % n_kv), b = (int)(sg / n_kv);
                 const int64_t t0 = (int64_t)split * kAttnSplit;
-                if (t0 >= attn_len(p, b, false)) continue;
+                if (t0 >= attn_len(p, b, false, lens_s)) continue;
                 if (!(ok = wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim))) break;
                 mbar_arrive_expect_tx(&kfull[stage], G * kAttnD * 2 + kAttnTileBytes);
                 for (int j = 0; j < G; ++j)
@@ -236,10 +247,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float (*red_m)[8] = red_m_all[grp];
         float (*red_s)[8] = red_s_all[grp];
         uint32_t local = 0;
-        for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
-            const int split = (int)(it % p.S), g = (int)((it / p.S) % p.Hkv), b = (int)(it / (p.S * p.Hkv));
+        for (uint32_t it = blockIdx.x; it < items; it += gridDim.x) {
+            const uint32_t sg = it / n_splits;
+            const int split = (int)(it - sg * n_splits), g = (int)(sg % n_kv), b = (int)(sg / n_kv);
             const int64_t t0 = (int64_t)split * kAttnSplit;
-            const int64_t L = attn_len(p, b, ct == 0 && grp == 0 && split == 0);
+            const int64_t L = attn_len(p, b, ct == 0 && grp == 0 && split == 0, lens_s);
             if (t0 >= L) continue;
             const uint32_t mine = local++;
             if (mine % kAttnGroups != (uint32_t)grp) continue;

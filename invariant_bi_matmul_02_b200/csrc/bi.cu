@@ -641,6 +641,7 @@ bi_status bi_decode_attention(const void *q, const void *k_cache, const void *v_
     const int64_t group = Hq / Hkv;
     if (D != bi::kAttnD || (group != 1 && group != 2 && group != 4 && group != 8)) return BI_ERR_UNSUPPORTED;
     if (B > 65535 || Hkv > 65535 || Hq > 65535 || bi::attn_splits(Lmax) > kI32Max) return BI_ERR_UNSUPPORTED;
+    if (B * Hkv * bi::attn_splits(Lmax) > kI32Max) return BI_ERR_UNSUPPORTED;  // work items are 32-bit indices
     if (B == 0) return BI_OK;
     if (!q || !k_cache || !v_cache || !seq_lens || !out || !scratch) return BI_ERR_INVALID_ARG;
     if (scratch_bytes < bi_decode_attention_scratch_bytes(B, Hq, D, Lmax)) return BI_ERR_INVALID_ARG;

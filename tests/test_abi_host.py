@@ -92,6 +92,13 @@ def test_host_validation_without_a_gpu(lib):
     # fused gate/up with [K, 2F] weights: the up half's first column F must be a multiple of 8
     assert lib.bi_matmul_silu_mul(fake, 200, fake, 1000, 0, fake, 504, 77, 500, 200, NULL) == A
     assert lib.bi_selftest_wait_timeout(10, NULL) == I
+    # decode attention: shapes the kernel does not take are refused before any pointer is read
+    da = lib.bi_decode_attention
+    assert da(fake, fake, fake, fake, fake, 2, 32, 8, 64, 128, 1.0, fake, 1 << 20, NULL) == U  # D != 128
+    assert da(fake, fake, fake, fake, fake, 2, 24, 8, 128, 128, 1.0, fake, 1 << 20, NULL) == U  # group 3
+    assert da(fake, fake, fake, fake, fake, 2, 30, 8, 128, 128, 1.0, fake, 1 << 20, NULL) == I  # Hq % Hkv
+    # B * Hkv * splits must stay below 2^31 (work items are 32-bit indices)
+    assert da(fake, fake, fake, fake, fake, 60000, 40000, 40000, 128, 128, 1.0, fake, 1 << 20, NULL) == U
     v = ctypes.c_int32(0)
     assert lib.bi_get_device_status(NULL, None) == I
 
