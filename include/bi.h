@@ -261,12 +261,14 @@ bi_status bi_silu_mul(const void *gu, void *h, int64_t M, int64_t F, void *strea
  * "What does temperature zero actually guarantee?" (attention is not batch-invariant by
  * default).
  *
- * Batch invariance: each sequence's cache is cut into splits of 128 tokens, a cut fixed by
+ * Batch invariance: each sequence's cache is cut into splits of 512 tokens, a cut fixed by
  * its own length (never by the batch size or the GPU's occupancy, unlike split-KV decoding
  * that sizes splits to fill the machine).  Per split, scores are fp32 dot products over D in
- * ascending order, the split's max and sum of exp(s - max) come from fixed trees, and the
- * weighted value sums run over tokens in ascending order; the splits are then folded in
- * ascending order.  A sequence's output does not depend on the other sequences in the batch.
+ * ascending order; the split is taken in four 128-token pieces in ascending order, each
+ * raising a running maximum by a fixed tree and rescaling the sums of exp(s - max) and the
+ * weighted value sums accumulated so far, which run over tokens in ascending order; the
+ * splits are then folded in ascending order.  A sequence's output does not depend on the
+ * other sequences in the batch.
  *
  *   q        device, bf16, [B, Hq, D];  out device, bf16, [B, Hq, D] (one rounding).
  *   k_cache, v_cache  device, bf16, [B, Lmax, Hkv, D]; only the first seq_lens[b] tokens of

@@ -9,12 +9,14 @@
 // not on the batch it is decoded in, its position there, or which CTA computes a split.
 //
 // Launch 1 is a persistent, warp-specialised kernel: one CTA per SM walks the (split, kv head,
-// sequence) work items round-robin.  Its producer warp stages each item's query rows (bulk
-// copies) and its K and V tiles (4-D TMA tensor loads, 128-byte swizzle) into a ring of
-// kAttnStages shared-memory stages, each completing on mbarriers.  Two groups of four consumer
-// warps take the CTA's items alternately, so one group's compute overlaps the other's and the
-// loads of the next items.  The cache streams from HBM without a gap between items.  The
-// arithmetic of an item is fixed and does not depend on the ring, the group or the CTA.
+// sequence) work items round-robin.  Its producer warp stages each split, kAttnChunk tokens at a
+// time, as the group's query rows (bulk copies) and K and V tiles (4-D TMA tensor loads, 128-byte
+// swizzle) into a ring of kAttnStages shared-memory stages, each completing on mbarriers.  Two
+// groups of four consumer warps take the CTA's splits alternately, so one group's compute
+// overlaps the other's and the loads of the next stages.  The cache streams from HBM without a
+// gap between items.  A split of kAttnSplit tokens keeps the partial results (written by launch 1,
+// read by launch 2) at a few percent of the cache's bytes.  The arithmetic of a split is fixed and
+// does not depend on the ring, the group or the CTA.
 //
 // Layouts (row-major, bf16): q [B, Hq, D]; k, v [B, Lmax, Hkv, D]; out [B, Hq, D].  Query
 // head h reads kv head h / (Hq / Hkv).  D = 128.
@@ -29,20 +31,22 @@
 namespace bi {
 
 constexpr int kAttnD = 128;
-constexpr int kAttnSplit = 128;                         // tokens per split
-constexpr int kAttnConsumers = 4;                       // consumer warps per group, 32 tokens each
-constexpr int kAttnGroups = 2;                          // consumer groups, alternate items
+constexpr int kAttnChunk = 128;                         // tokens per ring stage
+constexpr int kAttnSplit = 4 * kAttnChunk;              // tokens per split (one partial result)
+constexpr int kAttnConsumers = 4;                       // consumer warps per group, 32 tokens of a stage each
+constexpr int kAttnGroups = 2;                          // consumer groups, alternate splits
 constexpr int kAttnThreads = 32 * (1 + kAttnGroups * kAttnConsumers);  // warp 0 produces
 constexpr int kAttnMaxGroup = 8;                        // query heads per kv head
 constexpr int kAttnStages = 3;
 constexpr int kAttnQStride = kAttnD + 8;                // padded query row (bf16): conflict-free ldmatrix
-constexpr int kAttnBoxBytes = kAttnSplit * 64 * 2;      // one TMA box: 128 tokens x 64 d (16 KB)
+constexpr int kAttnBoxBytes = kAttnChunk * 64 * 2;      // one TMA box: 128 tokens x 64 d (16 KB)
 constexpr int kAttnTileBytes = 2 * kAttnBoxBytes;       // K or V of one split: 32 KB
 constexpr int kAttnQBytes = 16 * kAttnQStride * 2;      // query rows of a group, padded to 16 rows
 constexpr int kAttnStageBytes = 2 * kAttnTileBytes + ((kAttnQBytes + 1023) / 1024) * 1024;
 constexpr int kAttnSmem = kAttnStages * kAttnStageBytes + 1024;  // + alignment slack
 
 constexpr int kAttnOStride = kAttnD + 8;                // per-warp output rows in shared memory (floats)
+static_assert(kAttnChunk == 32 * kAttnConsumers, "each consumer warp owns 32 token rows of a stage");
 static_assert(kAttnConsumers * kAttnMaxGroup * kAttnOStride * 4 <= kAttnTileBytes,
               "per-warp partial outputs fit in the K tile they replace");
 
@@ -59,6 +63,11 @@ struct AttnParams {
 };
 
 __host__ __device__ inline int64_t attn_splits(int64_t L) { return (L + kAttnSplit - 1) / kAttnSplit; }
+// Ring stages of a split that starts `rest` tokens before the sequence's end (rest >= 1).
+__host__ __device__ inline int attn_chunks(int64_t rest)
+{
+    return rest >= kAttnSplit ? kAttnSplit / kAttnChunk : (int)((rest + kAttnChunk - 1) / kAttnChunk);
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
@@ -141,14 +150,18 @@ __device__ __forceinline__ bool wait_flag_at_least(volatile int *flag, int v, vo
 // shared memory.  Work item i: split i % S, kv head (i / S) % Hkv, sequence i / (S Hkv); items
 // past their sequence's length have no partial and are skipped by every role alike.
 //
-// Arithmetic per item (mma.sync m16n8k16, bf16 in, fp32 accumulate; warp w owns tokens
-// 32w .. 32w+31 of the split).  Scores: S = Q . K^T with Q the group's heads padded to 16 rows;
-// every score accumulates its eight 16-wide D steps in ascending order.  Per head, the split's
-// maximum and sum of exp(s - max) (fp32) come from fixed trees: a thread's own values in
-// order, the lane quad (xor 1, 2), the warps in order.  Weighted sums: O_w^T = V_w^T . P_w^T with
-// P split into two bf16 terms (about 16 significant bits), two 16-token steps in ascending order;
-// the four warps' O_w are added in warp order.  Value rows past the sequence's end are zeroed in
-// shared memory before use, so stale cache contents never reach the sums.
+// Arithmetic per split (mma.sync m16n8k16, bf16 in, fp32 accumulate), over its stages of
+// kAttnChunk tokens in ascending order; warp w owns tokens 32w .. 32w+31 of each stage.  Scores:
+// S = Q . K^T with Q the group's heads padded to 16 rows; every score accumulates its eight
+// 16-wide D steps in ascending order.  Per head and stage, the stage's maximum comes from a fixed
+// tree (a thread's own values in order, the lane quad xor 1, 2, the warps in order) and raises the
+// running maximum m; what is accumulated so far -- each thread's sum of exp(s - m) and each warp's
+// weighted sums -- is multiplied by exp(m_old - m) (0 at the first stage), then the stage's
+// exp(s - m) are added in order.  Weighted sums: O_w^T += V_w^T . P_w^T with P split into two bf16
+// terms (about 16 significant bits), two 16-token steps in ascending order.  At the split's end the
+// threads' sums meet in the lane quad (xor 1, 2), then the four warps' sums and O_w are added in
+// warp order.  Value rows past the sequence's end are zeroed in shared memory before use, so stale
+// cache contents never reach the sums.
 template <int G>  // query heads per kv head (1, 2, 4 or 8)
 __global__ void __launch_bounds__(kAttnThreads, 1)
     decode_attention_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -160,12 +173,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __shared__ float red_m_all[kAttnGroups][kAttnConsumers][8];  // per-warp maxima of the 8 head rows
     __shared__ float red_s_all[kAttnGroups][kAttnConsumers][8];  // per-warp sums of exp
     __shared__ int abort_flag_s;
-    __shared__ int progress_s[kAttnGroups];  // items a consumer group has started (local index + 1)
+    __shared__ int slot_use_s[kAttnStages];  // uses of each ring slot that a consumer group has passed
     // Every role walks all of the CTA's items and needs each one's sequence length: read once here
     // rather than from global memory per item.
     __shared__ int32_t lens_s[kAttnLensCached];
     volatile int *abort_flag = &abort_flag_s;
-    volatile int *progress = progress_s;
+    volatile int *slot_use = slot_use_s;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto k_tile = [&](int s) { return smem + s * kAttnStageBytes; };
@@ -179,7 +192,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(&empty[s], kAttnConsumers);  // one arrival per consumer warp
         }
         abort_flag_s = 0;
-        for (int g = 0; g < kAttnGroups; ++g) progress_s[g] = 0;
+        for (int st = 0; st < kAttnStages; ++st) slot_use_s[st] = 0;
         fence_mbar_init();
     }
     // Query rows G .. 15 of every stage stay zero (the copies fill rows 0 .. G-1 only).
@@ -205,27 +218,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t stage = 0, phase = 0;
             int issued = 0;
             bool ok = true;
-            for (uint32_t it = blockIdx.x; it < items; it += gridDim.x) {
+            for (uint32_t it = blockIdx.x; ok && it < items; it += gridDim.x) {
                 const uint32_t sg = it / n_splits;
                 const int split = (int)(it - sg * n_splits), g = (int)(sg % n_kv), b = (int)(sg / n_kv);
-                const int64_t t0 = (int64_t)split * kAttnSplit;
-                if (t0 >= attn_len(p, b, false, lens_s)) continue;
-                if (!(ok = wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim))) break;
-                mbar_arrive_expect_tx(&kfull[stage], G * kAttnD * 2 + kAttnTileBytes);
-                for (int j = 0; j < G; ++j)
-                    bulk_load(q_rows(stage) + j * kAttnQStride, p.q + ((int64_t)b * p.Hq + (int64_t)g * G + j) * kAttnD,
-                              kAttnD * 2, &kfull[stage]);
-                tma_load_4d(k_tile(stage), &tm_k, &kfull[stage], 0, g, (int32_t)t0, b);
-                tma_load_4d(k_tile(stage) + kAttnBoxBytes, &tm_k, &kfull[stage], 64, g, (int32_t)t0, b);
-                mbar_arrive_expect_tx(&vfull[stage], kAttnTileBytes);
-                tma_load_4d(v_tile(stage), &tm_v, &vfull[stage], 0, g, (int32_t)t0, b);
-                tma_load_4d(v_tile(stage) + kAttnBoxBytes, &tm_v, &vfull[stage], 64, g, (int32_t)t0, b);
-                ++issued;
-                advance(stage, phase, kAttnStages);
+                const int64_t t0 = (int64_t)split * kAttnSplit, L = attn_len(p, b, false, lens_s);
+                if (t0 >= L) continue;
+                // The split's stages in token order; each carries the group's query rows too.
+                const int nc = attn_chunks(L - t0);
+                for (int c = 0; c < nc; ++c) {
+                    const int32_t tc = (int32_t)(t0 + (int64_t)c * kAttnChunk);
+                    if (!(ok = wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim))) break;
+                    mbar_arrive_expect_tx(&kfull[stage], G * kAttnD * 2 + kAttnTileBytes);
+                    for (int j = 0; j < G; ++j)
+                        bulk_load(q_rows(stage) + j * kAttnQStride,
+                                  p.q + ((int64_t)b * p.Hq + (int64_t)g * G + j) * kAttnD, kAttnD * 2, &kfull[stage]);
+                    tma_load_4d(k_tile(stage), &tm_k, &kfull[stage], 0, g, tc, b);
+                    tma_load_4d(k_tile(stage) + kAttnBoxBytes, &tm_k, &kfull[stage], 64, g, tc, b);
+                    mbar_arrive_expect_tx(&vfull[stage], kAttnTileBytes);
+                    tma_load_4d(v_tile(stage), &tm_v, &vfull[stage], 0, g, tc, b);
+                    tma_load_4d(v_tile(stage) + kAttnBoxBytes, &tm_v, &vfull[stage], 64, g, tc, b);
+                    ++issued;
+                    advance(stage, phase, kAttnStages);
+                }
             }
             if (!ok) {
                 // A wait ran out: let every copy already issued land before shared memory goes
-                // away (the last kAttnStages items at most).
+                // away (the last kAttnStages stages at most).
                 for (int j = issued > kAttnStages ? issued - kAttnStages : 0; j < issued; ++j) {
                     const uint32_t par = (uint32_t)(j / kAttnStages) & 1u;
                     const uint64_t t0 = global_timer_ns();
@@ -238,147 +256,191 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     } else {
         // ------------------------------------------------------------------ consumers
-        // Group grp takes the CTA's items with local index i = grp, grp + 2, ...; item i sits in
-        // stage i % kAttnStages, that stage's use i / kAttnStages.
+        // Group grp takes the CTA's splits with local index i = grp, grp + 2, ...  Stages are
+        // numbered across all of the CTA's splits in producer order: stage number q sits in ring
+        // slot q % kAttnStages, that slot's use q / kAttnStages.
         const int grp = (warp - 1) / kAttnConsumers;
         const int cw = (warp - 1) % kAttnConsumers, ct = threadIdx.x - 32 - 32 * kAttnConsumers * grp;
         const int bar_id = 1 + grp;
         const int gid = lane >> 2, tig = lane & 3;
         float (*red_m)[8] = red_m_all[grp];
         float (*red_s)[8] = red_s_all[grp];
-        uint32_t local = 0;
-        for (uint32_t it = blockIdx.x; it < items; it += gridDim.x) {
+        uint32_t local = 0, q0 = 0;  // the split's local index and its first stage number
+        bool alive = true;
+        for (uint32_t it = blockIdx.x; alive && it < items; it += gridDim.x) {
             const uint32_t sg = it / n_splits;
             const int split = (int)(it - sg * n_splits), g = (int)(sg % n_kv), b = (int)(sg / n_kv);
             const int64_t t0 = (int64_t)split * kAttnSplit;
             const int64_t L = attn_len(p, b, ct == 0 && grp == 0 && split == 0, lens_s);
             if (t0 >= L) continue;
-            const uint32_t mine = local++;
+            const int nc = attn_chunks(L - t0);
+            const uint32_t mine = local++, first = q0;
+            q0 += (uint32_t)nc;
             if (mine % kAttnGroups != (uint32_t)grp) continue;
-            const int stage = (int)(mine % kAttnStages);
-            const uint32_t use = mine / kAttnStages;
-            const int n_tok = (int)(L - t0 < kAttnSplit ? L - t0 : kAttnSplit);
-            const uint8_t *ks = k_tile(stage);
-            uint8_t *vs = v_tile(stage);
-            const __nv_bfloat16 *qs = q_rows(stage);
-            // Items are started in order: once the group before this one has started item mine - 1,
-            // every earlier item -- the stage's previous use among them -- has started, so that use's
-            // copies have landed and the stage's barriers are at most one phase from the one
-            // wanted: a parity wait is exact.
-            const int prev_grp = grp == 0 ? kAttnGroups - 1 : grp - 1;
-            bool ok = mine == 0 || wait_flag_at_least(&progress[prev_grp], (int)mine, abort_flag, p.status, lim);
-            ok = ok && wait_bounded(&kfull[stage], use & 1u, abort_flag, p.status, lim);
-            if (!consumers_all(bar_id, ok)) break;
-            if (ct == 0) progress[grp] = (int)mine + 1;
 
-            // ---- scores: acc[nt] is the 16 x 8 tile (heads x tokens 32 cw + 8 nt ..)
-            float acc[4][4];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
-#pragma unroll
-            for (int kk = 0; kk < kAttnD / 16; ++kk) {
-                uint32_t af[4];
-                ldsm_x4(af, qs + ((lane & 7) + 8 * ((lane >> 3) & 1)) * kAttnQStride + 16 * kk + 8 * (lane >> 4));
-#pragma unroll
-                for (int nt = 0; nt < 4; nt += 2) {
-                    // matrices: (tile nt, d 0-7), (nt, d 8-15), (nt+1, d 0-7), (nt+1, d 8-15) of this step
-                    uint32_t bf[4];
-                    ldsm_x4(bf, kv_chunk(ks, 32 * cw + 8 * (nt + (lane >> 4)) + (lane & 7), 2 * kk + ((lane >> 3) & 1)));
-                    mma_16816_bf16(acc[nt], af, bf[0], bf[1]);
-                    mma_16816_bf16(acc[nt + 1], af, bf[2], bf[3]);
-                }
-            }
-            // scale and mask: element (row gid / gid+8, token 32 cw + 8 nt + 2 tig + {0,1})
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int tok = 32 * cw + 8 * nt + 2 * tig + (e & 1);
-                    acc[nt][e] = tok < n_tok ? acc[nt][e] * p.scale : kNegInf;
-                }
-
-            // ---- per-head max: own values in order, quad butterfly, warps in order.  Only rows
-            // 0..7 (e = 0, 1) hold heads; rows 8..15 are padding and are not used.
-            {
-                float m = acc[0][0];
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) m = fmaxf(fmaxf(m, acc[nt][0]), acc[nt][1]);
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-                if (tig == 0) red_m[cw][gid] = m;
-            }
-            consumers_sync(bar_id);  // every warp's maxima are posted; the K tile is no longer read
-            // ---- p = exp(s - max); per-head sums by the same trees.  Each thread folds the warps'
-            // maxima of its two heads itself, in warp order.
-            {
-                float m = red_m[0][gid];
-#pragma unroll
-                for (int w = 1; w < kAttnConsumers; ++w) m = fmaxf(m, red_m[w][gid]);
-                float l = 0.0f;
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        float &x = acc[nt][e];
-                        x = x == kNegInf ? 0.0f : __expf(x - m);
-                        l = __fadd_rn(l, x);
-                    }
-                l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 1));
-                l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 2));
-                if (tig == 0) red_s[cw][gid] = l;
-            }
-            if (!consumers_all(bar_id, wait_bounded(&vfull[stage], use & 1u, abort_flag, p.status, lim))) break;
-            if (n_tok < kAttnSplit) {
-                // Value rows past the sequence's end: zero, whatever the cache holds there.
-                for (int i = ct; i < (kAttnSplit - n_tok) * 16; i += 32 * kAttnConsumers)
-                    *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(kv_chunk(vs, n_tok + i / 16, i % 16))) =
-                        make_uint4(0u, 0u, 0u, 0u);
-                consumers_sync(bar_id);
-            }
-
-            // ---- O_w^T = V_w^T . P_w^T: d on the MMA's M (8 tiles of 16 rows), the group's heads on
-            // N (8 columns; columns G .. 7 are padding), tokens on K in two 16-token steps in
-            // ascending order.  Rows 0..7 of the score tiles (e = 0, 1: head gid, tokens 2 tig and
-            // 2 tig + 1 of tiles 2j and 2j + 1) are exactly the B fragments of P^T for step j, and
-            // the transposed ldmatrix of V yields the A fragments of V^T, so nothing is reshuffled.
-            // P enters as two bf16 terms, hi = bf16(p) and lo = bf16(p - hi), so the weights keep
-            // about 16 significant bits; per 16-token step hi is added first.
-            float o[kAttnD / 16][4];  // o[mt]: d 16 mt + gid (+ 8), heads 2 tig, 2 tig + 1
+            // Per head (row gid of the score tiles): the running maximum over the split's stages so
+            // far, and this thread's running sum of exp(s - m_run) over its tokens.  o holds this
+            // warp's weighted sums O_w^T (d 16 mt + gid (+ 8), heads 2 tig and 2 tig + 1), scaled to
+            // the same running maximum.
+            float m_run = kNegInf, l_t = 0.0f;
+            float o[kAttnD / 16][4];
 #pragma unroll
             for (int mt = 0; mt < kAttnD / 16; ++mt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) o[mt][e] = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const float pv[4] = {acc[2 * j][0], acc[2 * j][1], acc[2 * j + 1][0], acc[2 * j + 1][1]};
-                float hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    hi[e] = __bfloat162float(__float2bfloat16_rn(pv[e]));
-                    lo[e] = pv[e] - hi[e];
+            int stage = 0;
+            for (int c = 0; c < nc; ++c) {
+                const uint32_t qn = first + (uint32_t)c;
+                stage = (int)(qn % kAttnStages);
+                const uint32_t use = qn / kAttnStages;
+                const int64_t tc = t0 + (int64_t)c * kAttnChunk;
+                const int n_tok = (int)(L - tc < kAttnChunk ? L - tc : kAttnChunk);
+                const uint8_t *ks = k_tile(stage);
+                uint8_t *vs = v_tile(stage);
+                const __nv_bfloat16 *qs = q_rows(stage);
+                // Uses of a slot are passed in order: once the slot's previous use has been passed
+                // (by either group), the slot's barriers are at most one phase from the one wanted,
+                // so a parity wait is exact.  V is released with K, so the V wait needs no more.
+                bool ok = wait_flag_at_least(&slot_use[stage], (int)use, abort_flag, p.status, lim);
+                ok = ok && wait_bounded(&kfull[stage], use & 1u, abort_flag, p.status, lim);
+                if (!consumers_all(bar_id, ok)) {
+                    alive = false;
+                    break;
                 }
-                const uint32_t pb_hi0 = pack_bf16(hi[0], hi[1]), pb_hi1 = pack_bf16(hi[2], hi[3]);
-                const uint32_t pb_lo0 = pack_bf16(lo[0], lo[1]), pb_lo1 = pack_bf16(lo[2], lo[3]);
-                const int tok0 = 32 * cw + 16 * j;
+                if (ct == 0) slot_use[stage] = (int)use + 1;
+
+                // ---- scores: acc[nt] is the 16 x 8 tile (heads x tokens 32 cw + 8 nt ..)
+                float acc[4][4];
 #pragma unroll
-                for (int dt = 0; dt < kAttnD / 8; dt += 2) {
-                    // matrices (transposed): (tokens 0-7, d tile dt), (8-15, dt), (0-7, dt+1), (8-15, dt+1);
-                    // as A of V^T (rows d, columns tokens): a0 = (dt, 0-7), a1 = (dt+1, 0-7),
-                    // a2 = (dt, 8-15), a3 = (dt+1, 8-15).
-                    uint32_t vf[4];
-                    ldsm_x4_trans(vf, kv_chunk(vs, tok0 + (lane & 7) + 8 * ((lane >> 3) & 1), dt + (lane >> 4)));
-                    const uint32_t va[4] = {vf[0], vf[2], vf[1], vf[3]};
-                    mma_16816_bf16(o[dt / 2], va, pb_hi0, pb_hi1);
-                    mma_16816_bf16(o[dt / 2], va, pb_lo0, pb_lo1);
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
+#pragma unroll
+                for (int kk = 0; kk < kAttnD / 16; ++kk) {
+                    uint32_t af[4];
+                    ldsm_x4(af, qs + ((lane & 7) + 8 * ((lane >> 3) & 1)) * kAttnQStride + 16 * kk + 8 * (lane >> 4));
+#pragma unroll
+                    for (int nt = 0; nt < 4; nt += 2) {
+                        // matrices: (tile nt, d 0-7), (nt, d 8-15), (nt+1, d 0-7), (nt+1, d 8-15) of this step
+                        uint32_t bf[4];
+                        ldsm_x4(bf, kv_chunk(ks, 32 * cw + 8 * (nt + (lane >> 4)) + (lane & 7), 2 * kk + ((lane >> 3) & 1)));
+                        mma_16816_bf16(acc[nt], af, bf[0], bf[1]);
+                        mma_16816_bf16(acc[nt + 1], af, bf[2], bf[3]);
+                    }
+                }
+                // scale and mask: element (row gid / gid+8, token 32 cw + 8 nt + 2 tig + {0,1})
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int tok = 32 * cw + 8 * nt + 2 * tig + (e & 1);
+                        acc[nt][e] = tok < n_tok ? acc[nt][e] * p.scale : kNegInf;
+                    }
+
+                // ---- the stage's maximum per head: own values in order, quad butterfly, warps in
+                // order.  Only rows 0..7 (e = 0, 1) hold heads; rows 8..15 are padding.
+                {
+                    float m = acc[0][0];
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt) m = fmaxf(fmaxf(m, acc[nt][0]), acc[nt][1]);
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+                    if (tig == 0) red_m[cw][gid] = m;
+                }
+                consumers_sync(bar_id);  // every warp's maxima are posted; the K tile is no longer read
+                // ---- new running maximum, rescale what is accumulated, p = exp(s - m_new), sums.
+                float alpha;
+                {
+                    float m_c = red_m[0][gid];
+#pragma unroll
+                    for (int w = 1; w < kAttnConsumers; ++w) m_c = fmaxf(m_c, red_m[w][gid]);
+                    const float m_new = fmaxf(m_run, m_c);  // finite: the stage has a token
+                    alpha = __expf(m_run - m_new);          // 0 for the first stage
+                    m_run = m_new;
+                    float l = __fmul_rn(l_t, alpha);
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            float &x = acc[nt][e];
+                            x = x == kNegInf ? 0.0f : __expf(x - m_new);
+                            l = __fadd_rn(l, x);
+                        }
+                    l_t = l;
+                }
+                {
+                    // o's columns are heads 2 tig and 2 tig + 1, whose factors the lanes of rows
+                    // gid = 2 tig (lane 8 tig) and 2 tig + 1 (lane 8 tig + 4) hold.
+                    const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * tig);
+                    const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * tig + 4);
+#pragma unroll
+                    for (int mt = 0; mt < kAttnD / 16; ++mt) {
+                        o[mt][0] = __fmul_rn(o[mt][0], a0);
+                        o[mt][1] = __fmul_rn(o[mt][1], a1);
+                        o[mt][2] = __fmul_rn(o[mt][2], a0);
+                        o[mt][3] = __fmul_rn(o[mt][3], a1);
+                    }
+                }
+                if (!consumers_all(bar_id, wait_bounded(&vfull[stage], use & 1u, abort_flag, p.status, lim))) {
+                    alive = false;
+                    break;
+                }
+                if (n_tok < kAttnChunk) {
+                    // Value rows past the sequence's end: zero, whatever the cache holds there.
+                    for (int i = ct; i < (kAttnChunk - n_tok) * 16; i += 32 * kAttnConsumers)
+                        *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(kv_chunk(vs, n_tok + i / 16, i % 16))) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    consumers_sync(bar_id);
+                }
+
+                // ---- O_w^T += V_w^T . P_w^T: d on the MMA's M (8 tiles of 16 rows), the group's heads
+                // on N (8 columns; columns G .. 7 are padding), tokens on K in two 16-token steps in
+                // ascending order.  Rows 0..7 of the score tiles (e = 0, 1: head gid, tokens 2 tig and
+                // 2 tig + 1 of tiles 2j and 2j + 1) are exactly the B fragments of P^T for step j, and
+                // the transposed ldmatrix of V yields the A fragments of V^T, so nothing is reshuffled.
+                // P enters as two bf16 terms, hi = bf16(p) and lo = bf16(p - hi), so the weights keep
+                // about 16 significant bits; per 16-token step hi is added first.
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float pv[4] = {acc[2 * j][0], acc[2 * j][1], acc[2 * j + 1][0], acc[2 * j + 1][1]};
+                    float hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        hi[e] = __bfloat162float(__float2bfloat16_rn(pv[e]));
+                        lo[e] = pv[e] - hi[e];
+                    }
+                    const uint32_t pb_hi0 = pack_bf16(hi[0], hi[1]), pb_hi1 = pack_bf16(hi[2], hi[3]);
+                    const uint32_t pb_lo0 = pack_bf16(lo[0], lo[1]), pb_lo1 = pack_bf16(lo[2], lo[3]);
+                    const int tok0 = 32 * cw + 16 * j;
+#pragma unroll
+                    for (int dt = 0; dt < kAttnD / 8; dt += 2) {
+                        // matrices (transposed): (tokens 0-7, d tile dt), (8-15, dt), (0-7, dt+1),
+                        // (8-15, dt+1); as A of V^T (rows d, columns tokens): a0 = (dt, 0-7),
+                        // a1 = (dt+1, 0-7), a2 = (dt, 8-15), a3 = (dt+1, 8-15).
+                        uint32_t vf[4];
+                        ldsm_x4_trans(vf, kv_chunk(vs, tok0 + (lane & 7) + 8 * ((lane >> 3) & 1), dt + (lane >> 4)));
+                        const uint32_t va[4] = {vf[0], vf[2], vf[1], vf[3]};
+                        mma_16816_bf16(o[dt / 2], va, pb_hi0, pb_hi1);
+                        mma_16816_bf16(o[dt / 2], va, pb_lo0, pb_lo1);
+                    }
+                }
+                if (c + 1 < nc) {
+                    // Release the stage, one arrival per warp: the generic-proxy writes into it
+                    // (zeroed rows) are ordered before the next TMA writes.
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[stage]);
                 }
             }
-            // The K tile (read by every warp before the maxima barrier) holds the per-warp outputs,
-            // rows kAttnOStride floats apart.  A store's lanes cover d 16 mt + gid (+ 8) of heads
-            // 2 tig (+ 1): for up to four heads, rows 0 and 2 (or 1 and 3) sit 16 banks apart, so the
-            // 16 lanes that store land in distinct banks; eight heads share banks two ways.
-            float *so = reinterpret_cast<float *>(const_cast<uint8_t *>(ks));
+            if (!alive) break;
+
+            // ---- the split's partial result.  The last stage's K tile (read by every warp before
+            // that stage's maxima barrier) holds the per-warp outputs, rows kAttnOStride floats
+            // apart: a store's lanes cover d 16 mt + gid (+ 8) of heads 2 tig (+ 1); for up to four
+            // heads, rows 0 and 2 (or 1 and 3) sit 16 banks apart, so the 16 lanes that store land in
+            // distinct banks; eight heads share banks two ways.  Every warp has read the maxima of
+            // the last stage, so red_m[0] can take the running maxima and red_s the warps' sums.
+            float *so = reinterpret_cast<float *>(const_cast<uint8_t *>(k_tile(stage)));
 #pragma unroll
             for (int mt = 0; mt < kAttnD / 16; ++mt)
 #pragma unroll
@@ -386,6 +448,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     const int head = 2 * tig + (e & 1), col = 16 * mt + gid + 8 * (e >> 1);
                     if (head < G) so[(cw * kAttnMaxGroup + head) * kAttnOStride + col] = o[mt][e];
                 }
+            {
+                float l = __fadd_rn(l_t, __shfl_xor_sync(0xffffffffu, l_t, 1));
+                l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 2));
+                if (tig == 0) red_s[cw][gid] = l;
+                if (tig == 0 && cw == 0) red_m[0][gid] = m_run;
+            }
             consumers_sync(bar_id);
 #pragma unroll
             for (int j = 0; j < G; ++j) {
@@ -395,16 +463,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const int64_t bh = (int64_t)b * p.Hq + (int64_t)g * G + j;
                 p.part_acc[(bh * p.S + split) * kAttnD + ct] = r;
                 if (ct == 0) {
-                    float m = red_m[0][j], l = red_s[0][j];
-                    for (int w = 1; w < kAttnConsumers; ++w) {
-                        m = fmaxf(m, red_m[w][j]);
-                        l = __fadd_rn(l, red_s[w][j]);
-                    }
-                    p.part_ms[bh * p.S + split] = make_float2(m, l);
+                    float l = red_s[0][j];
+                    for (int w = 1; w < kAttnConsumers; ++w) l = __fadd_rn(l, red_s[w][j]);
+                    p.part_ms[bh * p.S + split] = make_float2(red_m[0][j], l);
                 }
             }
-            // Release the stage, one arrival per warp: the generic-proxy writes into it (partial
-            // outputs, zeroed rows) are ordered before the next TMA writes.
+            // Release the last stage, one arrival per warp: the generic-proxy writes into it
+            // (partial outputs, zeroed rows) are ordered before the next TMA writes.
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);

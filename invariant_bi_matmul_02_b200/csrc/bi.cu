@@ -208,7 +208,7 @@ bi_status encode_kv_map(CUtensorMap *map, const void *base, uint64_t D, uint64_t
     if (!enc) return BI_ERR_CUDA;
     const cuuint64_t dims[4] = {D, Hkv, Lmax, B};
     const cuuint64_t strides[3] = {D * 2, Hkv * D * 2, Lmax * Hkv * D * 2};
-    const cuuint32_t box[4] = {64, 1, (cuuint32_t)bi::kAttnSplit, 1};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)bi::kAttnChunk, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

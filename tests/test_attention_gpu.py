@@ -25,7 +25,7 @@ def make(seed, B, Hq, Hkv, Lmax):
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 8), (16, 8), (16, 2), (8, 1)])  # group sizes 4, 1, 2, 8, 8
-@pytest.mark.parametrize("lens", [[1, 128, 300], [127, 129, 256, 257], [5]])
+@pytest.mark.parametrize("lens", [[1, 128, 300], [127, 129, 256, 257], [5], [511, 512, 513, 1100]])
 def test_attention_parity(Hq, Hkv, lens):
     B, Lmax = len(lens), max(lens) + 3
     q, k, v = make(800, B, Hq, Hkv, Lmax)
