@@ -126,8 +126,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     griddep_launch_dependents();
 
     // Fused SiLU * up: a pair tile yields kHalfBN columns of h; CTA 0 stages gate rows
-    // n0 .. n0+127 and CTA 1 the up rows F + n0 .. so each CTA's accumulator holds gate in
-    // columns [0, kHalfBN) and up in [kHalfBN, kPairBN) for its 128 rows.
+    // n0 .. n0 + kHalfBN - 1 and CTA 1 the up rows F + n0 .., so each CTA's accumulator holds gate
+    // in columns [0, kHalfBN) and up in [kHalfBN, kPairBN) for its 128 rows.
     const int out_cols = p.fuse_silu ? kHalfBN : kPairBN;
     const int m_blocks = (p.M + kPairBM - 1) / kPairBM;
     const int n_blocks = (p.N + out_cols - 1) / out_cols;
