@@ -36,6 +36,23 @@ def test_attention_parity(Hq, Hkv, lens):
     assert bi.bi_get_device_status() == bi.BI_OK
 
 
+def test_attention_batch_beyond_the_cached_lengths():
+    """Launch 1 keeps the first 4096 sequence lengths in shared memory and reads the others from
+    global memory: a batch of 5000 short sequences of mixed lengths checks both paths against the
+    oracle, and a sequence past the cache gives the same bits as when it is decoded alone."""
+    B, Hq, Hkv, Lmax = 5000, 1, 1, 3
+    q, k, v = make(806, B, Hq, Hkv, Lmax)
+    sl = torch.tensor([1 + (i * 7) % Lmax for i in range(B)], dtype=torch.int32)
+    qd, kd, vd, ld = q.to(DEV), k.to(DEV), v.to(DEV), sl.to(DEV)
+    o = bi.bi_decode_attention(qd, kd, vd, ld)
+    ref = oracle.decode_attention(bf16_bits_np(q), bf16_bits_np(k), bf16_bits_np(v), sl.numpy(), D ** -0.5)
+    assert_bf16_close(o, ref, "attention B=5000")
+    for i in (0, 4095, 4096, 4999):
+        alone = bi.bi_decode_attention(qd[i:i + 1], kd[i:i + 1], vd[i:i + 1], ld[i:i + 1])
+        assert same_bits(alone, o[i:i + 1]), f"sequence {i}"
+    assert bi.bi_get_device_status() == bi.BI_OK
+
+
 def test_attention_long_sequences_sampled():
     B, Hq, Hkv, Lmax = 4, 32, 8, 4096
     q, k, v = make(801, B, Hq, Hkv, Lmax)
