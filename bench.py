@@ -253,7 +253,7 @@ def cpu_baseline(host: dict, x_host, budget_s: float = 15.0) -> dict:
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -270,7 +270,10 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
-    def stop(self) -> dict:
+    def stop(self, window=None) -> dict:
+        """Median SM clock and the throttle reasons seen.  With `window` = (t0, t1) host wall-clock
+        seconds, only samples taken inside it count (the sampler starts before the timed region,
+        and samples of an idle GPU would read its maximum clock)."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -279,22 +282,31 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        from datetime import datetime
+        rows = []
         for line in out.strip().splitlines():
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
+                ts = datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                ts = None
+            try:
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+        inside = [r for r in rows if window and r[0] is not None and window[0] <= r[0] <= window[1]]
+        use = inside if inside else rows
+        sm, smax, reasons = [r[1] for r in use], (use[-1][2] if use else None), set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in use:
+            for n, v in zip(names, r[3]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "window": "timed region" if inside else "whole sampling run"}
 
 
 # ----------------------------------------------------------------------------- main arms
@@ -349,12 +361,14 @@ def run_bi(args):
         sampler.start()
         time.sleep(0.3)  # let nvidia-smi attach before the timed region
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
     start.record(stream)
     for s in range(args.steps):
         run_step(wl, wl.x, lm_marks[s], only="lm_head")
     end.record(stream)
     torch.cuda.synchronize()
-    clocks = sampler.stop() if sampler else None
+    t_wall1 = time.time()
+    clocks = sampler.stop((t_wall0, t_wall1)) if sampler else None
     barrier()
     elapsed_ms = start.elapsed_time(end)
     lm_ms = sum(m[0].elapsed_time(m[1]) for m in lm_marks) / args.steps

@@ -55,17 +55,37 @@ class _FakeSmi:
 
 
 def test_clock_sampler_reports_median_and_active_reasons():
-    lines = ["0, 1800, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active",
-             "0, 1700, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
-             "0, 1900, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    t = "2026/12/03 10:00:00.{:03d}"
+    lines = [t.format(100) + ", 0, 1800, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active",
+             t.format(200) + ", 0, 1700, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+             t.format(300) + ", 0, 1900, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, Not Active",
              "garbled line"]
     s = bench.ClockSampler(0)
     s.proc = _FakeSmi("\n".join(lines))
     out = s.stop()
     assert out["sm_mhz"] == 1800 and out["sm_max_mhz"] == 1965
     assert out["reasons"] == ["sw_power_cap"] and out["samples"] == 3
-    s.proc = _FakeSmi("0, 900, 1965, 500.0, 0x8, Active, Not Active, Not Active, Not Active")
+    s.proc = _FakeSmi(t.format(0) + ", 0, 900, 1965, 500.0, 0x8, Active, Not Active, Not Active, Not Active")
     assert s.stop()["reasons"] == ["hw_slowdown"]
+
+
+def test_clock_sampler_keeps_the_samples_of_the_timed_region():
+    """Samples before the timed region (an idle GPU at its maximum clock) do not count."""
+    from datetime import datetime
+    t = "2026/12/03 10:00:0{}.000"
+    lines = [t.format(0) + ", 0, 1965, 1965, 150.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+             t.format(1) + ", 0, 1965, 1965, 160.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+             t.format(2) + ", 0, 1650, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+             t.format(3) + ", 0, 1700, 1965, 995.0, 0x4, Not Active, Not Active, Not Active, Active",
+             t.format(4) + ", 0, 1680, 1965, 985.0, 0x4, Not Active, Not Active, Not Active, Active"]
+    at = [datetime.strptime(t.format(i), "%Y/%m/%d %H:%M:%S.%f").timestamp() for i in range(5)]
+    s = bench.ClockSampler(0)
+    s.proc = _FakeSmi("\n".join(lines))
+    out = s.stop((at[2] - 0.5, at[4] + 0.5))
+    assert out["sm_mhz"] == 1680 and out["samples"] == 3 and out["window"] == "timed region"
+    assert out["reasons"] == ["sw_power_cap"]
+    s.proc = _FakeSmi("\n".join(lines))
+    assert s.stop((at[4] + 10, at[4] + 11))["window"] == "whole sampling run"  # nothing inside
 
 
 def test_roofline_point_takes_the_larger_bound():
