@@ -911,6 +911,8 @@ KERNEL_CASES = {
     "log_softmax_cluster": "bi_log_softmax_cluster M=1024 V=151936 bf16 -> fp32 (4 CTAs per row)",
     "silu_mul": "bi_silu_mul M=1024 F=12288",
     "decode_attention": "bi_decode_attention B=64 L=4096, 32 q / 8 kv heads of 128",
+    "decode_attention_sdpa": "torch scaled_dot_product_attention on the decode_attention case's inputs "
+                             "(a library reference for profiles; not batch-invariant)",
 }
 
 
@@ -970,7 +972,7 @@ def run_kernel_case(args):
         h = torch.empty(1024, FFN, dtype=torch.bfloat16, device=dev)
         fn = lambda: bi.bi_silu_mul(gu, out=h)
         work, unit = 6 * FFN * 1024, "GB/s"
-    elif name == "decode_attention":
+    elif name in ("decode_attention", "decode_attention_sdpa"):
         B, L, Hq, Hkv, D = 64, 4096, 32, 8, 128
         g = torch.Generator(device=dev)
         g.manual_seed(56)
@@ -981,6 +983,10 @@ def run_kernel_case(args):
         scr = torch.empty(bi.bi_decode_attention_scratch_bytes(B, Hq, D, L), dtype=torch.uint8, device=dev)
         o = torch.empty_like(q)
         fn = lambda: bi.bi_decode_attention(q, k, v, sl, scratch=scr, out=o)
+        if name == "decode_attention_sdpa":
+            import torch.nn.functional as F
+            qs, ks, vs = q.view(B, Hq, 1, D), k.permute(0, 2, 1, 3), v.permute(0, 2, 1, 3)
+            fn = lambda: F.scaled_dot_product_attention(qs, ks, vs, enable_gqa=True)
         work, unit = 2 * B * L * Hkv * D * 2, "GB/s"
     else:
         raise SystemExit(f"unknown kernel case {name}; choose from {sorted(KERNEL_CASES)}")
