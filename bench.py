@@ -582,7 +582,7 @@ def _rows_differing(t, ref1):
 
 SWEEP_GEMMS = [("q/o", HIDDEN, HIDDEN), ("k/v", HIDDEN, KV), ("gate/up", HIDDEN, FFN), ("down", FFN, HIDDEN),
                ("lm_head", HIDDEN, VOCAB)]
-SWEEP_M = [1, 64, 256, 1024, 2048]
+METRIC_SWEEP_M = [1, 64, 256, 1024, 2048]
 SWEEP_ROW_OPS = [("rmsnorm", HIDDEN, (1024, 16384)), ("mean", HIDDEN, (1024, 16384)),
                  ("log_softmax", VOCAB, (1, 64, 1024))]
 
@@ -622,10 +622,10 @@ def metric_sweep(device, peaks: dict, reps: int = 10) -> dict:
                        "N(0,1), weights N(0,0.02) [N,K]; peaks: burst", "gemm": [], "row_ops": []}
     for name, K, N in SWEEP_GEMMS:
         w = (torch.randn(N, K, generator=g, device=device) * 0.02).to(torch.bfloat16)
-        a = torch.randn(max(SWEEP_M), K, generator=g, device=device).to(torch.bfloat16)
+        a = torch.randn(max(METRIC_SWEEP_M), K, generator=g, device=device).to(torch.bfloat16)
         ref = torch.cat([bi.bi_matmul(a[i:i + 1], w) for i in range(8)])
         tref = torch.cat([F.linear(a[i:i + 1], w) for i in range(8)])
-        for M in SWEEP_M:
+        for M in METRIC_SWEEP_M:
             am = a[:M]
             c = torch.empty(M, N, dtype=torch.bfloat16, device=device)
             t_bi = us(lambda: bi.bi_matmul(am, w, out=c))

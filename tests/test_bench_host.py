@@ -98,3 +98,10 @@ def test_roofline_point_takes_the_larger_bound():
     # 1 GFLOP = 1 us of tensor time; 50 MB = 10 us of HBM time: HBM-bound, measured 20 us
     r = bench.roofline_point(1e9, 50e6, 20.0, peaks)
     assert r == {"bound": "hbm", "roofline_frac": 0.5}
+
+
+def test_sweep_lists_are_distinct():
+    """The extended sweep covers M = 1..2048 with the ragged points 3, 77 and 1000; the JSON
+    line's metric sweep keeps its own five points."""
+    assert bench.SWEEP_M == [1, 2, 3, 4, 8, 16, 32, 64, 77, 128, 256, 512, 1000, 1024, 2048]
+    assert bench.METRIC_SWEEP_M == [1, 64, 256, 1024, 2048]
