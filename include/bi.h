@@ -275,7 +275,7 @@ bi_status bi_silu_mul(const void *gu, void *h, int64_t M, int64_t F, void *strea
  *            sequence b are read.
  *   seq_lens device, int32, [B], each in 1 .. Lmax.  A value outside is clamped and
  *            BI_ERR_INVALID_ARG is recorded in the device status word.
- *   D must be 128 and Hq / Hkv one of 1, 2, 4, 8 (else BI_ERR_UNSUPPORTED); B, Hq, Hkv <= 65535
+ *   D must be 64 or 128 and Hq / Hkv one of 1, 2, 4, 8 (else BI_ERR_UNSUPPORTED); B, Hq, Hkv <= 65535
  *   and B * Hkv * ceil(Lmax / 512) < 2^31 (else BI_ERR_UNSUPPORTED).
  *   scratch  caller-owned device memory, 16-byte aligned, at least
  *            bi_decode_attention_scratch_bytes(B, Hq, D, Lmax) bytes; overwritten (two

@@ -30,7 +30,7 @@
 
 namespace bi {
 
-constexpr int kAttnD = 128;
+constexpr int kAttnD = 128;                             // largest head size; shared memory is laid out for it
 constexpr int kAttnChunk = 128;                         // tokens per ring stage
 constexpr int kAttnSplit = 4 * kAttnChunk;              // tokens per split (one partial result)
 constexpr int kAttnConsumers = 4;                       // consumer warps per group, 32 tokens of a stage each
@@ -162,11 +162,14 @@ __device__ __forceinline__ bool wait_flag_at_least(volatile int *flag, int v, vo
 // threads' sums meet in the lane quad (xor 1, 2), then the four warps' sums and O_w are added in
 // warp order.  Value rows past the sequence's end are zeroed in shared memory before use, so stale
 // cache contents never reach the sums.
-template <int G>  // query heads per kv head (1, 2, 4 or 8)
+template <int G, int D>  // G query heads per kv head (1, 2, 4 or 8); head size D (64 or 128)
 __global__ void __launch_bounds__(kAttnThreads, 1)
     decode_attention_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                                   const AttnParams p)
 {
+    static_assert(D == 64 || D == 128, "head size 64 or 128: one or two 64-wide TMA boxes per tile");
+    constexpr int kBoxes = D / 64;                      // 64-d TMA boxes per K or V tile
+    constexpr int kTileBytes = kBoxes * kAttnBoxBytes;  // bytes one K or V tile of a stage carries
     extern __shared__ uint8_t attn_raw[];
     uint8_t *smem = attn_raw + ((1024u - (smem_addr(attn_raw) & 1023u)) & 1023u);
     __shared__ uint64_t kfull[kAttnStages], vfull[kAttnStages], empty[kAttnStages];
@@ -228,15 +231,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int c = 0; c < nc; ++c) {
                     const int32_t tc = (int32_t)(t0 + (int64_t)c * kAttnChunk);
                     if (!(ok = wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim))) break;
-                    mbar_arrive_expect_tx(&kfull[stage], G * kAttnD * 2 + kAttnTileBytes);
+                    mbar_arrive_expect_tx(&kfull[stage], G * D * 2 + kTileBytes);
                     for (int j = 0; j < G; ++j)
                         bulk_load(q_rows(stage) + j * kAttnQStride,
-                                  p.q + ((int64_t)b * p.Hq + (int64_t)g * G + j) * kAttnD, kAttnD * 2, &kfull[stage]);
-                    tma_load_4d(k_tile(stage), &tm_k, &kfull[stage], 0, g, tc, b);
-                    tma_load_4d(k_tile(stage) + kAttnBoxBytes, &tm_k, &kfull[stage], 64, g, tc, b);
-                    mbar_arrive_expect_tx(&vfull[stage], kAttnTileBytes);
-                    tma_load_4d(v_tile(stage), &tm_v, &vfull[stage], 0, g, tc, b);
-                    tma_load_4d(v_tile(stage) + kAttnBoxBytes, &tm_v, &vfull[stage], 64, g, tc, b);
+                                  p.q + ((int64_t)b * p.Hq + (int64_t)g * G + j) * D, D * 2, &kfull[stage]);
+#pragma unroll
+                    for (int x = 0; x < kBoxes; ++x)
+                        tma_load_4d(k_tile(stage) + x * kAttnBoxBytes, &tm_k, &kfull[stage], 64 * x, g, tc, b);
+                    mbar_arrive_expect_tx(&vfull[stage], kTileBytes);
+#pragma unroll
+                    for (int x = 0; x < kBoxes; ++x)
+                        tma_load_4d(v_tile(stage) + x * kAttnBoxBytes, &tm_v, &vfull[stage], 64 * x, g, tc, b);
                     ++issued;
                     advance(stage, phase, kAttnStages);
                 }
@@ -283,9 +288,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // warp's weighted sums O_w^T (d 16 mt + gid (+ 8), heads 2 tig and 2 tig + 1), scaled to
             // the same running maximum.
             float m_run = kNegInf, l_t = 0.0f;
-            float o[kAttnD / 16][4];
+            float o[D / 16][4];
 #pragma unroll
-            for (int mt = 0; mt < kAttnD / 16; ++mt)
+            for (int mt = 0; mt < D / 16; ++mt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) o[mt][e] = 0.0f;
             int stage = 0;
@@ -316,7 +321,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
 #pragma unroll
-                for (int kk = 0; kk < kAttnD / 16; ++kk) {
+                for (int kk = 0; kk < D / 16; ++kk) {
                     uint32_t af[4];
                     ldsm_x4(af, qs + ((lane & 7) + 8 * ((lane >> 3) & 1)) * kAttnQStride + 16 * kk + 8 * (lane >> 4));
 #pragma unroll
@@ -374,7 +379,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * tig);
                     const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * tig + 4);
 #pragma unroll
-                    for (int mt = 0; mt < kAttnD / 16; ++mt) {
+                    for (int mt = 0; mt < D / 16; ++mt) {
                         o[mt][0] = __fmul_rn(o[mt][0], a0);
                         o[mt][1] = __fmul_rn(o[mt][1], a1);
                         o[mt][2] = __fmul_rn(o[mt][2], a0);
@@ -387,8 +392,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 if (n_tok < kAttnChunk) {
                     // Value rows past the sequence's end: zero, whatever the cache holds there.
-                    for (int i = ct; i < (kAttnChunk - n_tok) * 16; i += 32 * kAttnConsumers)
-                        *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(kv_chunk(vs, n_tok + i / 16, i % 16))) =
+                    for (int i = ct; i < (kAttnChunk - n_tok) * (D / 8); i += 32 * kAttnConsumers)
+                        *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(kv_chunk(vs, n_tok + i / (D / 8), i % (D / 8)))) =
                             make_uint4(0u, 0u, 0u, 0u);
                     consumers_sync(bar_id);
                 }
@@ -413,7 +418,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     const uint32_t pb_lo0 = pack_bf16(lo[0], lo[1]), pb_lo1 = pack_bf16(lo[2], lo[3]);
                     const int tok0 = 32 * cw + 16 * j;
 #pragma unroll
-                    for (int dt = 0; dt < kAttnD / 8; dt += 2) {
+                    for (int dt = 0; dt < D / 8; dt += 2) {
                         // matrices (transposed): (tokens 0-7, d tile dt), (8-15, dt), (0-7, dt+1),
                         // (8-15, dt+1); as A of V^T (rows d, columns tokens): a0 = (dt, 0-7),
                         // a1 = (dt+1, 0-7), a2 = (dt, 8-15), a3 = (dt+1, 8-15).
@@ -442,7 +447,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // the last stage, so red_m[0] can take the running maxima and red_s the warps' sums.
             float *so = reinterpret_cast<float *>(const_cast<uint8_t *>(k_tile(stage)));
 #pragma unroll
-            for (int mt = 0; mt < kAttnD / 16; ++mt)
+            for (int mt = 0; mt < D / 16; ++mt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int head = 2 * tig + (e & 1), col = 16 * mt + gid + 8 * (e >> 1);
@@ -457,11 +462,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             consumers_sync(bar_id);
 #pragma unroll
             for (int j = 0; j < G; ++j) {
-                float r = so[j * kAttnOStride + ct];
-                for (int w = 1; w < kAttnConsumers; ++w)
-                    r = __fadd_rn(r, so[(w * kAttnMaxGroup + j) * kAttnOStride + ct]);
                 const int64_t bh = (int64_t)b * p.Hq + (int64_t)g * G + j;
-                p.part_acc[(bh * p.S + split) * kAttnD + ct] = r;
+                if (ct < D) {  // thread ct sums column d = ct over the warps, in warp order
+                    float r = so[j * kAttnOStride + ct];
+                    for (int w = 1; w < kAttnConsumers; ++w)
+                        r = __fadd_rn(r, so[(w * kAttnMaxGroup + j) * kAttnOStride + ct]);
+                    p.part_acc[(bh * p.S + split) * D + ct] = r;
+                }
                 if (ct == 0) {
                     float l = red_s[0][j];
                     for (int w = 1; w < kAttnConsumers; ++w) l = __fadd_rn(l, red_s[w][j]);
@@ -478,18 +485,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncthreads();
 }
 
-// Launch 2: grid (Hq, B), kAttnD threads.  Fold the sequence's splits in ascending order.
-// The splits' maximum is exact in any order, so the block takes it in parallel; the weights
+// Launch 2: grid (Hq, B), D threads (one per column of the head).  Fold the sequence's splits
+// in ascending order.  The splits' maximum is exact in any order, so the block takes it in parallel; the weights
 // w_s = exp(m_s - max) and the split sums go to shared memory a chunk at a time, and each thread
 // folds l += sum_s w_s and o += acc_s w_s in ascending s with its value loads issued ahead.
-constexpr int kCombineChunk = kAttnD;
-
-__global__ void __launch_bounds__(kAttnD)
+template <int D>
+__global__ void __launch_bounds__(D)
     decode_attention_combine_kernel(const float2 *__restrict__ part_ms, const float *__restrict__ part_acc,
                                     const int32_t *__restrict__ lens, __nv_bfloat16 *__restrict__ out,
                                     int Hq, int64_t Lmax)
 {
-    __shared__ float w_s[kCombineChunk], l_s[kCombineChunk], red[kAttnD / 32];
+    constexpr int kCombineChunk = D;  // splits whose weights are staged at a time
+    __shared__ float w_s[kCombineChunk], l_s[kCombineChunk], red[D / 32];
     griddep_wait();  // every split's partials are complete
     griddep_launch_dependents();
     const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
@@ -499,16 +506,16 @@ __global__ void __launch_bounds__(kAttnD)
     const int64_t n = attn_splits(L);
     const int64_t bh = (int64_t)b * Hq + h;
     const float2 *ms = part_ms + bh * S;
-    const float *acc = part_acc + bh * S * kAttnD + d;
+    const float *acc = part_acc + bh * S * D + d;
     float m = kNegInf;
-    for (int64_t s = d; s < n; s += kAttnD) m = fmaxf(m, ms[s].x);
+    for (int64_t s = d; s < n; s += D) m = fmaxf(m, ms[s].x);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((d & 31) == 0) red[d >> 5] = m;
     __syncthreads();
     m = red[0];
 #pragma unroll
-    for (int w = 1; w < kAttnD / 32; ++w) m = fmaxf(m, red[w]);
+    for (int w = 1; w < D / 32; ++w) m = fmaxf(m, red[w]);
     float l = 0.0f, o = 0.0f;
     for (int64_t s0 = 0; s0 < n; s0 += kCombineChunk) {
         const int cnt = (int)(n - s0 < kCombineChunk ? n - s0 : kCombineChunk);
@@ -523,7 +530,7 @@ __global__ void __launch_bounds__(kAttnD)
         for (; j + 8 <= cnt; j += 8) {
             float a[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) a[u] = acc[(s0 + j + u) * kAttnD];
+            for (int u = 0; u < 8; ++u) a[u] = acc[(s0 + j + u) * D];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 l = fmaf(l_s[j + u], w_s[j + u], l);
@@ -532,10 +539,10 @@ __global__ void __launch_bounds__(kAttnD)
         }
         for (; j < cnt; ++j) {
             l = fmaf(l_s[j], w_s[j], l);
-            o = fmaf(acc[(s0 + j) * kAttnD], w_s[j], o);
+            o = fmaf(acc[(s0 + j) * D], w_s[j], o);
         }
     }
-    out[bh * kAttnD + d] = __float2bfloat16_rn(o / l);
+    out[bh * D + d] = __float2bfloat16_rn(o / l);
 }
 
 }  // namespace bi

@@ -43,6 +43,20 @@ DeviceState g_dev[kMaxDevices];
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Opt the decode-attention kernels of head size D into their shared memory.
+template <int D>
+bi_status attn_smem_opt_in()
+{
+    const void *fns[4] = {reinterpret_cast<const void *>(bi::decode_attention_split_kernel<1, D>),
+                          reinterpret_cast<const void *>(bi::decode_attention_split_kernel<2, D>),
+                          reinterpret_cast<const void *>(bi::decode_attention_split_kernel<4, D>),
+                          reinterpret_cast<const void *>(bi::decode_attention_split_kernel<8, D>)};
+    for (const void *fn : fns)
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kAttnSmem) != cudaSuccess)
+            return BI_ERR_CUDA;
+    return BI_OK;
+}
+
 // Opt the GEMM configuration T into its shared memory and count the CTA pairs that fit at once.
 template <typename T>
 bi_status pair_clusters(int sms, int *out)
@@ -83,15 +97,7 @@ bi_status device_state(DeviceState **out)
         if (pair_clusters<bi::WideTile>(d.sms, &d.gemm_clusters_wide) != BI_OK ||
             pair_clusters<bi::NarrowTile>(d.sms, &d.gemm_clusters_narrow) != BI_OK)
             return BI_ERR_CUDA;
-        if (cudaFuncSetAttribute(bi::decode_attention_split_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 bi::kAttnSmem) != cudaSuccess ||
-            cudaFuncSetAttribute(bi::decode_attention_split_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 bi::kAttnSmem) != cudaSuccess ||
-            cudaFuncSetAttribute(bi::decode_attention_split_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 bi::kAttnSmem) != cudaSuccess ||
-            cudaFuncSetAttribute(bi::decode_attention_split_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 bi::kAttnSmem) != cudaSuccess)
-            return BI_ERR_CUDA;
+        if (attn_smem_opt_in<64>() != BI_OK || attn_smem_opt_in<128>() != BI_OK) return BI_ERR_CUDA;
         if (cudaFuncSetAttribute(bi::log_softmax_stream_kernel<true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kLsmSmem) != cudaSuccess ||
             cudaFuncSetAttribute(bi::log_softmax_stream_kernel<false>,
@@ -275,6 +281,26 @@ bi_status launch_row_clusters(void (*kernel)(KArgs...), int64_t M, size_t smem, 
 
 // N is the number of output columns.  With fuse_silu, B holds 2N rows ([gate; up]) and
 // the output is silu(A . gate^T) * (A . up^T).
+// Launch 1 (group size G chosen at run time, head size D) and launch 2 of the decode attention.
+template <int D>
+bi_status launch_attention(int64_t group, dim3 grid, size_t smem, cudaStream_t s, const CUtensorMap &tm_k,
+                           const CUtensorMap &tm_v, const bi::AttnParams &p, const int32_t *seq_lens, void *out,
+                           int64_t B)
+{
+    bi_status st;
+    switch (group) {
+    case 1: st = launch_pdl(bi::decode_attention_split_kernel<1, D>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
+    case 2: st = launch_pdl(bi::decode_attention_split_kernel<2, D>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
+    case 4: st = launch_pdl(bi::decode_attention_split_kernel<4, D>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
+    case 8: st = launch_pdl(bi::decode_attention_split_kernel<8, D>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
+    default: return BI_ERR_UNSUPPORTED;
+    }
+    if (st != BI_OK) return st;
+    return launch_pdl(bi::decode_attention_combine_kernel<D>, dim3((unsigned)p.Hq, (unsigned)B), dim3(D), 0, s,
+                      static_cast<const float2 *>(p.part_ms), static_cast<const float *>(p.part_acc), seq_lens,
+                      static_cast<__nv_bfloat16 *>(out), (int)p.Hq, p.Lmax);
+}
+
 // Tile counts, tensor maps and the launch of the pair GEMM in configuration T.
 template <typename T>
 bi_status launch_pair(bi::GemmParams p, const void *A, int64_t lda, const void *B, int64_t ldb, int b_layout,
@@ -639,7 +665,7 @@ bi_status bi_decode_attention(const void *q, const void *k_cache, const void *v_
     if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Lmax <= 0) return B == 0 ? BI_OK : BI_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return BI_ERR_INVALID_ARG;
     const int64_t group = Hq / Hkv;
-    if (D != bi::kAttnD || (group != 1 && group != 2 && group != 4 && group != 8)) return BI_ERR_UNSUPPORTED;
+    if ((D != 64 && D != 128) || (group != 1 && group != 2 && group != 4 && group != 8)) return BI_ERR_UNSUPPORTED;
     if (B > 65535 || Hkv > 65535 || Hq > 65535 || bi::attn_splits(Lmax) > kI32Max) return BI_ERR_UNSUPPORTED;
     if (B * Hkv * bi::attn_splits(Lmax) > kI32Max) return BI_ERR_UNSUPPORTED;  // work items are 32-bit indices
     if (B == 0) return BI_OK;
@@ -676,17 +702,9 @@ bi_status bi_decode_attention(const void *q, const void *k_cache, const void *v_
     const int64_t items = B * Hkv * S;
     const dim3 grid((unsigned)(items < dev->sms ? items : dev->sms));
     const size_t smem = (size_t)bi::kAttnSmem;
-    switch (Hq / Hkv) {  // the group size is a property of the model, not of the batch
-    case 1: st = launch_pdl(bi::decode_attention_split_kernel<1>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
-    case 2: st = launch_pdl(bi::decode_attention_split_kernel<2>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
-    case 4: st = launch_pdl(bi::decode_attention_split_kernel<4>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
-    case 8: st = launch_pdl(bi::decode_attention_split_kernel<8>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
-    default: return BI_ERR_UNSUPPORTED;
-    }
-    if (st != BI_OK) return st;
-    return launch_pdl(bi::decode_attention_combine_kernel, dim3((unsigned)Hq, (unsigned)B), dim3(bi::kAttnD), 0, s,
-                      static_cast<const float2 *>(p.part_ms), static_cast<const float *>(p.part_acc), seq_lens,
-                      static_cast<__nv_bfloat16 *>(out), (int)Hq, Lmax);
+    // The group size and the head size are properties of the model, not of the batch.
+    return D == 64 ? launch_attention<64>(Hq / Hkv, grid, smem, s, tm_k, tm_v, p, seq_lens, out, B)
+                   : launch_attention<128>(Hq / Hkv, grid, smem, s, tm_k, tm_v, p, seq_lens, out, B);
 }
 
 bi_status bi_silu_mul(const void *gu, void *h, int64_t M, int64_t F, void *stream)

@@ -94,7 +94,7 @@ def test_host_validation_without_a_gpu(lib):
     assert lib.bi_selftest_wait_timeout(10, NULL) == I
     # decode attention: shapes the kernel does not take are refused before any pointer is read
     da = lib.bi_decode_attention
-    assert da(fake, fake, fake, fake, fake, 2, 32, 8, 64, 128, 1.0, fake, 1 << 20, NULL) == U  # D != 128
+    assert da(fake, fake, fake, fake, fake, 2, 32, 8, 96, 128, 1.0, fake, 1 << 20, NULL) == U  # D not 64 or 128
     assert da(fake, fake, fake, fake, fake, 2, 24, 8, 128, 128, 1.0, fake, 1 << 20, NULL) == U  # group 3
     assert da(fake, fake, fake, fake, fake, 2, 30, 8, 128, 128, 1.0, fake, 1 << 20, NULL) == I  # Hq % Hkv
     # B * Hkv * splits must stay below 2^31 (work items are 32-bit indices)

@@ -17,10 +17,10 @@ DEV = "cuda"
 D = 128
 
 
-def make(seed, B, Hq, Hkv, Lmax):
-    q = inputs.rows_normal(seed, 0, B * Hq, D).view(B, Hq, D)
-    k = inputs.rows_normal(seed + 1, 0, B * Lmax * Hkv, D).view(B, Lmax, Hkv, D)
-    v = inputs.rows_normal(seed + 2, 0, B * Lmax * Hkv, D).view(B, Lmax, Hkv, D)
+def make(seed, B, Hq, Hkv, Lmax, d=D):
+    q = inputs.rows_normal(seed, 0, B * Hq, d).view(B, Hq, d)
+    k = inputs.rows_normal(seed + 1, 0, B * Lmax * Hkv, d).view(B, Lmax, Hkv, d)
+    v = inputs.rows_normal(seed + 2, 0, B * Lmax * Hkv, d).view(B, Lmax, Hkv, d)
     return q, k, v
 
 
@@ -51,6 +51,32 @@ def test_attention_batch_beyond_the_cached_lengths():
         alone = bi.bi_decode_attention(qd[i:i + 1], kd[i:i + 1], vd[i:i + 1], ld[i:i + 1])
         assert same_bits(alone, o[i:i + 1]), f"sequence {i}"
     assert bi.bi_get_device_status() == bi.BI_OK
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (16, 2), (8, 8)])
+@pytest.mark.parametrize("lens", [[1, 128, 300], [511, 512, 513, 1100]])
+def test_attention_parity_head_size_64(Hq, Hkv, lens):
+    """Head size 64 (one 64-wide TMA box per tile) against the oracle, at stage and split edges."""
+    B, Lmax = len(lens), max(lens) + 3
+    q, k, v = make(830, B, Hq, Hkv, Lmax, d=64)
+    sl = torch.tensor(lens, dtype=torch.int32)
+    o = bi.bi_decode_attention(q.to(DEV), k.to(DEV), v.to(DEV), sl.to(DEV))
+    ref = oracle.decode_attention(bf16_bits_np(q), bf16_bits_np(k), bf16_bits_np(v), sl.numpy(), 64 ** -0.5)
+    assert_bf16_close(o, ref, f"attention D=64 Hq={Hq} Hkv={Hkv} lens={lens}")
+    assert bi.bi_get_device_status() == bi.BI_OK
+
+
+def test_attention_head_size_64_invariance_and_repeats():
+    P, Hq, Hkv, Lmax = 24, 16, 4, 1100
+    q, k, v = make(831, P, Hq, Hkv, Lmax, d=64)
+    lens = torch.tensor(inputs.batch_sizes(832, P, 1, Lmax), dtype=torch.int32)
+    qd, kd, vd, ld = q.to(DEV), k.to(DEV), v.to(DEV), lens.to(DEV)
+    ref = torch.cat([bi.bi_decode_attention(qd[i:i + 1], kd[i:i + 1], vd[i:i + 1], ld[i:i + 1]) for i in range(P)])
+    for t, b in enumerate(inputs.batch_sizes(833, 10, 1, P)):
+        idx = inputs.permutation(834 + t, P)[:b].to(DEV)
+        assert same_bits(bi.bi_decode_attention(qd[idx], kd[idx], vd[idx], ld[idx]), ref[idx]), f"trial {t}"
+    for _ in range(20):
+        assert same_bits(bi.bi_decode_attention(qd, kd, vd, ld), ref)
 
 
 def test_attention_long_sequences_sampled():
@@ -115,11 +141,11 @@ def test_attention_bad_lengths_are_reported():
 
 
 def test_attention_argument_errors():
-    q = torch.zeros(2, 8, 64, dtype=torch.bfloat16, device=DEV)
-    kv = torch.zeros(2, 16, 2, 64, dtype=torch.bfloat16, device=DEV)
+    q = torch.zeros(2, 8, 96, dtype=torch.bfloat16, device=DEV)
+    kv = torch.zeros(2, 16, 2, 96, dtype=torch.bfloat16, device=DEV)
     sl = torch.ones(2, dtype=torch.int32, device=DEV)
     with pytest.raises(bi.BiError) as e:
-        bi.bi_decode_attention(q, kv, kv, sl)  # D = 64: only D = 128 is built
+        bi.bi_decode_attention(q, kv, kv, sl)  # D = 96: head sizes 64 and 128 are built
     assert e.value.status == bi.BI_ERR_UNSUPPORTED
     q = torch.zeros(2, 6, D, dtype=torch.bfloat16, device=DEV)
     kv = torch.zeros(2, 16, 4, D, dtype=torch.bfloat16, device=DEV)

@@ -118,8 +118,9 @@ def test_log_softmax_variants_stay_in_bounds(V):
         y.check(f"bi_log_softmax_cluster V={V}")
 
 
-def test_decode_attention_outputs_stay_in_bounds():
-    B, Hq, Hkv, D, Lmax = 3, 16, 4, 128, 300
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_attention_outputs_stay_in_bounds(D):
+    B, Hq, Hkv, Lmax = 3, 16, 4, 300
     q = inputs.rows_normal(1108, 0, B * Hq, D).view(B, Hq, D).to(DEV)
     k = inputs.rows_normal(1109, 0, B * Lmax * Hkv, D).view(B, Lmax, Hkv, D).to(DEV)
     v = inputs.rows_normal(1110, 0, B * Lmax * Hkv, D).view(B, Lmax, Hkv, D).to(DEV)
