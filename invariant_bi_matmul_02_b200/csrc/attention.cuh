@@ -167,14 +167,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     decode_attention_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                                   const AttnParams p)
 {
-    static_assert(D == 64 || D == 128, "head size 64 or 128: one or two 64-wide TMA boxes per tile");
-    constexpr int kBoxes = D / 64;                      // 64-d TMA boxes per K or V tile
-    constexpr int kTileBytes = kBoxes * kAttnBoxBytes;  // bytes one K or V tile of a stage carries
+    static_assert(D == 64 || D == 128, "head size 64 or 128");
+    // A K or V tile is two 64-d TMA boxes of 128 tokens.  D = 128: both halves of the same 128
+    // tokens' rows.  D = 64: two consecutive 128-token pieces, so a stage carries as many bytes.
+    constexpr int kPieces = D == 64 ? 2 : 1;            // 128-token pieces per stage
     extern __shared__ uint8_t attn_raw[];
     uint8_t *smem = attn_raw + ((1024u - (smem_addr(attn_raw) & 1023u)) & 1023u);
     __shared__ uint64_t kfull[kAttnStages], vfull[kAttnStages], empty[kAttnStages];
     __shared__ float red_m_all[kAttnGroups][kAttnConsumers][8];  // per-warp maxima of the 8 head rows
     __shared__ float red_s_all[kAttnGroups][kAttnConsumers][8];  // per-warp sums of exp
+    __shared__ float mrun_all[kAttnGroups][8];                   // a split's running maxima, per head
     __shared__ int abort_flag_s;
     __shared__ int slot_use_s[kAttnStages];  // uses of each ring slot that a consumer group has passed
     // Every role walks all of the CTA's items and needs each one's sequence length: read once here
@@ -227,21 +229,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const int64_t t0 = (int64_t)split * kAttnSplit, L = attn_len(p, b, false, lens_s);
                 if (t0 >= L) continue;
                 // The split's stages in token order; each carries the group's query rows too.
-                const int nc = attn_chunks(L - t0);
-                for (int c = 0; c < nc; ++c) {
-                    const int32_t tc = (int32_t)(t0 + (int64_t)c * kAttnChunk);
+                const int nc = attn_chunks(L - t0), ns = (nc + kPieces - 1) / kPieces;
+                for (int c = 0; c < ns; ++c) {
+                    const int32_t tc = (int32_t)(t0 + (int64_t)c * kPieces * kAttnChunk);
                     if (!(ok = wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, lim))) break;
-                    mbar_arrive_expect_tx(&kfull[stage], G * D * 2 + kTileBytes);
+                    mbar_arrive_expect_tx(&kfull[stage], G * D * 2 + kAttnTileBytes);
                     for (int j = 0; j < G; ++j)
                         bulk_load(q_rows(stage) + j * kAttnQStride,
                                   p.q + ((int64_t)b * p.Hq + (int64_t)g * G + j) * D, D * 2, &kfull[stage]);
+                    // Box x: d offset 64 x (D = 128), or tokens tc + 128 x (D = 64; past the sequence
+                    // the box is loaded but never read).
 #pragma unroll
-                    for (int x = 0; x < kBoxes; ++x)
-                        tma_load_4d(k_tile(stage) + x * kAttnBoxBytes, &tm_k, &kfull[stage], 64 * x, g, tc, b);
-                    mbar_arrive_expect_tx(&vfull[stage], kTileBytes);
+                    for (int x = 0; x < 2; ++x)
+                        tma_load_4d(k_tile(stage) + x * kAttnBoxBytes, &tm_k, &kfull[stage], kPieces == 1 ? 64 * x : 0, g,
+                                    tc + (kPieces == 1 ? 0 : x * kAttnChunk), b);
+                    mbar_arrive_expect_tx(&vfull[stage], kAttnTileBytes);
 #pragma unroll
-                    for (int x = 0; x < kBoxes; ++x)
-                        tma_load_4d(v_tile(stage) + x * kAttnBoxBytes, &tm_v, &vfull[stage], 64 * x, g, tc, b);
+                    for (int x = 0; x < 2; ++x)
+                        tma_load_4d(v_tile(stage) + x * kAttnBoxBytes, &tm_v, &vfull[stage], kPieces == 1 ? 64 * x : 0, g,
+                                    tc + (kPieces == 1 ? 0 : x * kAttnChunk), b);
                     ++issued;
                     advance(stage, phase, kAttnStages);
                 }
@@ -278,9 +284,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int64_t t0 = (int64_t)split * kAttnSplit;
             const int64_t L = attn_len(p, b, ct == 0 && grp == 0 && split == 0, lens_s);
             if (t0 >= L) continue;
-            const int nc = attn_chunks(L - t0);
+            const int nc = attn_chunks(L - t0), ns = (nc + kPieces - 1) / kPieces;
             const uint32_t mine = local++, first = q0;
-            q0 += (uint32_t)nc;
+            q0 += (uint32_t)ns;
             if (mine % kAttnGroups != (uint32_t)grp) continue;
 
             // Per head (row gid of the score tiles): the running maximum over the split's stages so
@@ -294,14 +300,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) o[mt][e] = 0.0f;
             int stage = 0;
-            for (int c = 0; c < nc; ++c) {
+            for (int c = 0; c < ns; ++c) {
                 const uint32_t qn = first + (uint32_t)c;
                 stage = (int)(qn % kAttnStages);
                 const uint32_t use = qn / kAttnStages;
-                const int64_t tc = t0 + (int64_t)c * kAttnChunk;
-                const int n_tok = (int)(L - tc < kAttnChunk ? L - tc : kAttnChunk);
-                const uint8_t *ks = k_tile(stage);
-                uint8_t *vs = v_tile(stage);
                 const __nv_bfloat16 *qs = q_rows(stage);
                 // Uses of a slot are passed in order: once the slot's previous use has been passed
                 // (by either group), the slot's barriers are at most one phase from the one wanted,
@@ -313,6 +315,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     break;
                 }
                 if (ct == 0) slot_use[stage] = (int)use + 1;
+
+              // The stage's 128-token pieces in token order (one for D = 128, two for D = 64); the
+              // piece's K and V rows start at box hp of the tile.
+              for (int hp = 0; hp < kPieces && c * kPieces + hp < nc; ++hp) {
+                const int64_t tc = t0 + (int64_t)(c * kPieces + hp) * kAttnChunk;
+                const int n_tok = (int)(L - tc < kAttnChunk ? L - tc : kAttnChunk);
+                const uint8_t *ks = k_tile(stage) + hp * kAttnBoxBytes;
+                uint8_t *vs = v_tile(stage) + hp * kAttnBoxBytes;
 
                 // ---- scores: acc[nt] is the 16 x 8 tile (heads x tokens 32 cw + 8 nt ..)
                 float acc[4][4];
@@ -386,7 +396,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         o[mt][3] = __fmul_rn(o[mt][3], a1);
                     }
                 }
-                if (!consumers_all(bar_id, wait_bounded(&vfull[stage], use & 1u, abort_flag, p.status, lim))) {
+                if (hp == 0 && !consumers_all(bar_id, wait_bounded(&vfull[stage], use & 1u, abort_flag, p.status, lim))) {
                     alive = false;
                     break;
                 }
@@ -429,7 +439,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         mma_16816_bf16(o[dt / 2], va, pb_lo0, pb_lo1);
                     }
                 }
-                if (c + 1 < nc) {
+              }
+                if (!alive) break;
+                if (c + 1 < ns) {
                     // Release the stage, one arrival per warp: the generic-proxy writes into it
                     // (zeroed rows) are ordered before the next TMA writes.
                     fence_proxy_async_smem();
@@ -443,8 +455,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // that stage's maxima barrier) holds the per-warp outputs, rows kAttnOStride floats
             // apart: a store's lanes cover d 16 mt + gid (+ 8) of heads 2 tig (+ 1); for up to four
             // heads, rows 0 and 2 (or 1 and 3) sit 16 banks apart, so the 16 lanes that store land in
-            // distinct banks; eight heads share banks two ways.  Every warp has read the maxima of
-            // the last stage, so red_m[0] can take the running maxima and red_s the warps' sums.
+            // distinct banks; eight heads share banks two ways.  The running maxima and the warps'
+            // sums go to arrays that nothing else reads before the barrier below.
             float *so = reinterpret_cast<float *>(const_cast<uint8_t *>(k_tile(stage)));
 #pragma unroll
             for (int mt = 0; mt < D / 16; ++mt)
@@ -457,7 +469,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 float l = __fadd_rn(l_t, __shfl_xor_sync(0xffffffffu, l_t, 1));
                 l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, 2));
                 if (tig == 0) red_s[cw][gid] = l;
-                if (tig == 0 && cw == 0) red_m[0][gid] = m_run;
+                if (tig == 0 && cw == 0) mrun_all[grp][gid] = m_run;
             }
             consumers_sync(bar_id);
 #pragma unroll
@@ -472,7 +484,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (ct == 0) {
                     float l = red_s[0][j];
                     for (int w = 1; w < kAttnConsumers; ++w) l = __fadd_rn(l, red_s[w][j]);
-                    p.part_ms[bh * p.S + split] = make_float2(red_m[0][j], l);
+                    p.part_ms[bh * p.S + split] = make_float2(mrun_all[grp][j], l);
                 }
             }
             // Release the last stage, one arrival per warp: the generic-proxy writes into it
