@@ -9,9 +9,10 @@
 // not on the batch it is decoded in, its position there, or which CTA computes a split.
 //
 // Launch 1 is a persistent, warp-specialised kernel: one CTA per SM walks the (split, kv head,
-// sequence) work items round-robin.  Its producer warp stages each split, kAttnChunk tokens at a
-// time, as the group's query rows (bulk copies) and K and V tiles (4-D TMA tensor loads, 128-byte
-// swizzle) into a ring of kAttnStages shared-memory stages, each completing on mbarriers.  Two
+// sequence) work items round-robin.  Its producer warp stages each split as the group's query
+// rows (bulk copies) and K and V tiles (4-D TMA tensor loads of 128 tokens x 64 d boxes, 128-byte
+// swizzle) into a ring of kAttnStages shared-memory stages, each completing on mbarriers; a stage
+// holds 128 tokens of head size 128, or 256 tokens (two pieces of 128) of head size 64.  Two
 // groups of four consumer warps take the CTA's splits alternately, so one group's compute
 // overlaps the other's and the loads of the next stages.  The cache streams from HBM without a
 // gap between items.  A split of kAttnSplit tokens keeps the partial results (written by launch 1,
@@ -150,13 +151,14 @@ __device__ __forceinline__ bool wait_flag_at_least(volatile int *flag, int v, vo
 // shared memory.  Work item i: split i % S, kv head (i / S) % Hkv, sequence i / (S Hkv); items
 // past their sequence's length have no partial and are skipped by every role alike.
 //
-// Arithmetic per split (mma.sync m16n8k16, bf16 in, fp32 accumulate), over its stages of
-// kAttnChunk tokens in ascending order; warp w owns tokens 32w .. 32w+31 of each stage.  Scores:
+// Arithmetic per split (mma.sync m16n8k16, bf16 in, fp32 accumulate), over its pieces of
+// kAttnChunk tokens in ascending order (one or two per ring stage, by the head size; the
+// arithmetic is the same either way); warp w owns tokens 32w .. 32w+31 of each piece.  Scores:
 // S = Q . K^T with Q the group's heads padded to 16 rows; every score accumulates its eight
-// 16-wide D steps in ascending order.  Per head and stage, the stage's maximum comes from a fixed
+// 16-wide D steps in ascending order.  Per head and piece, the piece's maximum comes from a fixed
 // tree (a thread's own values in order, the lane quad xor 1, 2, the warps in order) and raises the
 // running maximum m; what is accumulated so far -- each thread's sum of exp(s - m) and each warp's
-// weighted sums -- is multiplied by exp(m_old - m) (0 at the first stage), then the stage's
+// weighted sums -- is multiplied by exp(m_old - m) (0 at the first piece), then the piece's
 // exp(s - m) are added in order.  Weighted sums: O_w^T += V_w^T . P_w^T with P split into two bf16
 // terms (about 16 significant bits), two 16-token steps in ascending order.  At the split's end the
 // threads' sums meet in the lane quad (xor 1, 2), then the four warps' sums and O_w are added in
