@@ -148,8 +148,9 @@ __device__ __forceinline__ bool wait_flag_at_least(volatile int *flag, int v, vo
 }
 
 // Launch 1: grid = min(work items, SMs) CTAs of kAttnThreads threads, kAttnSmem bytes of dynamic
-// shared memory.  Work item i: split i % S, kv head (i / S) % Hkv, sequence i / (S Hkv); items
-// past their sequence's length have no partial and are skipped by every role alike.
+// shared memory.  Work item i: for D = 128 kv head i % Hkv, split (i / Hkv) % S, sequence
+// i / (Hkv S); for D = 64 split i % S, kv head (i / S) % Hkv, sequence i / (S Hkv).  Items past
+// their sequence's length have no partial and are skipped by every role alike.
 //
 // Arithmetic per split (mma.sync m16n8k16, bf16 in, fp32 accumulate), over its pieces of
 // kAttnChunk tokens in ascending order (one or two per ring stage, by the head size; the
@@ -217,6 +218,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // The host guarantees B * Hkv * S < 2^31, so item indices and their coordinates are 32-bit.
     const uint32_t items = (uint32_t)p.B * (uint32_t)p.Hkv * (uint32_t)p.S;
     const uint32_t n_splits = (uint32_t)p.S, n_kv = (uint32_t)p.Hkv;
+    // Item order (a property of the head size, not of the batch; no item's arithmetic depends on
+    // it): D = 128, kv head fastest, so the heads of the same tokens -- adjacent pieces of the same
+    // cache rows -- are fetched by neighbouring CTAs at about the same time; D = 64, split fastest
+    // (measured faster there).
+    auto item_coords = [&](uint32_t it, int &split, int &g, int &b) {
+        if (D == 128) {
+            const uint32_t sg = it / n_kv;
+            g = (int)(it - sg * n_kv);
+            split = (int)(sg % n_splits);
+            b = (int)(sg / n_splits);
+        } else {
+            const uint32_t sg = it / n_splits;
+            split = (int)(it - sg * n_splits);
+            g = (int)(sg % n_kv);
+            b = (int)(sg / n_kv);
+        }
+    };
     const uint64_t lim = p.wait_limit_ns;
 
     if (warp == 0) {
@@ -226,8 +244,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             int issued = 0;
             bool ok = true;
             for (uint32_t it = blockIdx.x; ok && it < items; it += gridDim.x) {
-                const uint32_t sg = it / n_splits;
-                const int split = (int)(it - sg * n_splits), g = (int)(sg % n_kv), b = (int)(sg / n_kv);
+                int split, g, b;
+                item_coords(it, split, g, b);
                 const int64_t t0 = (int64_t)split * kAttnSplit, L = attn_len(p, b, false, lens_s);
                 if (t0 >= L) continue;
                 // The split's stages in token order; each carries the group's query rows too.
@@ -281,8 +299,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint32_t local = 0, q0 = 0;  // the split's local index and its first stage number
         bool alive = true;
         for (uint32_t it = blockIdx.x; alive && it < items; it += gridDim.x) {
-            const uint32_t sg = it / n_splits;
-            const int split = (int)(it - sg * n_splits), g = (int)(sg % n_kv), b = (int)(sg / n_kv);
+            int split, g, b;
+            item_coords(it, split, g, b);
             const int64_t t0 = (int64_t)split * kAttnSplit;
             const int64_t L = attn_len(p, b, ct == 0 && grp == 0 && split == 0, lens_s);
             if (t0 >= L) continue;
