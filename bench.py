@@ -675,6 +675,33 @@ def metric_sweep(device, peaks: dict, reps: int = 10) -> dict:
                                    "torch_rows_differing_from_m1": _rows_differing(ft(xm).reshape(M, -1),
                                                                                    tref[:n])})
         del x, ref, tref
+    # Decode attention (f2) at the Qwen3-8B decode shape, B = 64 sequences of L = 4096 cached
+    # tokens, 32 query / 8 kv heads, head sizes 128 and 64, against torch SDPA; the first 8
+    # sequences are also decoded alone, for both.
+    out["attention"] = []
+    for D in (128, 64):
+        B, L, Hq, Hkv = 64, 4096, 32, 8
+        q = torch.randn(B, Hq, D, generator=g, device=device).to(torch.bfloat16)
+        k = torch.randn(B, L, Hkv, D, generator=g, device=device).to(torch.bfloat16)
+        v = torch.randn(B, L, Hkv, D, generator=g, device=device).to(torch.bfloat16)
+        sl = torch.full((B,), L, dtype=torch.int32, device=device)
+        scr = torch.empty(bi.bi_decode_attention_scratch_bytes(B, Hq, D, L), dtype=torch.uint8, device=device)
+        o = torch.empty_like(q)
+        sdpa = lambda qq, kk, vv: F.scaled_dot_product_attention(qq.view(qq.shape[0], Hq, 1, D), kk.permute(0, 2, 1, 3),
+                                                                 vv.permute(0, 2, 1, 3), enable_gqa=True).view(qq.shape)
+        t_bi = us(lambda: bi.bi_decode_attention(q, k, v, sl, scratch=scr, out=o))
+        t_t = us(lambda: sdpa(q, k, v))
+        alone = torch.cat([bi.bi_decode_attention(q[i:i + 1], k[i:i + 1], v[i:i + 1], sl[i:i + 1]) for i in range(8)])
+        talone = torch.cat([sdpa(q[i:i + 1], k[i:i + 1], v[i:i + 1]) for i in range(8)])
+        nbytes = 2.0 * B * L * Hkv * D * 2
+        out["attention"].append({"op": "decode_attention", "B": B, "L": L, "Hq": Hq, "Hkv": Hkv, "D": D,
+                                 "bi_us": round(t_bi, 1), "gbs": round(nbytes / t_bi / 1e3, 1),
+                                 "hbm_frac": round(nbytes / t_bi / 1e3 / peaks["hbm_gbs"], 3),
+                                 "torch_sdpa_us": round(t_t, 1),
+                                 "rows_differing_from_alone": _rows_differing(o.reshape(B, -1), alone.reshape(8, -1)),
+                                 "torch_rows_differing_from_alone": _rows_differing(sdpa(q, k, v).reshape(B, -1),
+                                                                                    talone.reshape(8, -1))})
+        del q, k, v, scr, o, alone, talone
     del flush_buf
     torch.cuda.empty_cache()
     return out
