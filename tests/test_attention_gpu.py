@@ -37,7 +37,7 @@ def test_attention_parity(Hq, Hkv, lens):
 
 
 def test_attention_batch_beyond_the_cached_lengths():
-    """Launch 1 keeps the first 4096 sequence lengths in shared memory and reads the others from
+    """The kernel keeps the first 4096 sequence lengths in shared memory and reads the others from
     global memory: a batch of 5000 short sequences of mixed lengths checks both paths against the
     oracle, and a sequence past the cache gives the same bits as when it is decoded alone."""
     B, Hq, Hkv, Lmax = 5000, 1, 1, 3
@@ -129,6 +129,55 @@ def test_attention_repeatable_100_runs():
     first = bi.bi_decode_attention(qd, kd, vd, sl, scratch=scratch)
     for _ in range(100):
         assert same_bits(bi.bi_decode_attention(qd, kd, vd, sl, scratch=scratch), first)
+
+
+def test_attention_scratch_contents_do_not_matter():
+    """The splits' partial results live in caller scratch of any contents: random bytes, all
+    ones, or 64-bit words with the top bit set give the bits of a zeroed scratch, also on a
+    second call over what the first one left."""
+    B, Hq, Hkv, Lmax = 6, 16, 4, 2600
+    q, k, v = make(840, B, Hq, Hkv, Lmax)
+    sl = torch.tensor([2600, 1, 512, 513, 2047, 1500], dtype=torch.int32).to(DEV)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    n = bi.bi_decode_attention_scratch_bytes(B, Hq, D, Lmax)
+    assert n % 8 == 0
+    scratch = torch.zeros(n, dtype=torch.uint8, device=DEV)
+    ref = bi.bi_decode_attention(qd, kd, vd, sl, scratch=scratch)
+    rng = np.random.default_rng(841)
+    stale = rng.integers(0, 1 << 62, n // 8, dtype=np.uint64) | np.uint64(1 << 63)
+    fills = [rng.integers(0, 256, n, dtype=np.uint8), np.full(n, 255, dtype=np.uint8), stale.view(np.uint8)]
+    for i, f in enumerate(fills):
+        scratch.copy_(torch.from_numpy(f).to(DEV))
+        assert same_bits(bi.bi_decode_attention(qd, kd, vd, sl, scratch=scratch), ref), f"fill {i}"
+        assert same_bits(bi.bi_decode_attention(qd, kd, vd, sl, scratch=scratch), ref), f"fill {i}, again"
+    assert bi.bi_get_device_status() == bi.BI_OK
+
+
+def test_attention_replayed_from_a_cuda_graph():
+    """Both launches of a call (the second dependent on the first through programmatic
+    dependent launch) capture into a CUDA graph; new query rows before each replay give the
+    bits of an eager call."""
+    B, Hq, Hkv, Lmax = 8, 16, 4, 1500
+    q, k, v = make(842, B, Hq, Hkv, Lmax)
+    sl = torch.tensor(inputs.batch_sizes(843, B, 1, Lmax), dtype=torch.int32).to(DEV)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    scratch = torch.empty(bi.bi_decode_attention_scratch_bytes(B, Hq, D, Lmax), dtype=torch.uint8, device=DEV)
+    out = torch.empty_like(qd)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        bi.bi_decode_attention(qd, kd, vd, sl, scratch=scratch, out=out)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        bi.bi_decode_attention(qd, kd, vd, sl, scratch=scratch, out=out)
+    for t in range(6):
+        qd.copy_(inputs.rows_normal(844 + t, 0, B * Hq, D).view(B, Hq, D).to(DEV))
+        graph.replay()
+        eager = bi.bi_decode_attention(qd, kd, vd, sl)
+        assert same_bits(out, eager), f"replay {t}"
+    del graph
+    assert bi.bi_get_device_status() == bi.BI_OK
 
 
 def test_attention_bad_lengths_are_reported():
