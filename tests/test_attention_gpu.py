@@ -88,6 +88,25 @@ def test_attention_long_sequences_sampled():
     assert_bf16_close(o, ref, "attention Lmax=4096")
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_attention_more_than_eight_splits(d):
+    """Sequences of more than 8 splits of 512 tokens (the second launch folds them in chunks of
+    weights staged in shared memory) and of exactly 8, against the oracle; each sequence alone,
+    in a cache cut to its own length, gives the bits it has in the batch."""
+    B, Hq, Hkv, Lmax = 3, 8, 2, 6000
+    q, k, v = make(850, B, Hq, Hkv, Lmax, d=d)
+    sl = torch.tensor([6000, 4097, 4096], dtype=torch.int32)
+    qd, kd, vd, ld = q.to(DEV), k.to(DEV), v.to(DEV), sl.to(DEV)
+    o = bi.bi_decode_attention(qd, kd, vd, ld)
+    ref = oracle.decode_attention(bf16_bits_np(q), bf16_bits_np(k), bf16_bits_np(v), sl.numpy(), d ** -0.5)
+    assert_bf16_close(o, ref, f"attention D={d} lens={sl.tolist()}")
+    for i in range(B):
+        alone = bi.bi_decode_attention(qd[i:i + 1], kd[i:i + 1, :int(sl[i])].contiguous(),
+                                       vd[i:i + 1, :int(sl[i])].contiguous(), ld[i:i + 1])
+        assert same_bits(alone, o[i:i + 1]), f"sequence {i}"
+    assert bi.bi_get_device_status() == bi.BI_OK
+
+
 def test_attention_batch_invariance_over_compositions():
     P, Hq, Hkv, Lmax = 48, 32, 8, 1024
     q, k, v = make(802, P, Hq, Hkv, Lmax)
