@@ -745,8 +745,22 @@ def run_host_overhead(args):
     h1, m1 = bi.bi_tensor_map_cache_stats()
     miss = host_us(lambda i: pool[(i * 7) % 4096:(i * 7) % 4096 + 1])
     h2, m2 = bi.bi_tensor_map_cache_stats()
+    # The C entry point alone (ctypes call with prepared arguments, maps cached): what the
+    # binding's checks add is the difference.
+    lib = bi.load()
+    c_args = (pool.data_ptr(), K, w.data_ptr(), K, bi.BI_B_NK, c.data_ptr(), N, bi.BI_BF16, 1, N, K,
+              torch.cuda.current_stream().cuda_stream)
+    for _ in range(50):
+        lib.bi_matmul(*c_args)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        lib.bi_matmul(*c_args)
+    c_abi = (time.perf_counter() - t0) / calls * 1e6
+    torch.cuda.synchronize()
     print(json.dumps({"host_overhead": "bi_matmul M=1 K=N=256 through the binding",
                       "host_us_per_call_cache_hit": round(hit, 2), "host_us_per_call_one_miss": round(miss, 2),
+                      "host_us_per_call_c_abi_only": round(c_abi, 2),
                       "hits_misses_hit_loop": [h1 - h0, m1 - m0], "hits_misses_miss_loop": [h2 - h1, m2 - m1]}))
 
 

@@ -88,17 +88,26 @@ def _current_device() -> int:
     return torch.cuda.current_device()
 
 
-def _same_device(index: int, name: str):
+def _same_device(index: int, name: str, cur: int | None = None):
     """The library launches on the current device and looks up its per-device state there, so
-    every tensor and the stream of a call must live on that device."""
-    cur = _current_device()
+    every tensor and the stream of a call must live on that device.  `cur`: the current device,
+    when the caller has already looked it up."""
+    if cur is None:
+        cur = _current_device()
     if index != cur:
         raise ValueError(f"{name} is on cuda:{index} but the current device is cuda:{cur}; "
                          "call under `with torch.cuda.device(...)`")
 
 
-def _stream(stream):
+# The current stream's raw handle without building a torch.cuda.Stream object (3 us per call on
+# the host otherwise); the public call where a torch build lacks it.
+_raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream, cur: int | None = None):
     if stream is None:
+        if _raw_current_stream is not None:
+            return _raw_current_stream(_current_device() if cur is None else cur)
         return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, torch.cuda.Stream):
         _same_device(stream.device.index, "stream")
@@ -106,21 +115,28 @@ def _stream(stream):
     return int(stream)
 
 
-def _need_cuda(t: torch.Tensor, name: str, dtypes):
+def _need_cuda(t: torch.Tensor, name: str, dtypes, cur: int | None = None) -> int:
+    """Check that t is a CUDA tensor of one of `dtypes` on the current device; returns the
+    current device, so that a call's other checks need not look it up again."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if t.dtype not in dtypes:
         raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
-    _same_device(t.get_device(), name)
+    if cur is None:
+        cur = _current_device()
+    _same_device(t.get_device(), name, cur)
+    return cur
 
 
 def _ld(t: torch.Tensor, name: str) -> int:
     """Leading dimension of a 2-D tensor with unit-stride rows."""
     if t.dim() != 2:
         raise ValueError(f"{name} must be 2-D")
-    if t.shape[1] > 1 and t.stride(1) != 1:
+    rows, cols = t.shape
+    s0, s1 = t.stride()
+    if cols > 1 and s1 != 1:
         raise ValueError(f"{name} rows must be contiguous")
-    return t.stride(0) if t.shape[0] > 1 else max(t.stride(0), t.shape[1])
+    return s0 if rows > 1 else max(s0, cols)
 
 
 def _contig(t: torch.Tensor, name: str):
@@ -147,17 +163,17 @@ def _gemm_shapes(a, b, b_layout):
 def bi_matmul(a: torch.Tensor, b: torch.Tensor, b_layout: str = "nk", out: torch.Tensor | None = None,
               out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
     """C = A . B (b_layout 'kn': B [K, N]; 'nk': B [N, K], i.e. C = A . B^T)."""
-    _need_cuda(a, "A", (torch.bfloat16,))
-    _need_cuda(b, "B", (torch.bfloat16,))
+    cur = _need_cuda(a, "A", (torch.bfloat16,))
+    _need_cuda(b, "B", (torch.bfloat16,), cur)
     M, N, K = _gemm_shapes(a, b, b_layout)
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=a.device)
-    _need_cuda(out, "C", (torch.bfloat16, torch.float32))
+    _need_cuda(out, "C", (torch.bfloat16, torch.float32), cur)
     if tuple(out.shape) != (M, N):
         raise ValueError("C must be [M, N]")
     st = load().bi_matmul(a.data_ptr(), _ld(a, "A"), b.data_ptr(), _ld(b, "B"),
                           BI_B_KN if b_layout == "kn" else BI_B_NK, out.data_ptr(), _ld(out, "C"),
-                          _DT[out.dtype], M, N, K, _stream(stream))
+                          _DT[out.dtype], M, N, K, _stream(stream, cur))
     _check("bi_matmul", st)
     return out
 
@@ -166,9 +182,9 @@ def bi_addmm(input: torch.Tensor, a: torch.Tensor, b: torch.Tensor, b_layout: st
              out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
              stream=None) -> torch.Tensor:
     """C = input + A . B; input is a bias [N] or a matrix [M, N] (bf16)."""
-    _need_cuda(a, "A", (torch.bfloat16,))
-    _need_cuda(b, "B", (torch.bfloat16,))
-    _need_cuda(input, "input", (torch.bfloat16,))
+    cur = _need_cuda(a, "A", (torch.bfloat16,))
+    _need_cuda(b, "B", (torch.bfloat16,), cur)
+    _need_cuda(input, "input", (torch.bfloat16,), cur)
     M, N, K = _gemm_shapes(a, b, b_layout)
     if input.dim() == 1:
         if input.shape[0] != N:
@@ -182,12 +198,12 @@ def bi_addmm(input: torch.Tensor, a: torch.Tensor, b: torch.Tensor, b_layout: st
         ld_in = _ld(input, "input")
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=a.device)
-    _need_cuda(out, "C", (torch.bfloat16, torch.float32))
+    _need_cuda(out, "C", (torch.bfloat16, torch.float32), cur)
     if tuple(out.shape) != (M, N):
         raise ValueError("C must be [M, N]")
     st = load().bi_addmm(input.data_ptr(), ld_in, a.data_ptr(), _ld(a, "A"), b.data_ptr(), _ld(b, "B"),
                          BI_B_KN if b_layout == "kn" else BI_B_NK, out.data_ptr(), _ld(out, "C"),
-                         _DT[out.dtype], M, N, K, _stream(stream))
+                         _DT[out.dtype], M, N, K, _stream(stream, cur))
     _check("bi_addmm", st)
     return out
 
@@ -196,20 +212,20 @@ def bi_matmul_silu_mul(a: torch.Tensor, b: torch.Tensor, b_layout: str = "nk",
                        out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """H = silu(A . gate) * (A . up) with B the stacked [gate; up] weight ('nk': [2F, K];
     'kn': [K, 2F]); the glue runs in the GEMM's epilogue."""
-    _need_cuda(a, "A", (torch.bfloat16,))
-    _need_cuda(b, "B", (torch.bfloat16,))
+    cur = _need_cuda(a, "A", (torch.bfloat16,))
+    _need_cuda(b, "B", (torch.bfloat16,), cur)
     M, N2, K = _gemm_shapes(a, b, b_layout)
     if N2 % 2:
         raise ValueError("B must stack gate and up: an even number of output rows")
     F = N2 // 2
     if out is None:
         out = torch.empty((M, F), dtype=torch.bfloat16, device=a.device)
-    _need_cuda(out, "H", (torch.bfloat16,))
+    _need_cuda(out, "H", (torch.bfloat16,), cur)
     if tuple(out.shape) != (M, F):
         raise ValueError("H must be [M, F]")
     st = load().bi_matmul_silu_mul(a.data_ptr(), _ld(a, "A"), b.data_ptr(), _ld(b, "B"),
                                    BI_B_KN if b_layout == "kn" else BI_B_NK, out.data_ptr(),
-                                   _ld(out, "H"), M, F, K, _stream(stream))
+                                   _ld(out, "H"), M, F, K, _stream(stream, cur))
     _check("bi_matmul_silu_mul", st)
     return out
 
