@@ -35,6 +35,7 @@ struct DeviceState {
     int sms = 0;
     int gemm_clusters_wide = 0;    // CTA pairs of each GEMM configuration that fit on the device at once
     int gemm_clusters_narrow = 0;
+    int mean_rows_blocks_per_sm = 0;  // co-resident 1024-thread blocks of the persistent mean
     int32_t *status = nullptr;
 };
 
@@ -98,6 +99,11 @@ bi_status device_state(DeviceState **out)
             pair_clusters<bi::NarrowTile>(d.sms, &d.gemm_clusters_narrow) != BI_OK)
             return BI_ERR_CUDA;
         if (attn_smem_opt_in<64>() != BI_OK || attn_smem_opt_in<128>() != BI_OK) return BI_ERR_CUDA;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.mean_rows_blocks_per_sm, bi::mean_rows_kernel,
+                                                          bi::kMeanRowsThreads, 0) !=
+                cudaSuccess ||
+            d.mean_rows_blocks_per_sm < 1)
+            return BI_ERR_CUDA;
         if (cudaFuncSetAttribute(bi::log_softmax_stream_kernel<true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bi::kLsmSmem) != cudaSuccess ||
             cudaFuncSetAttribute(bi::log_softmax_stream_kernel<false>,
@@ -501,11 +507,15 @@ bi_status bi_mean(const float *x, float *y, int64_t M, int64_t H, void *stream)
     bi_status st = BI_OK;
     if (H % 4 == 0) {
         if (!aligned16(x)) return BI_ERR_ALIGNMENT;
-        if (H / 4 >= 8 * (int64_t)T)
-            st = launch_pdl(bi::mean_vec_kernel<true>, dim3((unsigned)M), dim3(T), 0, s,
-                            reinterpret_cast<const float4 *>(x), y, H);
-        else
-            st = launch_pdl(bi::mean_vec_kernel<false>, dim3((unsigned)M), dim3(T), 0, s,
+        if (H / 4 >= 8 * (int64_t)T && T == bi::kMeanRowsThreads) {
+            DeviceState *dev = nullptr;
+            st = device_state(&dev);
+            if (st != BI_OK) return st;
+            const int64_t fit = (int64_t)dev->sms * dev->mean_rows_blocks_per_sm;
+            st = launch_pdl(bi::mean_rows_kernel, dim3((unsigned)(M < fit ? M : fit)), dim3(T), 0, s,
+                            reinterpret_cast<const float4 *>(x), y, H, M);
+        } else
+            st = launch_pdl(bi::mean_vec_kernel, dim3((unsigned)M), dim3(T), 0, s,
                             reinterpret_cast<const float4 *>(x), y, H);
         return st;
     }

@@ -161,12 +161,11 @@ __global__ void __launch_bounds__(1024) rmsnorm_scalar_kernel(const __nv_bfloat1
 // --------------------------------------------------------------- mean
 
 // Vector path: H % 4 == 0.  Chunk c (4 floats) belongs to thread c % T; each thread
-// keeps four running sums (one per float4 lane) and folds them as (s0+s1)+(s2+s3).
-// LONG: eight float4 loads in flight per thread (rows of >= 8 T groups, which run one 1024-thread
-// block per SM); otherwise four.  The adds keep the ascending group order in both, so the sums
-// are the same bits either way.  x is read once, with an evict-first hint, so the reads do not
-// push out of L2 the lines of x (e.g. the last rows a log_softmax just wrote) not yet read.
-template <bool LONG>
+// keeps four running sums (one per float4 lane), adds its chunks in ascending order with four
+// float4 loads in flight, and folds the sums as (s0+s1)+(s2+s3).  x is read once, with an
+// evict-first hint, so the reads do not push out of L2 the lines of x (e.g. the last rows a
+// log_softmax just wrote) not yet read.  Rows of at least 8 T chunks run mean_rows_kernel below,
+// whose per-row arithmetic is the same.
 __global__ void __launch_bounds__(1024) mean_vec_kernel(const float4 *__restrict__ x,
                                                        float *__restrict__ y, int64_t H)
 {
@@ -178,17 +177,6 @@ __global__ void __launch_bounds__(1024) mean_vec_kernel(const float4 *__restrict
     float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
     int64_t c = threadIdx.x;
     const int T = blockDim.x;
-    if (LONG) {
-        for (; c + 7 * (int64_t)T < nch; c += 8 * (int64_t)T) {
-            float4 g[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) g[k] = __ldcs(xr + c + k * (int64_t)T);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                s0 += g[k].x; s1 += g[k].y; s2 += g[k].z; s3 += g[k].w;
-            }
-        }
-    }
     for (; c + 3 * (int64_t)T < nch; c += 4 * (int64_t)T) {
         float4 a = __ldcs(xr + c), b = __ldcs(xr + c + T), d = __ldcs(xr + c + 2 * T),
                e = __ldcs(xr + c + 3 * T);
@@ -204,6 +192,67 @@ __global__ void __launch_bounds__(1024) mean_vec_kernel(const float4 *__restrict
     float s = __fadd_rn(__fadd_rn(s0, s1), __fadd_rn(s2, s3));
     s = block_sum(s, red);
     if (threadIdx.x == 0) y[blockIdx.x] = s / (float)H;
+}
+
+// Long rows (H / 4 >= 8 T), persistent: block b takes rows b, b + G, b + 2G, ... (G blocks, as
+// many as fit at once), so rows do not wait for block launches; eight float4 loads per thread are
+// in flight, and each block issues the first eight of its next row before the current row's
+// block reduction, so the reduction overlaps those reads.  Per row the arithmetic is
+// mean_vec_kernel's: thread t adds its chunks t, t + T, ... in ascending order into four running
+// sums, folds them as (s0+s1)+(s2+s3), and the block tree adds the threads' sums.  (B200, fp32
+// rows of 151936, L2 flushed: 103.9 us at M = 1024 against 108.6 us with a block per row; the
+// same bits.)
+constexpr int kMeanRowsThreads = 1024;  // the thread count mean_threads(H) gives every long row
+__global__ void __launch_bounds__(kMeanRowsThreads) mean_rows_kernel(const float4 *__restrict__ x, float *__restrict__ y,
+                                                        int64_t H, int64_t M)
+{
+    __shared__ float red[32];
+    griddep_wait();  // the previous kernel's output (x) is complete
+    griddep_launch_dependents();
+    const int nch = (int)(H / 4);  // H < 2^31
+    constexpr int T = kMeanRowsThreads;
+    int64_t row = blockIdx.x;
+    if (row >= M) return;
+    float4 g[8];
+    const float4 *xr = x + row * nch;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) g[k] = __ldcs(xr + threadIdx.x + k * T);
+    for (;;) {
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+        int c = threadIdx.x;
+        for (;;) {  // g holds groups c, c + T, ..., c + 7T
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                s0 += g[k].x; s1 += g[k].y; s2 += g[k].z; s3 += g[k].w;
+            }
+            c += 8 * T;
+            if (c + 7 * T >= nch) break;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) g[k] = __ldcs(xr + c + k * T);
+        }
+        for (; c + 3 * T < nch; c += 4 * T) {
+            float4 a = __ldcs(xr + c), b = __ldcs(xr + c + T), d = __ldcs(xr + c + 2 * T), e = __ldcs(xr + c + 3 * T);
+            s0 += a.x; s1 += a.y; s2 += a.z; s3 += a.w;
+            s0 += b.x; s1 += b.y; s2 += b.z; s3 += b.w;
+            s0 += d.x; s1 += d.y; s2 += d.z; s3 += d.w;
+            s0 += e.x; s1 += e.y; s2 += e.z; s3 += e.w;
+        }
+        for (; c < nch; c += T) {
+            float4 a = __ldcs(xr + c);
+            s0 += a.x; s1 += a.y; s2 += a.z; s3 += a.w;
+        }
+        const int64_t next = row + gridDim.x;
+        if (next < M) {
+            xr = x + next * nch;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) g[k] = __ldcs(xr + threadIdx.x + k * T);
+        }
+        float sum = __fadd_rn(__fadd_rn(s0, s1), __fadd_rn(s2, s3));
+        sum = block_sum(sum, red);
+        if (threadIdx.x == 0) y[row] = sum / (float)H;
+        if (next >= M) break;
+        row = next;
+    }
 }
 
 __global__ void __launch_bounds__(1024) mean_scalar_kernel(const float *__restrict__ x,
