@@ -19,9 +19,9 @@
  *
  * How each entry point fixes its order (the same for every M):
  *   - bi_matmul / bi_addmm: tcgen05/TMEM tiles fed by TMA; the tile width is a
- *     function of the output width N alone (bi_gemm_config), never of M; every
+ *     function of the weight's shape alone (bi_gemm_config), never of M; every
  *     output element accumulates its K products in fp32, 16 at a time, in
- *     ascending K, in either configuration; no split-K, no stream-K.
+ *     ascending K, in every configuration; no split-K, no stream-K.
  *   - bi_rmsnorm / bi_mean / bi_log_softmax: one thread block per row; the
  *     block size and each thread's element set depend only on the row length;
  *     partial results merge through a fixed warp-shuffle tree and a fixed
@@ -311,15 +311,19 @@ bi_status bi_selftest_wait_timeout(int64_t limit_ns, void *stream);
 const char *bi_status_string(bi_status status);
 
 /*
- * bi_gemm_config -- report the tile configuration the GEMM entry points use for an
- * output width n (the N of bi_matmul / bi_addmm, the F of bi_matmul_silu_mul): output
- * tile bm x bn, K per pipeline stage bk, number of stages, and the K step of one
- * tensor-core instruction.  The configuration depends on n alone -- every M of a
- * given weight matrix runs the same one -- and both configurations take the same
- * 16-wide K steps in ascending order, so an element's bits do not depend on it.
- * n <= 0 reports the configuration of wide outputs.  Any pointer may be NULL.
+ * bi_gemm_config -- report the tile configuration the GEMM entry points use for a
+ * weight of `weight_rows` rows in [N, K] (BI_B_NK) storage: N for bi_matmul /
+ * bi_addmm, 2F for bi_matmul_silu_mul.  It reports the output tile bm x bn, K per
+ * pipeline stage bk, the number of stages, and the K step of one tensor-core
+ * instruction.  bn is 128 up to 1024 rows. Above that it is 192 where 192-column
+ * tiles fill the B200's CTA pairs in fewer cost-weighted waves than 256-column tiles
+ * for a 1024-row batch (e.g. 6144 or 24576 rows), else 256. [K, N] (BI_B_KN)
+ * weights run bn = 256 where this reports 192.  The configuration depends on the
+ * weight alone -- every M of a given weight runs the same one -- and all
+ * configurations take the same 16-wide K steps in ascending order, so an element's
+ * bits do not depend on it.  weight_rows <= 0 reports bn = 256.  Any pointer may be NULL.
  */
-void bi_gemm_config(int64_t n, int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int32_t *mma_k);
+void bi_gemm_config(int64_t weight_rows, int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int32_t *mma_k);
 
 /*
  * bi_tensor_map_cache_stats -- how many TMA tensor-map look-ups of the GEMM entry points were

@@ -399,10 +399,11 @@ def bi_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
     _check("bi_selftest_wait_timeout", load().bi_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
 
-def bi_gemm_config(n: int = 0) -> dict:
-    """Tile configuration of the GEMM entry points for output width n (n <= 0: wide outputs)."""
+def bi_gemm_config(weight_rows: int = 0) -> dict:
+    """Tile configuration of the GEMM entry points for an [N, K] weight of `weight_rows` rows
+    (N of bi_matmul / bi_addmm, 2F of bi_matmul_silu_mul; <= 0: the 256-column tile)."""
     vals = [_i32(0) for _ in range(5)]
-    load().bi_gemm_config(int(n), *[ctypes.byref(v) for v in vals])
+    load().bi_gemm_config(int(weight_rows), *[ctypes.byref(v) for v in vals])
     return dict(zip(("bm", "bn", "bk", "stages", "mma_k"), (int(v.value) for v in vals)))
 
 

@@ -35,6 +35,7 @@ struct DeviceState {
     int sms = 0;
     int gemm_clusters_wide = 0;    // CTA pairs of each GEMM configuration that fit on the device at once
     int gemm_clusters_narrow = 0;
+    int gemm_clusters_mid = 0;
     int mean_rows_blocks_per_sm = 0;  // co-resident 1024-thread blocks of the persistent mean
     int32_t *status = nullptr;
 };
@@ -96,7 +97,8 @@ bi_status device_state(DeviceState **out)
         if (cudaGetSymbolAddress(&sym, g_bi_status) != cudaSuccess) return BI_ERR_CUDA;
         d.status = static_cast<int32_t *>(sym);
         if (pair_clusters<bi::WideTile>(d.sms, &d.gemm_clusters_wide) != BI_OK ||
-            pair_clusters<bi::NarrowTile>(d.sms, &d.gemm_clusters_narrow) != BI_OK)
+            pair_clusters<bi::NarrowTile>(d.sms, &d.gemm_clusters_narrow) != BI_OK ||
+            pair_clusters<bi::MidTile>(d.sms, &d.gemm_clusters_mid) != BI_OK)
             return BI_ERR_CUDA;
         if (attn_smem_opt_in<64>() != BI_OK || attn_smem_opt_in<128>() != BI_OK) return BI_ERR_CUDA;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.mean_rows_blocks_per_sm, bi::mean_rows_kernel,
@@ -391,8 +393,14 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
 
     // The tile configuration is a function of the output width N alone; every M of a given
     // weight runs the same one.
-    if (N <= bi::kNarrowMaxN)
+    switch (bi::pair_config(b_rows, b_layout == BI_B_NK)) {
+    case bi::kPairNarrow:
         return launch_pair<bi::NarrowTile>(p, A, lda, B, ldb, b_layout, b_rows, dev->gemm_clusters_narrow, s);
+    case bi::kPairMid:
+        return launch_pair<bi::MidTile>(p, A, lda, B, ldb, b_layout, b_rows, dev->gemm_clusters_mid, s);
+    default:
+        break;
+    }
     return launch_pair<bi::WideTile>(p, A, lda, B, ldb, b_layout, b_rows, dev->gemm_clusters_wide, s);
 }
 
@@ -772,13 +780,17 @@ const char *bi_status_string(bi_status status)
     return "BI_ERR_UNKNOWN";
 }
 
-void bi_gemm_config(int64_t n, int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int32_t *mma_k)
+void bi_gemm_config(int64_t weight_rows, int32_t *bm, int32_t *bn, int32_t *bk, int32_t *stages, int32_t *mma_k)
 {
-    const bool narrow = n > 0 && n <= bi::kNarrowMaxN;
+    const bi::PairConfig c = weight_rows > 0 ? bi::pair_config(weight_rows, true) : bi::kPairWide;
     if (bm) *bm = bi::kPairBM;
-    if (bn) *bn = narrow ? bi::NarrowTile::kBN : bi::WideTile::kBN;
-    if (stages) *stages = narrow ? bi::NarrowTile::kStages : bi::WideTile::kStages;
-    if (bk) *bk = narrow ? bi::NarrowTile::kStageK : bi::WideTile::kStageK;
+    if (bn) *bn = c == bi::kPairNarrow ? bi::NarrowTile::kBN : c == bi::kPairMid ? bi::MidTile::kBN : bi::WideTile::kBN;
+    if (stages)
+        *stages = c == bi::kPairNarrow ? bi::NarrowTile::kStages : c == bi::kPairMid ? bi::MidTile::kStages
+                                                                                      : bi::WideTile::kStages;
+    if (bk)
+        *bk = c == bi::kPairNarrow ? bi::NarrowTile::kStageK : c == bi::kPairMid ? bi::MidTile::kStageK
+                                                                                  : bi::WideTile::kStageK;
     if (mma_k) *mma_k = bi::kMmaK;
 }
 

@@ -9,12 +9,14 @@
 // accumulator, every later step adds in ascending K.  It depends only on K -- not on M,
 // N, the row's position, or which pair computes the tile.  No split-K, no stream-K.
 //
-// Two instantiations exist, and the host picks one from the weight's output width N
-// alone (never from M): the wide tile (BN = 256, SK = 64) and, for N <= 1024, the
-// narrow tile (BN = 128, SK = 128), whose more numerous tiles fill more of the GPU and
-// whose 8 MMAs per stage amortise the issuing thread's per-stage barrier wait and commit.
-// Both run the same 16-wide K steps in the same order, so a row's bits do not depend on
-// which one ran (the tests compare them).
+// Three instantiations exist, and the host picks one from the weight's number of rows
+// alone (never from M; pair_config below): the wide tile (BN = 256, SK = 64), the 192-column
+// tile (BN = 192, SK = 128) where its smaller tiles fill the GPU's CTA pairs in fewer
+// cost-weighted waves, and for weights of up to 1024 rows the narrow tile (BN = 128,
+// SK = 128), whose more numerous tiles fill more of the GPU.  Eight MMAs per 128-deep stage
+// amortise the issuing thread's per-stage barrier wait and commit at the narrower widths.  All
+// run the same 16-wide K steps in the same order, so a row's bits do not depend on which one
+// ran (the tests compare them).
 //
 // Pipeline, per CTA pair:
 //   full[s]   (leader)  armed by the leader's producer with both CTAs' bytes; both
@@ -58,7 +60,8 @@ struct PairTile {
     static constexpr int kSmem = kStages * kStageBytes + kSmemMisc;
     static constexpr uint32_t kTmemCols = pow2_at_least(2 * BN);
 
-    static_assert(BN % 128 == 0 && BN <= 256, "pair tile N must be 128 or 256 ([K, N] B needs 64-column groups)");
+    static_assert(BN % 64 == 0 && BN <= 256, "pair tile N: a multiple of 64 up to 256");
+    static constexpr bool kKNOk = kHalf % 64 == 0;   // [K, N] B is staged in 64-column groups
     static_assert(SK % kBK == 0 && SK >= kBK, "a stage holds whole swizzle atoms");
     static_assert(kStages >= 2 && kStages <= 32, "two to 32 stages (one producer lane per stage at the tail)");
     static_assert(kSmem + 1024 <= 256 * 1024, "shared addresses fit the 14-bit descriptor address field");
@@ -67,8 +70,27 @@ struct PairTile {
 };
 
 using WideTile = PairTile<256, 64>;     // 7 stages of 64 K
+using MidTile = PairTile<192, 128>;     // 4 stages of 128 K ([N, K] weights only)
 using NarrowTile = PairTile<128, 128>;  // 4 stages of 128 K
-constexpr int64_t kNarrowMaxN = 1024;   // output widths up to this use NarrowTile
+constexpr int64_t kNarrowMaxN = 1024;   // weights of up to this many rows use NarrowTile
+
+// Which configuration a weight runs, from its number of rows R alone (N of a plain product, 2F
+// of the fused gate/up product; either way a tile row of 256 outputs needs ceil(R / BN) tiles):
+// NarrowTile up to kNarrowMaxN rows; above that MidTile if, for a reference batch of 1024 rows
+// (4 tile rows) on the B200's 74 CTA pairs, its waves of tiles weighted by the measured cost of a
+// 192-column wave (0.8 of a 256-column one: 20.6 against 25.7 us per LM-head wave) come out
+// fewer than WideTile's, else WideTile.  [K, N] weights, staged in 64-column groups per CTA, take
+// WideTile where the rule says MidTile.  The rule never sees M, and every configuration takes the
+// same 16-wide K steps in ascending order, so the choice does not change a bit of the result.
+enum PairConfig { kPairNarrow = 0, kPairMid = 1, kPairWide = 2 };
+constexpr int64_t kRefPairs = 74, kRefTileRows = 4;
+__host__ inline PairConfig pair_config(int64_t weight_rows, bool nk)
+{
+    if (weight_rows <= kNarrowMaxN) return kPairNarrow;
+    if (!nk) return kPairWide;
+    auto waves = [&](int64_t bn) { return (kRefTileRows * ((weight_rows + bn - 1) / bn) + kRefPairs - 1) / kRefPairs; };
+    return 4 * waves(MidTile::kBN) < 5 * waves(WideTile::kBN) ? kPairMid : kPairWide;
+}
 
 template <int BN, int SK>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)

@@ -44,13 +44,23 @@ def test_status_strings_and_config(lib):
     assert binding.status_string(binding.BI_ERR_TIMEOUT) == "BI_ERR_TIMEOUT"
     assert binding.status_string(99) == "BI_ERR_UNKNOWN"
     wide = binding.bi_gemm_config()
-    assert wide == binding.bi_gemm_config(151936) == binding.bi_gemm_config(1025)
+    # 256-column tiles where 192-column ones would not save a cost-weighted wave at 1024 rows
+    # on 74 CTA pairs: q/o and down (4096 rows: 16 against 22 tiles per tile row, 1 wave against
+    # 2), gate/up unfused (12288: 3 waves against 4 x 0.8), the LM head (151936: 33 against 43)
+    for rows in (151936, 12288, 4096):
+        assert binding.bi_gemm_config(rows) == wide, rows
     assert wide["bm"] == 256 and wide["bn"] == 256 and wide["bk"] == 64 and wide["mma_k"] == 16
+    # 192-column tiles: fused q/k/v (6144: 2 waves against 2 x 0.8), fused gate/up (24576:
+    # 6 against 7 x 0.8), and widths just above the narrow range (1025: 1 against 1 x 0.8)
+    mid = binding.bi_gemm_config(6144)
+    for rows in (24576, 2048, 1025):
+        assert binding.bi_gemm_config(rows) == mid, rows
+    assert mid["bm"] == 256 and mid["bn"] == 192 and mid["bk"] == 128 and mid["mma_k"] == 16
     narrow = binding.bi_gemm_config(1024)
     assert narrow == binding.bi_gemm_config(1)
     assert narrow["bm"] == 256 and narrow["bn"] == 128 and narrow["bk"] == 128 and narrow["mma_k"] == 16
     # every stage fits in the 227 KB a CTA may use, with room for the barriers
-    for cfg in (wide, narrow):
+    for cfg in (wide, mid, narrow):
         assert cfg["stages"] >= 2
         assert cfg["stages"] * (128 + cfg["bn"] // 2) * cfg["bk"] * 2 <= 227 * 1024 - 1536
     assert binding.bi_version() >= 201

@@ -225,11 +225,12 @@ def test_batch_invariance_sweep_wide_and_deep(K, N):
 @pytest.mark.parametrize("layout", ["nk", "kn"])
 @pytest.mark.parametrize("K", [4096, 4104])
 def test_tile_width_does_not_change_bits(K, layout):
-    """Outputs up to 1024 columns wide run the 128-column tile with 128-deep stages, wider ones
-    the 256-column tile with 64-deep stages.  Both take the same 16-wide K steps in ascending
-    order, so the first 1024 columns of a 1280-column product (wide tile) equal, bit for bit,
-    the product with only those 1024 weight rows (narrow tile) -- for plain, bias and fused
-    SiLU * up outputs, at ragged M and K."""
+    """Weights of up to 1024 rows run the 128-column tile with 128-deep stages, wider ones the
+    192-column tile with 128-deep stages ([N, K] storage, where it needs fewer cost-weighted
+    waves) or the 256-column tile with 64-deep stages.  All take the same 16-wide K steps in
+    ascending order, so the first 1024 columns of a 1280-column product equal, bit for bit, the
+    product with only those 1024 weight rows (narrow tile) -- for plain, bias and fused SiLU * up
+    outputs, at ragged M and K."""
     assert bi.bi_gemm_config(1024)["bn"] != bi.bi_gemm_config(1280)["bn"]
     w = weight(250, 1280, K, "nk").to(DEV)
     gate, up = w, weight(251, 1280, K, "nk").to(DEV)
@@ -250,6 +251,24 @@ def test_tile_width_does_not_change_bits(K, layout):
         h_wide = bi.bi_matmul_silu_mul(a, gu_wide, layout)
         h_narrow = bi.bi_matmul_silu_mul(a, gu_narrow, layout)
         assert same_bits(h_wide[:, :1024], h_narrow), f"fused M={M} K={K} {layout}"
+
+
+@pytest.mark.parametrize("K", [4096, 1000])
+def test_mid_tile_matches_wide_tile_bits(K):
+    """A 6144-row weight (the fused q/k/v projection) stored [N, K] runs the 192-column tile; the
+    same weight stored [K, N] runs the 256-column tile.  Plain, bias and fused SiLU * up products
+    agree bit for bit at ragged M, up to 1024 rows (where the tiles' wave counts differ)."""
+    assert bi.bi_gemm_config(6144)["bn"] == 192 and bi.bi_gemm_config(0)["bn"] == 256
+    w = weight(260, 6144, K, "nk").to(DEV)
+    wt = w.t().contiguous()
+    bias = inputs.bias(261, 6144).to(DEV)
+    for M in (1, 77, 300, 1024):
+        a = inputs.rows_normal(262, 0, M, K).to(DEV)
+        assert same_bits(bi.bi_matmul(a, w, "nk"), bi.bi_matmul(a, wt, "kn")), f"matmul M={M} K={K}"
+        assert same_bits(bi.bi_addmm(bias, a, w, "nk"), bi.bi_addmm(bias, a, wt, "kn")), f"addmm M={M} K={K}"
+        assert same_bits(bi.bi_matmul_silu_mul(a, w, "nk"), bi.bi_matmul_silu_mul(a, wt, "kn")), \
+            f"fused M={M} K={K}"
+    assert bi.bi_get_device_status() == bi.BI_OK
 
 
 def test_lm_head_logits_invariance():
