@@ -485,7 +485,10 @@ def run_bi(args):
                               else "gate/up GEMM, then bi_silu_mul",
                        "log_softmax": "bi_log_softmax after the LM head",
                        "l2": "working set ~3 GB > 126 MB L2; no flush",
-                       "gemm_tile": bi.bi_gemm_config()},
+                       # the tile each GEMM of the step runs, from its weight's rows alone
+                       "gemm_tile": {op: bi.bi_gemm_config(rows) for op, rows in
+                                     (("qkv", HIDDEN + 2 * KV), ("o", HIDDEN), ("gate_up", 2 * FFN),
+                                      ("down", HIDDEN), ("lm_head", VOCAB))}},
             "roofline": {"kernel": "bi_matmul LM head launch [%d x 4096] x [4096 x 151936]" % M,
                          "bound": "tensor", "achieved": round(achieved, 1), "peak": peak_tf,
                          "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
