@@ -314,6 +314,9 @@ template <typename T>
 bi_status launch_pair(bi::GemmParams p, const void *A, int64_t lda, const void *B, int64_t ldb, int b_layout,
                       int64_t b_rows, int pairs, cudaStream_t s)
 {
+    // [K, N] weights are staged in 64-column groups per CTA; pair_config never sends them to a
+    // tile whose half-width is not a multiple of 64.
+    if (b_layout == BI_B_KN && !T::kKNOk) return BI_ERR_UNSUPPORTED;
     const int64_t M = p.M, N = p.N, K = p.K;
     p.m_blocks = (int32_t)((M + bi::kPairBM - 1) / bi::kPairBM);
     p.n_blocks = (int32_t)(p.fuse_silu ? (N + T::kHalf - 1) / T::kHalf : (N + T::kBN - 1) / T::kBN);
