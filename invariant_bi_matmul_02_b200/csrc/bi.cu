@@ -394,8 +394,8 @@ bi_status gemm_common(const void *input, int64_t ld_input, int addend_mode, cons
         return launch(bi::gemm_k0_fill_kernel, dim3((unsigned)blocks), dim3(256), 0, s, p);
     }
 
-    // The tile configuration is a function of the output width N alone; every M of a given
-    // weight runs the same one.
+    // The tile configuration is a function of the weight alone (its rows and storage); every M of
+    // a given weight runs the same one.
     switch (bi::pair_config(b_rows, b_layout == BI_B_NK)) {
     case bi::kPairNarrow:
         return launch_pair<bi::NarrowTile>(p, A, lda, B, ldb, b_layout, b_rows, dev->gemm_clusters_narrow, s);
