@@ -22,7 +22,8 @@
  *     function of the weight's shape alone (bi_gemm_config), never of M; every
  *     output element accumulates its K products in fp32, 16 at a time, in
  *     ascending K, in every configuration; no split-K, no stream-K.
- *   - bi_rmsnorm / bi_mean / bi_log_softmax: one thread block per row; the
+ *   - bi_rmsnorm / bi_mean / bi_log_softmax: each row is reduced by one thread
+ *     block (for long-row means, persistent blocks take rows in turn); the
  *     block size and each thread's element set depend only on the row length;
  *     partial results merge through a fixed warp-shuffle tree and a fixed
  *     cross-warp tree.
