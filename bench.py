@@ -556,7 +556,9 @@ def run_reference(args):
 
 SWEEP_M = [1, 2, 3, 4, 8, 16, 32, 64, 77, 128, 256, 512, 1000, 1024, 2048]
 SWEEP_SHAPES = [("q/o", HIDDEN, HIDDEN), ("k/v", HIDDEN, KV), ("gate/up", HIDDEN, FFN),
-                ("down", FFN, HIDDEN), ("lm_head", HIDDEN, VOCAB)]
+                ("down", FFN, HIDDEN), ("lm_head", HIDDEN, VOCAB),
+                # the step's stacked weights, which run the 256x192 tile
+                ("qkv", HIDDEN, HIDDEN + 2 * KV), ("gate+up", HIDDEN, 2 * FFN)]
 
 
 def _timed(fn, flush, reps):
