@@ -265,6 +265,8 @@ def test_mid_tile_matches_wide_tile_bits(K):
     for M in (1, 77, 300, 1024):
         a = inputs.rows_normal(262, 0, M, K).to(DEV)
         assert same_bits(bi.bi_matmul(a, w, "nk"), bi.bi_matmul(a, wt, "kn")), f"matmul M={M} K={K}"
+        assert same_bits(bi.bi_matmul(a, w, "nk", out_dtype=torch.float32),
+                         bi.bi_matmul(a, wt, "kn", out_dtype=torch.float32)), f"matmul fp32 M={M} K={K}"
         assert same_bits(bi.bi_addmm(bias, a, w, "nk"), bi.bi_addmm(bias, a, wt, "kn")), f"addmm M={M} K={K}"
         assert same_bits(bi.bi_matmul_silu_mul(a, w, "nk"), bi.bi_matmul_silu_mul(a, wt, "kn")), \
             f"fused M={M} K={K}"
