@@ -280,7 +280,9 @@ bi_status bi_silu_mul(const void *gu, void *h, int64_t M, int64_t F, void *strea
  *   and B * Hkv * ceil(Lmax / 512) < 2^31 (else BI_ERR_UNSUPPORTED).
  *   scratch  caller-owned device memory, 16-byte aligned, at least
  *            bi_decode_attention_scratch_bytes(B, Hq, D, Lmax) bytes; overwritten (two
- *            launches on `stream`), so overlapping calls need separate scratch.
+ *            launches on `stream`; one when Lmax <= 512, where every sequence is one split
+ *            and the first launch writes out itself), so overlapping calls need separate
+ *            scratch.
  *   q, caches 16-byte aligned; seq_lens 4-byte aligned.
  */
 bi_status bi_decode_attention(const void *q, const void *k_cache, const void *v_cache,

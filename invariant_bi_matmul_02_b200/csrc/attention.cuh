@@ -6,7 +6,9 @@
 // exp(score - max) and the matching weighted sum of value rows.  Launch 2 folds the splits of
 // each (sequence, query head) in ascending split order.  Every reduction is a fixed sequence
 // or a fixed tree, so a sequence's output depends on its own query, cache and length only --
-// not on the batch it is decoded in, its position there, or which CTA computes a split.
+// not on the batch it is decoded in, its position there, or which CTA computes a split.  When
+// Lmax <= kAttnSplit every sequence is one split, and launch 1 does launch 2's fold of it itself
+// (the same operations on the same values), so launch 2 is not made.
 //
 // Launch 1 is a persistent, warp-specialised kernel: one CTA per SM walks the (split, kv head,
 // sequence) work items round-robin.  Its producer warp stages each split as the group's query
@@ -56,6 +58,7 @@ struct AttnParams {
     const int32_t *lens;
     float2 *part_ms;  // [B, Hq, S] (max, sum)
     float *part_acc;  // [B, Hq, S, D]
+    __nv_bfloat16 *out;  // non-null when every sequence is one split (S = 1): launch 1 writes out
     int32_t Hq, Hkv, B;
     int64_t Lmax, S;  // S = splits of Lmax
     float scale;
@@ -506,9 +509,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     float r = so[j * kAttnOStride + ct];
                     for (int w = 1; w < kAttnConsumers; ++w)
                         r = __fadd_rn(r, so[(w * kAttnMaxGroup + j) * kAttnOStride + ct]);
-                    p.part_acc[(bh * p.S + split) * D + ct] = r;
+                    if (p.out != nullptr) {
+                        // Every sequence is one split: the combine launch's fold of one split,
+                        // here, with the same operations on the same values (so the same bits).
+                        float l = red_s[0][j];
+                        for (int w = 1; w < kAttnConsumers; ++w) l = __fadd_rn(l, red_s[w][j]);
+                        const float m = mrun_all[grp][j];
+                        const float wt = __expf(m - m);
+                        p.out[bh * D + ct] = __float2bfloat16_rn(fmaf(r, wt, 0.0f) / fmaf(l, wt, 0.0f));
+                    } else {
+                        p.part_acc[(bh * p.S + split) * D + ct] = r;
+                    }
                 }
-                if (ct == 0) {
+                if (ct == 0 && p.out == nullptr) {
                     float l = red_s[0][j];
                     for (int w = 1; w < kAttnConsumers; ++w) l = __fadd_rn(l, red_s[w][j]);
                     p.part_ms[bh * p.S + split] = make_float2(mrun_all[grp][j], l);

@@ -303,7 +303,7 @@ bi_status launch_attention(int64_t group, dim3 grid, size_t smem, cudaStream_t s
     case 8: st = launch_pdl(bi::decode_attention_split_kernel<8, D>, grid, dim3(bi::kAttnThreads), smem, s, tm_k, tm_v, p); break;
     default: return BI_ERR_UNSUPPORTED;
     }
-    if (st != BI_OK) return st;
+    if (st != BI_OK || p.out != nullptr) return st;  // one split per sequence: launch 1 wrote out
     return launch_pdl(bi::decode_attention_combine_kernel<D>, dim3((unsigned)p.Hq, (unsigned)B), dim3(D), 0, s,
                       static_cast<const float2 *>(p.part_ms), static_cast<const float *>(p.part_acc), seq_lens,
                       static_cast<__nv_bfloat16 *>(out), (int)p.Hq, p.Lmax);
@@ -709,6 +709,8 @@ bi_status bi_decode_attention(const void *q, const void *k_cache, const void *v_
     p.lens = seq_lens;
     p.part_acc = static_cast<float *>(scratch);
     p.part_ms = reinterpret_cast<float2 *>(p.part_acc + (size_t)B * Hq * S * D);
+    // With Lmax <= 512 every sequence is one split, whose fold launch 1 does itself.
+    p.out = S == 1 ? static_cast<__nv_bfloat16 *>(out) : nullptr;
     p.Hq = (int32_t)Hq;
     p.Hkv = (int32_t)Hkv;
     p.B = (int32_t)B;

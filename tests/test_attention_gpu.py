@@ -107,6 +107,24 @@ def test_attention_more_than_eight_splits(d):
     assert bi.bi_get_device_status() == bi.BI_OK
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_attention_one_split_caches_fold_in_launch_one(d):
+    """With Lmax <= 512 every sequence is one split and launch 1 writes the output itself; the same
+    sequences in a cache of Lmax = 600 take the combine launch.  The bits agree, and both match
+    the oracle."""
+    B, Hq, Hkv = 5, 16, 4
+    lens = [500, 1, 129, 256, 417]
+    q, k, v = make(860, B, Hq, Hkv, 600, d=d)
+    sl = torch.tensor(lens, dtype=torch.int32)
+    qd, ld = q.to(DEV), sl.to(DEV)
+    two = bi.bi_decode_attention(qd, k.to(DEV), v.to(DEV), ld)
+    one = bi.bi_decode_attention(qd, k[:, :500].contiguous().to(DEV), v[:, :500].contiguous().to(DEV), ld)
+    assert same_bits(one, two)
+    ref = oracle.decode_attention(bf16_bits_np(q), bf16_bits_np(k), bf16_bits_np(v), sl.numpy(), d ** -0.5)
+    assert_bf16_close(one, ref, f"attention D={d} Lmax=500")
+    assert bi.bi_get_device_status() == bi.BI_OK
+
+
 def test_attention_batch_invariance_over_compositions():
     P, Hq, Hkv, Lmax = 48, 32, 8, 1024
     q, k, v = make(802, P, Hq, Hkv, Lmax)
